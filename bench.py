@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill]
+                    [--impl ours|reference] [--no-extras]
+
+Workload (default "decode"): the 384-expert layer (hidden 4096, top-8,
+expert intermediate 2048, bf16 weights ~19 GB, router logits biased by a
+Zipf(1.1) prior over a seeded expert permutation) run once at each decode
+batch 1, 2, 4, 8, 16, 64; one "step" is the six forwards (95 tokens), each a
+full pass of route -> permute -> expert FFN -> combine. "prefill" runs one
+4096-token chunk per step. Inputs are seeded synthetic tensors already in HBM;
+L2 is flushed (a 256 MiB write) before every forward, outside the timed
+events. Time is device time from CUDA events on the launching stream, summed
+over the K timed steps, max over ranks.
+
+With N > 1 (torchrun) every rank holds its own replica of the layer and
+processes its own tokens: there is no collective in the data path
+("replicas", weak scaling); value = tokens of all ranks / max rank time.
+
+Extras (rank 0, N = 1): the dominant kernel's roofline (gate/up GEMM, HBM bytes
+per launch over its event-timed duration), per-batch and prefill breakdowns,
+the end-to-end number through the public API with host buffers, and the CPU
+oracle timed on a bounded sample as a baseline.
+
+--impl reference times the CPU oracle (the correctness reference of this
+repository; the pages this follows publish no runnable code) on the host
+cores, on the same workload definition, one bounded sample per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (decode B=1..64, prefill 4096) and % of HBM / tensor-pipe roofline"
+H, E, K, I = 4096, 384, 8, 2048
+DECODE_BATCHES = [1, 2, 4, 8, 16, 64]
+ZIPF_S = 1.1
+SEED = 0
+EXPERT_BYTES = 2 * (2 * I * H + H * I)  # bf16 gate/up + down per expert
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ dist --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world, backend):
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=600))
+
+
+def dist_barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def dist_max(world, v, device):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(world, v, device):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- layer --
+
+def build_layer(device, wdtype=0):
+    import mixture_experts_layer_24_b200 as M
+    layer = M.MoeLayer(H, E, K, I, wdtype=wdtype, device=device)
+    keep = []
+    for e in range(E):
+        g, d = synth.expert_weights(e, H, I, seed=SEED, device=device)
+        layer.register(e, g, d)
+        keep.append((g, d))
+    wr = synth.router_weight(E, H, seed=SEED, device=device)
+    bias = synth.zipf_logit_bias(E, ZIPF_S, seed=SEED).to(device)
+    torch.cuda.synchronize(device)
+    return layer, wr, bias, keep
+
+
+def touched_experts(layer, x, wr, bias):
+    idx, _ = layer.route(x, wr, bias)
+    return int(torch.unique(idx).numel())
+
+
+def time_forwards(layer, xs, wr, bias, flush, stream, steps):
+    """Device ms of `steps` passes over xs (one forward each), L2 flushed before each."""
+    pairs = []
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            for x in xs:
+                flush.fill_(1)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                layer.forward(x, wr, bias, stream=stream)
+                b.record(stream)
+                pairs.append((a, b))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in pairs)
+
+
+# --------------------------------------------------------- cpu baseline --
+
+_EXPERT_CACHE = ({}, {})  # host copies of generated experts, reused across samples
+
+def oracle_sample(n_tokens, first_token, threads, budget_s):
+    """Times the CPU oracle on up to n_tokens tokens of the workload (stopping
+    once budget_s is spent); returns (tokens, seconds, description)."""
+    import oracle
+    wr = synth.router_weight(E, H, seed=SEED).numpy()
+    bias = synth.zipf_logit_bias(E, ZIPF_S, seed=SEED).numpy()
+    done, secs = 0, 0.0
+    gu, dn = _EXPERT_CACHE
+    while done < n_tokens and secs < budget_s:
+        x = synth.tokens(1, H, seed=SEED, first_token=first_token + done)
+        xu = oracle.as_u16(x)
+        _, idx, _ = oracle.route(xu, wr, bias, K, threads)
+        for e in np.unique(idx):
+            if int(e) not in gu:
+                g, d = synth.expert_weights(int(e), H, I, seed=SEED)
+                gu[int(e)], dn[int(e)] = oracle.as_u16(g), oracle.as_u16(d)
+        t0 = time.perf_counter()
+        oracle.forward(xu, wr, bias, K, E, gu, dn, threads=threads)
+        secs += time.perf_counter() - t0
+        done += 1
+    return done, secs
+
+
+# ------------------------------------------------------------- reference --
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    threads = os.cpu_count() or 1
+    sample = 1  # tokens per step: one decode token through the full layer
+    for _ in range(args.warmup):
+        oracle_sample(sample, 0, threads, 1e9)
+    tok, secs = 0, 0.0
+    for s in range(args.steps):
+        n, t = oracle_sample(sample, 1000 + s, threads, 1e9)
+        tok += n
+        secs += t
+    v = tok / secs
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "decode_sweep_bf16", "hidden": H, "experts": E, "top_k": K,
+                       "intermediate": I, "zipf_s": ZIPF_S, "parallelism": "replicas"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{sample} decode token(s) per step through the whole layer "
+                                       "(route, permute, 8 experts' SwiGLU FFN, combine), fp32 plain C, OpenMP"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours --
+
+def run_ours(args):
+    import mixture_experts_layer_24_b200 as M
+    from mixture_experts_layer_24_b200 import build as B
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    if rank == 0:
+        B.build()
+    dist_barrier(world)
+    M.lib()
+
+    layer, wr, bias, keep = build_layer(device)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    tok_base = 100000 * rank  # each replica gets its own tokens
+    if args.workload == "decode":
+        batches = DECODE_BATCHES
+        workload = "decode_sweep_bf16"
+    else:
+        batches = [4096]
+        workload = "prefill4096_bf16"
+    xs = [synth.tokens(b, H, seed=SEED, device=device, first_token=tok_base + 1000 * i)
+          for i, b in enumerate(batches)]
+    layer.workspace(16384 if (world == 1 and not args.no_extras) else max(batches))  # no allocation while timing
+    tokens_per_step = sum(batches)
+
+    # warm-up
+    time_forwards(layer, xs, wr, bias, flush, stream, max(args.warmup, 0))
+    status = layer.status()
+    if status:
+        raise SystemExit(f"device status {status} after warm-up")
+
+    clocks = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    launches0 = layer.launches()
+    clocks.start()
+    ms = time_forwards(layer, xs, wr, bias, flush, stream, args.steps)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    launches = layer.launches() - launches0
+    dist_barrier(world)
+    ms_max = dist_max(world, ms, device)
+    total_tokens = dist_sum(world, tokens_per_step * args.steps, device)
+    value = total_tokens / (ms_max / 1000.0)
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload, "hidden": H, "experts": E, "top_k": K, "intermediate": I,
+                       "batches": batches, "zipf_s": ZIPF_S, "weights": "bf16, seeded N(0,0.02)",
+                       "l2": "flushed (256 MiB write) before every forward, outside the timed events",
+                       "parallelism": f"replicas x{world}"},
+            "gpu_launches": launches, "gpu_launches_per_step": launches / max(args.steps, 1), "clocks": clk}
+
+    if world == 1 and not args.no_extras:
+        line.update(extras(layer, wr, bias, xs, batches, flush, stream, args, device))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    layer.close()
+    return 0
+
+
+def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
+    import mixture_experts_layer_24_b200 as M
+    hbm, tf_burst, tf_sust, peak_kind = peaks()
+    out = {}
+    # --- per-kernel device time (events inside the library, same stream) ---
+    steps = max(3, args.steps)
+    M.moe_profile_enable(layer.ctx, True)
+    M.moe_profile_read(layer.ctx, reset=True)
+    time_forwards(layer, xs, wr, bias, flush, stream, steps)
+    prof = M.moe_profile_read(layer.ctx, reset=True)
+    M.moe_profile_enable(layer.ctx, False)
+    touched = [touched_experts(layer, x, wr, bias) for x in xs]
+    gu_bytes = sum(t * 2 * I * H * 2 + b * K * H * 2 + b * K * I * 2 for t, b in zip(touched, batches))
+    dn_bytes = sum(t * H * I * 2 + b * K * I * 2 + b * K * H * 4 for t, b in zip(touched, batches))
+    gu_ms, gu_n = prof["gate_up"]
+    dn_ms, dn_n = prof["down"]
+    per_launch_bytes = gu_bytes / len(batches)
+    achieved = (gu_bytes * steps) / (gu_ms / 1000.0) / 1e9
+    out["roofline"] = {"bound": "hbm", "kernel": "ffn gate/up GEMM + SwiGLU (tcgen05)", "achieved": achieved,
+                       "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                       "peak_source": f"{peak_kind} hbm_gbs",
+                       "algorithmic_bytes_per_launch": per_launch_bytes,
+                       "avg_launch_us": 1000.0 * gu_ms / max(gu_n, 1)}
+    total_ms = sum(v[0] for v in prof.values())
+    out["kernels"] = {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps,
+                          "share": v[0] / total_ms if total_ms else 0.0} for k, v in prof.items() if v[1]}
+    out["kernels"]["down"]["achieved_GBps"] = (dn_bytes * steps) / (dn_ms / 1000.0) / 1e9 if dn_ms else None
+
+    # --- per-batch / prefill breakdown ---
+    br = {}
+    for b, x, t in zip(batches, xs, touched):
+        ms = time_forwards(layer, [x], wr, bias, flush, stream, 5) / 5
+        nbytes = t * EXPERT_BYTES + E * H * 4 + b * H * 2 * 2
+        br[f"B{b}"] = {"us_per_layer": 1000 * ms, "tokens_per_s": b / (ms / 1000), "touched_experts": t,
+                       "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+    if args.workload == "decode":
+        for T in (512, 4096, 16384):
+            x = synth.tokens(T, H, seed=SEED, device=device, first_token=500000)
+            reps = 3 if T < 16384 else 2
+            ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
+            t = touched_experts(layer, x, wr, bias)
+            flops = 2.0 * T * K * (2 * I * H + H * I) + 2.0 * T * E * H
+            nbytes = t * EXPERT_BYTES + E * H * 4 + T * H * 4
+            br[f"prefill{T}"] = {"us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
+                                 "tensor_frac": (flops / (ms / 1000) / 1e12) / tf_burst,
+                                 "hbm_frac": (nbytes / (ms / 1000) / 1e9) / hbm,
+                                 "combined_roofline_frac": max(flops / (tf_burst * 1e12), nbytes / (hbm * 1e9)) /
+                                 (ms / 1000)}
+    out["breakdown"] = br
+
+    # --- end to end through the public API, host buffers ---
+    hx = [x.cpu().pin_memory() for x in xs]
+    hout = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
+    dx = [torch.empty_like(x) for x in xs]
+    pairs = []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            for i in range(len(xs)):
+                flush.fill_(1)
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                dx[i].copy_(hx[i], non_blocking=True)
+                y = layer.forward(dx[i], wr, bias, stream=stream)
+                hout[i].copy_(y, non_blocking=True)
+                b.record(stream)
+                pairs.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in pairs)
+    io = sum(b * H * 2 for b in batches)
+    out["e2e"] = {"value": sum(batches) * args.steps / (e2e_ms / 1000), "unit": "tokens/s",
+                  "h2d_bytes_per_step": io, "d2h_bytes_per_step": io}
+
+    # --- CPU oracle on a bounded sample ---
+    threads = os.cpu_count() or 1
+    n, secs = oracle_sample(64, 2000, threads, 15.0)
+    out["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                           "sample": f"{n} decode tokens (batch 1 each) through the whole layer, "
+                                     f"{secs:.1f} s of CPU time, fp32 plain C oracle with OpenMP"}
+    if layer.status():
+        out["device_status"] = layer.status()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--no-extras", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,317 @@
+"""ctypes binding of libmoe (include/moe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors (or None) where the C side takes pointers, and passes the current torch
+CUDA stream unless one is given. Nothing is computed in Python; if
+``libmoe.so`` cannot be loaded the first call raises -- there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_BF16 = 0
+MOE_FP8_E4M3_B128 = 1
+MOE_LOC_HBM = 0
+MOE_LOC_HOST_PINNED = 1
+MOE_DEV_BAD_EXPERT = 1
+MOE_DEV_NO_SLOT = 2
+MOE_DEV_TIMEOUT = 4
+
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+                4: "MOE_ERR_SLOT", 5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_OOM"}
+
+EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route", "moe_permute",
+           "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_e4m3", "moe_slots_create",
+           "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
+           "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
+           "moe_profile_enable", "moe_profile_read"]
+
+PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("intermediate", ctypes.c_int), ("wdtype", ctypes.c_int), ("flags", ctypes.c_int)]
+
+
+class MoeSlotsStats(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_int64), ("cold_staged", ctypes.c_int64), ("bytes_staged", ctypes.c_int64),
+                ("last_cold", ctypes.c_int32), ("last_touched", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Loads libmoe.so (built by ``python -m mixture_experts_layer_24_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with python -m mixture_experts_layer_24_b200.build")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, S, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "moe_ctx_create": ([ctypes.POINTER(P), ctypes.POINTER(MoeConfig)], S),
+        "moe_ctx_destroy": ([P], S),
+        "moe_workspace_size": ([P, I], Z),
+        "moe_route": ([P, P, P, P, I, P, P, P, Z, P], S),
+        "moe_permute": ([P, P, I, P, P, P, P, P, P, Z, P], S),
+        "moe_expert_ffn": ([P, P, P, P, P, P, P, I, P, P, Z, P], S),
+        "moe_combine": ([P, P, P, I, P, P], S),
+        "moe_forward": ([P, P, P, P, P, I, P, P, Z, P], S),
+        "moe_quantize_e4m3": ([P, I, I, I, P, P, P], S),
+        "moe_slots_create": ([ctypes.POINTER(P), P, I], S),
+        "moe_slots_destroy": ([P], S),
+        "moe_slots_register": ([P, I, P, P, P, P, I], S),
+        "moe_slots_query": ([P, I, ctypes.POINTER(I), ctypes.POINTER(I)], S),
+        "moe_slots_stats": ([P, ctypes.POINTER(MoeSlotsStats)], S),
+        "moe_plan_hot_set": ([P, I, I, P], S),
+        "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_int32), I], S),
+        "moe_last_error": ([], ctypes.c_char_p),
+        "moe_launch_count": ([P], ctypes.c_int64),
+        "moe_profile_enable": ([P, I], S),
+        "moe_profile_read": ([P, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], S),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise MoeError(st, where, lib().moe_last_error().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None  # the call will fail its own checks; there is no CPU path
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------ C entry points --
+
+def moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16):
+    cfg = MoeConfig(hidden, n_experts, top_k, intermediate, wdtype, 0)
+    h = ctypes.c_void_p()
+    _check(lib().moe_ctx_create(ctypes.byref(h), ctypes.byref(cfg)), "moe_ctx_create")
+    return h
+
+
+def moe_ctx_destroy(ctx):
+    _check(lib().moe_ctx_destroy(ctx), "moe_ctx_destroy")
+
+
+def moe_workspace_size(ctx, T: int) -> int:
+    return int(lib().moe_workspace_size(ctx, T))
+
+
+def moe_route(ctx, x, w_router, logit_bias, T, topk_idx, topk_w, ws, stream=None):
+    _check(lib().moe_route(ctx, _p(x), _p(w_router), _p(logit_bias), T, _p(topk_idx), _p(topk_w), _p(ws),
+                           _nbytes(ws), _s(stream)), "moe_route")
+
+
+def moe_permute(ctx, topk_idx, T, counts, offsets, perm_src, perm_k, inv, ws, stream=None):
+    _check(lib().moe_permute(ctx, _p(topk_idx), T, _p(counts), _p(offsets), _p(perm_src), _p(perm_k), _p(inv),
+                             _p(ws), _nbytes(ws), _s(stream)), "moe_permute")
+
+
+def moe_expert_ffn(ctx, slots, x, perm_src, perm_k, offsets, topk_w, T, y_pair, ws, stream=None):
+    _check(lib().moe_expert_ffn(ctx, slots, _p(x), _p(perm_src), _p(perm_k), _p(offsets), _p(topk_w), T,
+                                _p(y_pair), _p(ws), _nbytes(ws), _s(stream)), "moe_expert_ffn")
+
+
+def moe_combine(ctx, y_pair, inv, T, out, stream=None):
+    _check(lib().moe_combine(ctx, _p(y_pair), _p(inv), T, _p(out), _s(stream)), "moe_combine")
+
+
+def moe_forward(ctx, slots, x, w_router, logit_bias, T, out, ws, stream=None):
+    _check(lib().moe_forward(ctx, slots, _p(x), _p(w_router), _p(logit_bias), T, _p(out), _p(ws), _nbytes(ws),
+                             _s(stream)), "moe_forward")
+
+
+def moe_quantize_e4m3(src, rows, cols, block_rows, q, scales, stream=None):
+    _check(lib().moe_quantize_e4m3(_p(src), rows, cols, block_rows, _p(q), _p(scales), _s(stream)),
+           "moe_quantize_e4m3")
+
+
+def moe_slots_create(ctx, n_spare_slots: int):
+    h = ctypes.c_void_p()
+    _check(lib().moe_slots_create(ctypes.byref(h), ctx, n_spare_slots), "moe_slots_create")
+    return h
+
+
+def moe_slots_destroy(slots):
+    _check(lib().moe_slots_destroy(slots), "moe_slots_destroy")
+
+
+def moe_slots_register(slots, expert, w_gu, w_dn, s_gu=None, s_dn=None, location=MOE_LOC_HBM):
+    _check(lib().moe_slots_register(slots, expert, _p(w_gu), _p(w_dn), _p(s_gu), _p(s_dn), location),
+           "moe_slots_register")
+
+
+def moe_slots_query(slots, expert):
+    loc, slot = ctypes.c_int(), ctypes.c_int()
+    _check(lib().moe_slots_query(slots, expert, ctypes.byref(loc), ctypes.byref(slot)), "moe_slots_query")
+    return loc.value, slot.value
+
+
+def moe_slots_stats(slots) -> dict:
+    st = MoeSlotsStats()
+    _check(lib().moe_slots_stats(slots, ctypes.byref(st)), "moe_slots_stats")
+    return {k: getattr(st, k) for k, _ in MoeSlotsStats._fields_}
+
+
+def moe_plan_hot_set(hist, n_hot: int):
+    """hist: int64 CPU tensor [E] -> int32 CPU tensor [n_hot]."""
+    hist = hist.to(torch.int64).contiguous()
+    hot = torch.empty(n_hot, dtype=torch.int32)
+    _check(lib().moe_plan_hot_set(_p(hist), hist.numel(), n_hot, _p(hot)), "moe_plan_hot_set")
+    return hot
+
+
+def moe_get_device_status(ctx, reset: bool = True) -> int:
+    v = ctypes.c_int32()
+    _check(lib().moe_get_device_status(ctx, ctypes.byref(v), int(reset)), "moe_get_device_status")
+    return v.value
+
+
+def moe_launch_count(ctx) -> int:
+    return int(lib().moe_launch_count(ctx))
+
+
+def moe_profile_enable(ctx, enable: bool = True):
+    _check(lib().moe_profile_enable(ctx, int(enable)), "moe_profile_enable")
+
+
+def moe_profile_read(ctx, reset: bool = True) -> dict:
+    """{kind: (total_ms, launches)} for every kernel kind (synchronises)."""
+    out = {}
+    for k, name in enumerate(PROF_KINDS):
+        ms, n = ctypes.c_double(), ctypes.c_int64()
+        _check(lib().moe_profile_read(ctx, k, ctypes.byref(ms), ctypes.byref(n), int(reset)), "moe_profile_read")
+        out[name] = (ms.value, n.value)
+    return out
+
+
+# ------------------------------------------------------------- convenience --
+
+class MoeLayer:
+    """One MoE layer: a context, its slot table and a reusable workspace.
+
+    Registered weight tensors are kept referenced here because the library
+    borrows them."""
+
+    def __init__(self, hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16, n_spare_slots=0, device=None):
+        self.H, self.E, self.K, self.I, self.wdtype = hidden, n_experts, top_k, intermediate, wdtype
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        with torch.cuda.device(self.device):
+            self.ctx = moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype)
+            self.slots = moe_slots_create(self.ctx, n_spare_slots)
+        self._keep = {}
+        self._ws = None
+
+    def register(self, e, w_gu, w_dn, s_gu=None, s_dn=None, location=MOE_LOC_HBM):
+        self._keep[e] = (w_gu, w_dn, s_gu, s_dn)
+        moe_slots_register(self.slots, e, w_gu, w_dn, s_gu, s_dn, location)
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = moe_workspace_size(self.ctx, T)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
+        return self._ws
+
+    def forward(self, x, w_router, logit_bias=None, out=None, stream=None):
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        moe_forward(self.ctx, self.slots, x, w_router, logit_bias, T, out, self.workspace(T), stream)
+        return out
+
+    def route(self, x, w_router, logit_bias=None, stream=None):
+        T = x.shape[0]
+        idx = torch.empty((T, self.K), dtype=torch.int32, device=self.device)
+        w = torch.empty((T, self.K), dtype=torch.float32, device=self.device)
+        moe_route(self.ctx, x, w_router, logit_bias, T, idx, w, self.workspace(T), stream)
+        return idx, w
+
+    def permute(self, topk_idx, stream=None):
+        T = topk_idx.shape[0]
+        P = T * self.K
+        d = self.device
+        counts = torch.empty(self.E, dtype=torch.int32, device=d)
+        offsets = torch.empty(self.E + 1, dtype=torch.int32, device=d)
+        perm_src = torch.empty(P, dtype=torch.int32, device=d)
+        perm_k = torch.empty(P, dtype=torch.int32, device=d)
+        inv = torch.empty((T, self.K), dtype=torch.int32, device=d)
+        moe_permute(self.ctx, topk_idx, T, counts, offsets, perm_src, perm_k, inv, self.workspace(T), stream)
+        return counts, offsets, perm_src, perm_k, inv
+
+    def expert_ffn(self, x, perm_src, perm_k, offsets, topk_w, stream=None):
+        T = x.shape[0]
+        y = torch.empty((T * self.K, self.H), dtype=torch.float32, device=self.device)
+        moe_expert_ffn(self.ctx, self.slots, x, perm_src, perm_k, offsets, topk_w, T, y, self.workspace(T), stream)
+        return y
+
+    def combine(self, y_pair, inv, stream=None):
+        T = inv.shape[0]
+        out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        moe_combine(self.ctx, y_pair, inv, T, out, stream)
+        return out
+
+    def status(self, reset=True) -> int:
+        return moe_get_device_status(self.ctx, reset)
+
+    def stats(self) -> dict:
+        return moe_slots_stats(self.slots)
+
+    def launches(self) -> int:
+        return moe_launch_count(self.ctx)
+
+    def close(self):
+        if getattr(self, "slots", None) is not None:
+            moe_slots_destroy(self.slots)
+            self.slots = None
+        if getattr(self, "ctx", None) is not None:
+            moe_ctx_destroy(self.ctx)
+            self.ctx = None
+        self._keep = {}
+        self._ws = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

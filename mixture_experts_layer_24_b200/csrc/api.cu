@@ -1,0 +1,760 @@
+// api.cu -- the C ABI of libmoe: context, workspace layout, the expert-slot
+// table (residency + cold-expert staging), and the entry points that chain
+// the kernels of route.cu, permute.cu, ffn_gemm.cu, quant.cu and combine.cu.
+//
+// Residency follows the "hotsplit" recipes wiki (Home page): hot experts stay
+// in HBM, cold experts live in pinned host memory and are brought in on
+// demand. Here a cold expert routed to by the batch is copied by the copy
+// engine into a spare HBM slot and computed by the SAME kernels, tile shapes
+// and K order as a resident one, so outputs are bit-identical to the
+// all-resident run (vLLM-Moet, topairepos.com page, hybrid results table,
+// row "identity").
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status_t fail(moe_status_t st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+#define MOE_CUDA(call)                                                                              \
+  do {                                                                                              \
+    cudaError_t err_ = (call);                                                                      \
+    if (err_ != cudaSuccess)                                                                        \
+      return fail(MOE_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(err_));             \
+  } while (0)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+struct moe_ctx {
+  moe_config_t cfg;
+  int device = 0;
+  int* d_status = nullptr;
+  int host_status = 0;
+  EncodeTiledFn encode = nullptr;
+  std::atomic<int64_t> launches{0};
+  // kernel timing (moe_profile_*)
+  bool prof_on = false;
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> prof_pending;
+  std::vector<cudaEvent_t> ev_pool;
+  double prof_ms[MOE_PROF_KINDS] = {};
+  int64_t prof_n[MOE_PROF_KINDS] = {};
+  std::mutex prof_mu;
+
+  cudaEvent_t take_event() {
+    if (!ev_pool.empty()) {
+      cudaEvent_t e = ev_pool.back();
+      ev_pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+
+namespace {
+// Counts one kernel launch and, when timing is on, brackets it with events on
+// the launching stream.
+struct Prof {
+  moe_ctx* c;
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  Prof(moe_ctx* c_, int kind_, cudaStream_t s_) : c(c_), kind(kind_), s(s_) {
+    if (c->prof_on) {
+      std::lock_guard<std::mutex> g(c->prof_mu);
+      a = c->take_event();
+      cudaEventRecord(a, s);
+    }
+  }
+  ~Prof() {
+    c->launches.fetch_add(1, std::memory_order_relaxed);
+    if (a) {
+      std::lock_guard<std::mutex> g(c->prof_mu);
+      cudaEvent_t b = c->take_event();
+      cudaEventRecord(b, s);
+      c->prof_pending.push_back({kind, a, b});
+    }
+  }
+};
+}  // namespace
+
+struct moe_slots {
+  moe_ctx* ctx = nullptr;
+  int E = 0, n_spare = 0;
+  std::vector<int> loc;  // -1 unregistered, MOE_LOC_*
+  std::vector<const void*> gu, dn;
+  std::vector<const float*> sgu, sdn;
+  std::vector<MapEntry> h_maps;  // [E + n_spare]
+  std::vector<int32_t> h_map_of; // [E]
+  MapEntry* d_maps = nullptr;
+  int32_t* d_map_of = nullptr;
+  uint8_t* spare = nullptr;
+  size_t off_dn = 0, off_sgu = 0, off_sdn = 0, slot_bytes = 0;
+  size_t bytes_gu = 0, bytes_dn = 0, bytes_sgu = 0, bytes_sdn = 0;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t ev_ready[2] = {nullptr, nullptr};
+  cudaEvent_t ev_free[2] = {nullptr, nullptr};
+  int32_t* h_pinned = nullptr;  // offsets readback + list staging
+  size_t h_pinned_ints = 0;
+  int n_host = 0;
+  moe_slots_stats_t stats{};
+  std::mutex mu;
+};
+
+namespace {
+
+// ----------------------------------------------------------- workspace --
+
+struct WsLayout {
+  size_t logits, rank, chunk_counts, topk_idx, topk_w, counts, offsets, perm_src, perm_k, inv;
+  size_t list_expert, list_map, nt_prefix, x_perm, x_scale, h, hq, h_scale, y_pair, total;
+};
+
+WsLayout ws_layout(const moe_config_t& c, int T) {
+  WsLayout L{};
+  const size_t P = (size_t)T * c.top_k, E = c.n_experts, H = c.hidden, I = c.intermediate;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += align256(bytes);
+    return at;
+  };
+  L.logits = take((size_t)T * E * 4);
+  L.rank = take(P * 4);
+  L.chunk_counts = take(64 * E * 4);
+  L.topk_idx = take(P * 4);
+  L.topk_w = take(P * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.perm_src = take(P * 4);
+  L.perm_k = take(P * 4);
+  L.inv = take(P * 4);
+  L.list_expert = take((2 * E + 64) * 4);
+  L.list_map = take((2 * E + 64) * 4);
+  L.nt_prefix = take((2 * E + 64) * 4);
+  L.x_perm = take(P * H * (fp8 ? 1 : 2));
+  L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
+  L.h = take(P * I * 2);
+  L.hq = take(fp8 ? P * I : 0);
+  L.h_scale = take(fp8 ? P * (I / 128) * 4 : 0);
+  L.y_pair = take(P * H * 4);
+  L.total = o;
+  return L;
+}
+
+moe_status_t check_cfg(const moe_config_t& c) {
+  if (c.hidden <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.intermediate <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "config sizes must be positive");
+  if (c.wdtype != MOE_BF16 && c.wdtype != MOE_FP8_E4M3_B128) return fail(MOE_ERR_INVALID_ARG, "unknown wdtype");
+  if (c.flags != 0) return fail(MOE_ERR_INVALID_ARG, "flags must be 0");
+  if (c.hidden % 128 || c.intermediate % 128) return fail(MOE_ERR_UNSUPPORTED, "H and I must be multiples of 128");
+  if (c.hidden > 8192 || c.intermediate > 8192) return fail(MOE_ERR_UNSUPPORTED, "H and I must be <= 8192");
+  if (c.top_k > 32 || c.top_k > c.n_experts || c.n_experts > 1024)
+    return fail(MOE_ERR_UNSUPPORTED, "need 1 <= K <= 32 and K <= E <= 1024");
+  return MOE_OK;
+}
+
+moe_status_t check_T(const moe_ctx_t* ctx, int T) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (T > 65536) return fail(MOE_ERR_UNSUPPORTED, "T must be <= 65536");
+  (void)ctx;
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_ctx_t* ctx, int T, const void* ws, size_t ws_bytes) {
+  const WsLayout L = ws_layout(ctx->cfg, T);
+  if (!ws && L.total > 0) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (ws_bytes < L.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small (see moe_workspace_size)");
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t encode_2d(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, bool fp8, uint64_t inner, uint64_t rows,
+                       uint32_t box_rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = ctx->encode(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                 const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
+moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void* dn, const float* sgu,
+                        const float* sdn) {
+  const moe_config_t& c = ctx->cfg;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  std::memset(me, 0, sizeof(*me));
+  moe_status_t st = encode_2d(ctx, &me->gu, gu, fp8, c.hidden, 2ull * c.intermediate, 128);
+  if (st != MOE_OK) return st;
+  st = encode_2d(ctx, &me->dn, dn, fp8, c.intermediate, c.hidden, 128);
+  if (st != MOE_OK) return st;
+  me->s_gu = sgu;
+  me->s_dn = sdn;
+  return MOE_OK;
+}
+
+
+// Runs the two GEMMs (and, for FP8, the quantiser of h between them) for one
+// expert list whose arrays live in the workspace at list offset `lo`.
+moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void* ws, int T, int bn,
+                       const int32_t* perm_src, const int32_t* perm_k, const int32_t* offsets, const float* topk_w,
+                       float* y_pair, const int32_t* list_expert, const int32_t* list_map, const int32_t* nt_prefix,
+                       int L, int max_ntiles, cudaStream_t s) {
+  const moe_config_t& c = ctx->cfg;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  const int P = T * c.top_k;
+  CUtensorMap xmap, hmap;
+  moe_status_t st = encode_2d(ctx, &xmap, at<void>(ws, W.x_perm), fp8, c.hidden, P, bn);
+  if (st != MOE_OK) return st;
+  st = encode_2d(ctx, &hmap, fp8 ? at<void>(ws, W.hq) : at<void>(ws, W.h), fp8, c.intermediate, P, bn);
+  if (st != MOE_OK) return st;
+  GemmArgs a{};
+  a.maps = sl->d_maps;
+  a.list_expert = list_expert;
+  a.list_map = list_map;
+  a.nt_prefix = nt_prefix;
+  a.offsets = offsets;
+  a.L = L;
+  a.H = c.hidden;
+  a.I = c.intermediate;
+  a.K = c.top_k;
+  a.h_out = at<void>(ws, W.h);
+  a.y_out = y_pair;
+  a.topk_w = topk_w;
+  a.perm_src = perm_src;
+  a.perm_k = perm_k;
+  a.status = ctx->d_status;
+  a.act_scale = fp8 ? at<float>(ws, W.x_scale) : nullptr;
+  {
+    Prof p(ctx, MOE_PROF_GATE_UP, s);
+    MOE_CUDA(launch_ffn_gemm(kGateUp, c.wdtype, bn, xmap, a, (c.intermediate / 128) * max_ntiles, s));
+  }
+  if (fp8) {
+    {
+      Prof p(ctx, MOE_PROF_QUANT, s);
+      MOE_CUDA(launch_quant_rows_e4m3_count(at<void>(ws, W.h), offsets, c.n_experts, P, c.intermediate,
+                                            at<uint8_t>(ws, W.hq), at<float>(ws, W.h_scale), s));
+    }
+    a.act_scale = at<float>(ws, W.h_scale);
+  }
+  {
+    Prof p(ctx, MOE_PROF_DOWN, s);
+    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, a, (c.hidden / 128) * max_ntiles, s));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+// =================================================================== ABI ==
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+moe_status_t moe_ctx_create(moe_ctx_t** out, const moe_config_t* cfg) {
+  if (!out || !cfg) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  *out = nullptr;
+  moe_status_t st = check_cfg(*cfg);
+  if (st != MOE_OK) return st;
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  MOE_CUDA(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10) return fail(MOE_ERR_UNSUPPORTED, "libmoe needs an sm_100 (B200-class) device");
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  MOE_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+  if (!fn || q != cudaDriverEntryPointSuccess) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled not found");
+  moe_ctx_t* ctx = new moe_ctx_t();
+  ctx->cfg = *cfg;
+  ctx->device = dev;
+  ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess) {
+    delete ctx;
+    return fail(MOE_ERR_OOM, "cudaMalloc of the status word failed");
+  }
+  cudaMemset(ctx->d_status, 0, sizeof(int));
+  cudaDeviceSynchronize();
+  *out = ctx;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_destroy(moe_ctx_t* ctx) {
+  if (!ctx) return MOE_OK;
+  for (auto& r : ctx->prof_pending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : ctx->ev_pool) cudaEventDestroy(e);
+  cudaFree(ctx->d_status);
+  delete ctx;
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_ctx_t* ctx, int T) {
+  if (!ctx || T < 0) return 0;
+  return ws_layout(ctx->cfg, T).total;
+}
+
+int64_t moe_launch_count(const moe_ctx_t* ctx) { return ctx ? ctx->launches.load() : 0; }
+
+moe_status_t moe_profile_enable(moe_ctx_t* ctx, int enable) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  std::lock_guard<std::mutex> g(ctx->prof_mu);
+  ctx->prof_on = enable != 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_read(moe_ctx_t* ctx, int kind, double* total_ms, int64_t* launches, int reset) {
+  if (!ctx || !total_ms || !launches) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  if (kind < 0 || kind >= MOE_PROF_KINDS) return fail(MOE_ERR_INVALID_ARG, "unknown kernel kind");
+  std::lock_guard<std::mutex> g(ctx->prof_mu);
+  for (auto& r : ctx->prof_pending) {
+    MOE_CUDA(cudaEventSynchronize(r.b));
+    float ms = 0.f;
+    MOE_CUDA(cudaEventElapsedTime(&ms, r.a, r.b));
+    ctx->prof_ms[r.kind] += ms;
+    ctx->prof_n[r.kind] += 1;
+    ctx->ev_pool.push_back(r.a);
+    ctx->ev_pool.push_back(r.b);
+  }
+  ctx->prof_pending.clear();
+  *total_ms = ctx->prof_ms[kind];
+  *launches = ctx->prof_n[kind];
+  if (reset) {
+    ctx->prof_ms[kind] = 0.0;
+    ctx->prof_n[kind] = 0;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(moe_ctx_t* ctx, int32_t* status, int reset) {
+  if (!ctx || !status) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  MOE_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  MOE_CUDA(cudaMemcpy(&v, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost));
+  *status = v | ctx->host_status;
+  if (reset) {
+    MOE_CUDA(cudaMemset(ctx->d_status, 0, sizeof(int)));
+    ctx->host_status = 0;
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_route(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  const moe_config_t& c = ctx->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout W = ws_layout(c, T);
+  float* logits = at<float>(ws, W.logits);
+  {
+    Prof p(ctx, MOE_PROF_ROUTER, s);
+    MOE_CUDA(launch_router_logits(x, w_router, logit_bias, T, c.hidden, c.n_experts, logits, s));
+  }
+  {
+    Prof p(ctx, MOE_PROF_TOPK, s);
+    MOE_CUDA(launch_topk(logits, T, c.n_experts, c.top_k, topk_idx, topk_w, ctx->d_status, s));
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_permute(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
+                         int32_t* perm_src, int32_t* perm_k, int32_t* inv, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if (T > 0 && (!topk_idx || !perm_src || !perm_k || !inv)) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  const moe_config_t& c = ctx->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout W = ws_layout(c, T);
+  const int chunk = permute_chunk_tokens(T, c.top_k);
+  const int n_chunks = T > 0 ? (T + chunk - 1) / chunk : 0;
+  int32_t* cc = at<int32_t>(ws, W.chunk_counts);
+  if (T > 0) {
+    Prof p(ctx, MOE_PROF_PERMUTE, s);
+    MOE_CUDA(launch_permute_rank(topk_idx, T, c.top_k, c.n_experts, chunk, at<int32_t>(ws, W.rank), cc,
+                                 ctx->d_status, s));
+  }
+  {
+    Prof p(ctx, MOE_PROF_PERMUTE, s);
+    MOE_CUDA(launch_permute_scan(cc, n_chunks, c.n_experts, counts, offsets, s));
+  }
+  if (T > 0) {
+    Prof p(ctx, MOE_PROF_PERMUTE, s);
+    MOE_CUDA(launch_permute_scatter(topk_idx, at<int32_t>(ws, W.rank), cc, offsets, T, c.top_k, c.n_experts, chunk,
+                                    perm_src, perm_k, inv, s));
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
+                            const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T,
+                            float* y_pair, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ctx || !sl) return fail(MOE_ERR_INVALID_ARG, "NULL context or slot table");
+  if (sl->ctx != ctx) return fail(MOE_ERR_SLOT, "slot table belongs to another context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !perm_src || !perm_k || !offsets || !topk_w || !y_pair) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  const moe_config_t& c = ctx->cfg;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout W = ws_layout(c, T);
+  const int E = c.n_experts, P = T * c.top_k;
+  const int bn = ffn_block_n(T, c.wdtype);
+  std::lock_guard<std::mutex> lock(sl->mu);
+  sl->stats.calls++;
+
+  int32_t* le = at<int32_t>(ws, W.list_expert);
+  int32_t* lm = at<int32_t>(ws, W.list_map);
+  int32_t* np = at<int32_t>(ws, W.nt_prefix);
+  const int ntile_bound = (P + bn - 1) / bn + std::min(E, P);
+
+  // activation rows in sorted-pair order (quantised for FP8)
+  {
+  Prof pg(ctx, MOE_PROF_GATHER, s);
+  if (fp8) {
+    MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                      at<float>(ws, W.x_scale), s));
+  } else {
+    MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s));
+  }
+  }
+
+  if (sl->n_host == 0) {
+    {
+      Prof p(ctx, MOE_PROF_PERMUTE, s);
+      MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s));
+    }
+    sl->stats.last_cold = 0;
+    sl->stats.last_touched = -1;
+    return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
+                     s);
+  }
+
+  // ---- hot/cold: read the per-expert offsets back, stage the routed cold experts
+  int32_t* hoff = sl->h_pinned;
+  MOE_CUDA(cudaMemcpyAsync(hoff, offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaStreamSynchronize(s));
+  std::vector<int> hot, cold;
+  int touched = 0;
+  for (int e = 0; e < E; ++e) {
+    const int cnt = hoff[e + 1] - hoff[e];
+    if (cnt <= 0) continue;
+    ++touched;
+    if (sl->loc[e] == MOE_LOC_HBM) hot.push_back(e);
+    else if (sl->loc[e] == MOE_LOC_HOST_PINNED) cold.push_back(e);
+    else ctx->host_status |= MOE_DEV_NO_SLOT;
+  }
+  sl->stats.last_touched = touched;
+  sl->stats.last_cold = (int32_t)cold.size();
+  if (!cold.empty() && sl->n_spare <= 0) return fail(MOE_ERR_SLOT, "cold experts routed but no spare slots");
+  const bool two_buf = (int)cold.size() > sl->n_spare && sl->n_spare >= 2;
+  const int bsz = two_buf ? sl->n_spare / 2 : sl->n_spare;
+
+  // list staging: [hot][batch0][batch1]...; each list: experts, maps, prefix (L+1)
+  struct ListRef {
+    int L, e_off, p_off;
+  };
+  std::vector<ListRef> lists;
+  int32_t* stage = sl->h_pinned + (E + 1);
+  std::vector<int32_t> he, hm, hp;
+  auto add_list = [&](const std::vector<int>& ex, int map_base) {
+    ListRef r{(int)ex.size(), (int)he.size(), (int)hp.size()};
+    int acc = 0;
+    for (size_t i = 0; i < ex.size(); ++i) {
+      const int e = ex[i];
+      he.push_back(e);
+      hm.push_back(map_base < 0 ? e : map_base + (int)i);
+      hp.push_back(acc);
+      acc += (hoff[e + 1] - hoff[e] + bn - 1) / bn;
+    }
+    hp.push_back(acc);
+    lists.push_back(r);
+  };
+  if (!hot.empty()) add_list(hot, -1);
+  const int n_batches = cold.empty() ? 0 : ((int)cold.size() + bsz - 1) / bsz;
+  for (int b = 0; b < n_batches; ++b) {
+    std::vector<int> part(cold.begin() + (size_t)b * bsz,
+                          cold.begin() + std::min(cold.size(), (size_t)(b + 1) * bsz));
+    add_list(part, E + (two_buf ? (b & 1) * bsz : 0));
+  }
+  const size_t n_e = he.size(), n_p = hp.size();
+  std::memcpy(stage, he.data(), n_e * 4);
+  std::memcpy(stage + n_e, hm.data(), n_e * 4);
+  std::memcpy(stage + 2 * n_e, hp.data(), n_p * 4);
+  // three device arrays from one staging block (lists region holds 2E+64 ints each)
+  MOE_CUDA(cudaMemcpyAsync(le, stage, n_e * 4, cudaMemcpyHostToDevice, s));
+  MOE_CUDA(cudaMemcpyAsync(lm, stage + n_e, n_e * 4, cudaMemcpyHostToDevice, s));
+  MOE_CUDA(cudaMemcpyAsync(np, stage + 2 * n_e, n_p * 4, cudaMemcpyHostToDevice, s));
+
+  size_t li = 0;
+  if (!hot.empty()) {
+    const ListRef& r = lists[li++];
+    st = run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le + r.e_off, lm + r.e_off,
+                   np + r.p_off, r.L, ntile_bound, s);
+    if (st != MOE_OK) return st;
+  }
+  for (int b = 0; b < n_batches; ++b) {
+    const ListRef& r = lists[li++];
+    const int buf = two_buf ? (b & 1) : 0;
+    MOE_CUDA(cudaStreamWaitEvent(sl->copy_stream, sl->ev_free[buf], 0));
+    for (int i = 0; i < r.L; ++i) {
+      const int e = he[r.e_off + i];
+      uint8_t* slot = sl->spare + (size_t)(buf * bsz + i) * sl->slot_bytes;
+      MOE_CUDA(cudaMemcpyAsync(slot, sl->gu[e], sl->bytes_gu, cudaMemcpyHostToDevice, sl->copy_stream));
+      MOE_CUDA(cudaMemcpyAsync(slot + sl->off_dn, sl->dn[e], sl->bytes_dn, cudaMemcpyHostToDevice, sl->copy_stream));
+      if (fp8) {
+        MOE_CUDA(cudaMemcpyAsync(slot + sl->off_sgu, sl->sgu[e], sl->bytes_sgu, cudaMemcpyHostToDevice,
+                                 sl->copy_stream));
+        MOE_CUDA(cudaMemcpyAsync(slot + sl->off_sdn, sl->sdn[e], sl->bytes_sdn, cudaMemcpyHostToDevice,
+                                 sl->copy_stream));
+      }
+      sl->stats.cold_staged++;
+      sl->stats.bytes_staged += (int64_t)(sl->bytes_gu + sl->bytes_dn + (fp8 ? sl->bytes_sgu + sl->bytes_sdn : 0));
+    }
+    MOE_CUDA(cudaEventRecord(sl->ev_ready[buf], sl->copy_stream));
+    MOE_CUDA(cudaStreamWaitEvent(s, sl->ev_ready[buf], 0));
+    st = run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le + r.e_off, lm + r.e_off,
+                   np + r.p_off, r.L, ntile_bound, s);
+    if (st != MOE_OK) return st;
+    MOE_CUDA(cudaEventRecord(sl->ev_free[buf], s));
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_combine(moe_ctx_t* ctx, const float* y_pair, const int32_t* inv, int T, void* out,
+                         moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y_pair || !inv || !out) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  Prof p(ctx, MOE_PROF_COMBINE, static_cast<cudaStream_t>(stream));
+  MOE_CUDA(launch_combine(y_pair, inv, T, ctx->cfg.top_k, ctx->cfg.hidden, out, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const float* w_router,
+                         const float* logit_bias, int T, void* out, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  if (!ctx || !sl) return fail(MOE_ERR_INVALID_ARG, "NULL context or slot table");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !out) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout W = ws_layout(ctx->cfg, T);
+  int32_t* idx = at<int32_t>(ws, W.topk_idx);
+  float* w = at<float>(ws, W.topk_w);
+  if ((st = moe_route(ctx, x, w_router, logit_bias, T, idx, w, ws, ws_bytes, stream)) != MOE_OK) return st;
+  int32_t* counts = at<int32_t>(ws, W.counts);
+  int32_t* offsets = at<int32_t>(ws, W.offsets);
+  int32_t* ps = at<int32_t>(ws, W.perm_src);
+  int32_t* pk = at<int32_t>(ws, W.perm_k);
+  int32_t* inv = at<int32_t>(ws, W.inv);
+  if ((st = moe_permute(ctx, idx, T, counts, offsets, ps, pk, inv, ws, ws_bytes, stream)) != MOE_OK) return st;
+  float* y = at<float>(ws, W.y_pair);
+  if ((st = moe_expert_ffn(ctx, sl, x, ps, pk, offsets, w, T, y, ws, ws_bytes, stream)) != MOE_OK) return st;
+  return moe_combine(ctx, y, inv, T, out, stream);
+}
+
+moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
+                               moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 128) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0 and cols % 128 == 0");
+  if (block_rows != 1 && block_rows != 128) return fail(MOE_ERR_UNSUPPORTED, "block_rows must be 1 or 128");
+  if (rows == 0) return MOE_OK;
+  if (!src || !q || !scales) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  MOE_CUDA(launch_quant_e4m3(src, rows, cols, block_rows, q, scales, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+// ----------------------------------------------------------------- slots --
+
+moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
+  if (!out || !ctx || n_spare < 0) return fail(MOE_ERR_INVALID_ARG, "bad argument");
+  *out = nullptr;
+  const moe_config_t& c = ctx->cfg;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  moe_slots_t* sl = new moe_slots_t();
+  sl->ctx = ctx;
+  sl->E = c.n_experts;
+  sl->n_spare = n_spare;
+  sl->loc.assign(sl->E, -1);
+  sl->gu.assign(sl->E, nullptr);
+  sl->dn.assign(sl->E, nullptr);
+  sl->sgu.assign(sl->E, nullptr);
+  sl->sdn.assign(sl->E, nullptr);
+  sl->h_maps.assign(sl->E + n_spare, MapEntry{});
+  sl->h_map_of.assign(sl->E, -1);
+  const size_t esz = fp8 ? 1 : 2;
+  sl->bytes_gu = 2ull * c.intermediate * c.hidden * esz;
+  sl->bytes_dn = (size_t)c.hidden * c.intermediate * esz;
+  sl->bytes_sgu = fp8 ? (2ull * c.intermediate / 128) * (c.hidden / 128) * 4 : 0;
+  sl->bytes_sdn = fp8 ? ((size_t)c.hidden / 128) * (c.intermediate / 128) * 4 : 0;
+  sl->off_dn = align256(sl->bytes_gu);
+  sl->off_sgu = sl->off_dn + align256(sl->bytes_dn);
+  sl->off_sdn = sl->off_sgu + align256(sl->bytes_sgu);
+  sl->slot_bytes = sl->off_sdn + align256(sl->bytes_sdn);
+  auto cleanup = [&](moe_status_t st, const std::string& msg) {
+    moe_slots_destroy(sl);
+    return fail(st, msg);
+  };
+  if (cudaMalloc(&sl->d_maps, sizeof(MapEntry) * (sl->E + n_spare)) != cudaSuccess)
+    return cleanup(MOE_ERR_OOM, "cudaMalloc of the map table failed");
+  if (cudaMalloc(&sl->d_map_of, sizeof(int32_t) * sl->E) != cudaSuccess)
+    return cleanup(MOE_ERR_OOM, "cudaMalloc of the slot index failed");
+  if (n_spare > 0 && cudaMalloc(&sl->spare, sl->slot_bytes * n_spare) != cudaSuccess)
+    return cleanup(MOE_ERR_OOM, "cudaMalloc of the spare slots failed");
+  sl->h_pinned_ints = (size_t)(sl->E + 1) + 4 * (size_t)sl->E + 256;
+  if (cudaHostAlloc(&sl->h_pinned, sizeof(int32_t) * sl->h_pinned_ints, cudaHostAllocDefault) != cudaSuccess)
+    return cleanup(MOE_ERR_OOM, "cudaHostAlloc failed");
+  if (cudaStreamCreateWithFlags(&sl->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return cleanup(MOE_ERR_CUDA, "cudaStreamCreate failed");
+  for (int i = 0; i < 2; ++i) {
+    if (cudaEventCreateWithFlags(&sl->ev_ready[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sl->ev_free[i], cudaEventDisableTiming) != cudaSuccess)
+      return cleanup(MOE_ERR_CUDA, "cudaEventCreate failed");
+  }
+  for (int i = 0; i < n_spare; ++i) {
+    uint8_t* slot = sl->spare + (size_t)i * sl->slot_bytes;
+    moe_status_t st = make_entry(ctx, &sl->h_maps[sl->E + i], slot, slot + sl->off_dn,
+                                 fp8 ? reinterpret_cast<const float*>(slot + sl->off_sgu) : nullptr,
+                                 fp8 ? reinterpret_cast<const float*>(slot + sl->off_sdn) : nullptr);
+    if (st != MOE_OK) {
+      std::string m = g_last_error;
+      return cleanup(st, m);
+    }
+  }
+  if (cudaMemcpy(sl->d_maps, sl->h_maps.data(), sizeof(MapEntry) * (sl->E + n_spare), cudaMemcpyHostToDevice) !=
+          cudaSuccess ||
+      cudaMemcpy(sl->d_map_of, sl->h_map_of.data(), sizeof(int32_t) * sl->E, cudaMemcpyHostToDevice) != cudaSuccess)
+    return cleanup(MOE_ERR_CUDA, "cudaMemcpy of the slot table failed");
+  *out = sl;
+  return MOE_OK;
+}
+
+moe_status_t moe_slots_destroy(moe_slots_t* sl) {
+  if (!sl) return MOE_OK;
+  if (sl->copy_stream) cudaStreamSynchronize(sl->copy_stream);
+  for (int i = 0; i < 2; ++i) {
+    if (sl->ev_ready[i]) cudaEventDestroy(sl->ev_ready[i]);
+    if (sl->ev_free[i]) cudaEventDestroy(sl->ev_free[i]);
+  }
+  if (sl->copy_stream) cudaStreamDestroy(sl->copy_stream);
+  if (sl->h_pinned) cudaFreeHost(sl->h_pinned);
+  if (sl->spare) cudaFree(sl->spare);
+  if (sl->d_maps) cudaFree(sl->d_maps);
+  if (sl->d_map_of) cudaFree(sl->d_map_of);
+  delete sl;
+  return MOE_OK;
+}
+
+moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, const void* w_dn, const float* s_gu,
+                                const float* s_dn, int location) {
+  if (!sl) return fail(MOE_ERR_INVALID_ARG, "NULL slot table");
+  if (expert < 0 || expert >= sl->E) return fail(MOE_ERR_SLOT, "expert index out of range");
+  if (!w_gu || !w_dn) return fail(MOE_ERR_INVALID_ARG, "NULL weights");
+  const bool fp8 = sl->ctx->cfg.wdtype == MOE_FP8_E4M3_B128;
+  if (fp8 != (s_gu != nullptr) || fp8 != (s_dn != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "scales must be given for FP8 weights and only for them");
+  if (location != MOE_LOC_HBM && location != MOE_LOC_HOST_PINNED) return fail(MOE_ERR_INVALID_ARG, "bad location");
+  std::lock_guard<std::mutex> lock(sl->mu);
+  if (location == MOE_LOC_HBM) {
+    if ((reinterpret_cast<uintptr_t>(w_gu) | reinterpret_cast<uintptr_t>(w_dn)) % 16)
+      return fail(MOE_ERR_INVALID_ARG, "device weights must be 16-byte aligned");
+    MapEntry me;
+    moe_status_t st = make_entry(sl->ctx, &me, w_gu, w_dn, s_gu, s_dn);
+    if (st != MOE_OK) return st;
+    sl->h_maps[expert] = me;
+    sl->h_map_of[expert] = expert;
+    MOE_CUDA(cudaMemcpy(sl->d_maps + expert, &me, sizeof(MapEntry), cudaMemcpyHostToDevice));
+  } else {
+    sl->h_map_of[expert] = -1;
+  }
+  const int prev = sl->loc[expert];
+  if (prev == MOE_LOC_HOST_PINNED) sl->n_host--;
+  if (location == MOE_LOC_HOST_PINNED) sl->n_host++;
+  sl->loc[expert] = location;
+  sl->gu[expert] = w_gu;
+  sl->dn[expert] = w_dn;
+  sl->sgu[expert] = s_gu;
+  sl->sdn[expert] = s_dn;
+  MOE_CUDA(cudaMemcpy(sl->d_map_of + expert, &sl->h_map_of[expert], sizeof(int32_t), cudaMemcpyHostToDevice));
+  return MOE_OK;
+}
+
+moe_status_t moe_slots_query(const moe_slots_t* sl, int expert, int* location, int* slot) {
+  if (!sl || !location || !slot) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  if (expert < 0 || expert >= sl->E) return fail(MOE_ERR_SLOT, "expert index out of range");
+  *location = sl->loc[expert];
+  *slot = sl->loc[expert] == MOE_LOC_HBM ? sl->h_map_of[expert] : -1;
+  return MOE_OK;
+}
+
+moe_status_t moe_slots_stats(const moe_slots_t* sl, moe_slots_stats_t* stats) {
+  if (!sl || !stats) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  *stats = sl->stats;
+  return MOE_OK;
+}
+
+moe_status_t moe_plan_hot_set(const int64_t* hist, int E, int n_hot, int32_t* hot) {
+  if (!hist || !hot || E <= 0 || n_hot < 0 || n_hot > E) return fail(MOE_ERR_INVALID_ARG, "bad argument");
+  std::vector<int> order(E);
+  for (int e = 0; e < E; ++e) order[e] = e;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return hist[a] > hist[b]; });
+  for (int i = 0; i < n_hot; ++i) hot[i] = order[i];
+  return MOE_OK;
+}
+
+}  // extern "C"

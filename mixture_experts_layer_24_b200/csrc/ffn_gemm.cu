@@ -1,0 +1,522 @@
+// ffn_gemm.cu -- grouped expert FFN on the 5th-generation tensor cores.
+//
+// Per routed pair (token t, expert e, slot k) of a DeepSeek-class MoE layer
+// (vLLM-Moet, topairepos.com page, model table: the "b12x" MoE GPU kernels of
+// the hybrid's step breakdown are this step):
+//   gate/up:  g = Wg[e] x_t, u = Wu[e] x_t (fp32 accumulate), h = bf16(silu(g) * u)
+//   down:     y_pair = w[t,k] * (Wd[e] h)                     (fp32)
+//
+// Orientation ("swap AB"): the expert's weight rows are the MMA M operand
+// (128 rows per CTA) and the pairs routed to the expert are the N operand
+// (BN columns), both K-major in shared memory with the 128-byte swizzle and
+// fed by TMA. Each CTA computes one (expert, 128-row tile, BN-pair tile) over
+// the full K, K-blocks in increasing order, with no split-K, so the fp32 sum
+// behind any output element is the same whatever BN, the batch or the set of
+// resident experts; only the columns a CTA owns differ.
+//
+// Warp roles (one CTA per tile):
+//   warps 0..3 (bf16) / 0..7 (fp8): epilogue (TMEM -> registers -> global)
+//   next warp: TMA producer (one elected lane)
+//   last warp: TMEM allocator + MMA issuer (one elected lane)
+// Gate/up CTAs hold two accumulators, gate rows [j, j+128) and up rows
+// [I+j, I+j+128), so one thread owns g and u of the same (j, pair) and SwiGLU
+// happens in the epilogue without any exchange.
+//
+// FP8 (e4m3 operands, kind::f8f6f4): one stage is one 128-wide K block, which
+// is one scale block of both operands. The MMA writes each block's partial
+// sum P_kb into one of two TMEM buffers; the epilogue promotes it in fp32
+// registers, acc = fmaf(P_kb, s_act[pair, kb] * s_w[rowblock, kb], acc),
+// K blocks in increasing order.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr uint32_t kABytes = 128 * 128;  // one 128-row x 128-byte operand tile
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
+  return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
+}
+
+template <int MODE, int BN>
+struct Bf16Cfg {
+  static constexpr int NA = MODE == kGateUp ? 2 : 1;
+  static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(NA * BN);
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+};
+
+template <int MODE, int BN>
+struct Fp8Cfg {
+  static constexpr int NA = MODE == kGateUp ? 2 : 1;
+  static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;
+  static constexpr int kMaxKB = 64;  // K / 128 <= 64 (K <= 8192)
+  static constexpr uint32_t kScaleBytes = BN * kMaxKB * 4;
+  static constexpr int kStagesRaw = (200 * 1024 - (int)kScaleBytes) / (int)kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(2 * NA * BN);
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kScaleBytes + 256;
+};
+
+struct TileInfo {
+  int e, mapi, mt, row0, nvalid;
+};
+
+// Finds this CTA's (expert, M tile, N tile); false if the CTA has no tile.
+__device__ __forceinline__ bool decode_tile(const GemmArgs& a, int m_tiles, int bn, TileInfo& ti) {
+  const int total = a.nt_prefix[a.L] * m_tiles;
+  const int tile = blockIdx.x;
+  if (tile >= total) return false;
+  // once any CTA has given up on a wait, the rest of the grid stands down
+  if (a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT)) return false;
+  int lo = 0, hi = a.L;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.nt_prefix[mid] * m_tiles <= tile) lo = mid;
+    else hi = mid;
+  }
+  const int nti = a.nt_prefix[lo + 1] - a.nt_prefix[lo];
+  const int local = tile - a.nt_prefix[lo] * m_tiles;
+  const int mt = local / nti, nt = local - mt * nti;
+  ti.e = a.list_expert[lo];
+  ti.mapi = a.list_map[lo];
+  ti.mt = mt;
+  ti.row0 = a.offsets[ti.e] + nt * bn;
+  ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
+  return true;
+}
+
+__device__ __forceinline__ void tensormap_acquire(const void* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
+}
+
+// ====================================================================== bf16
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ CUtensorMap act_map,
+                                                          const GemmArgs a) {
+  using C = Bf16Cfg<MODE, BN>;
+  constexpr int NA = C::NA, S = C::kStages;
+  constexpr uint32_t STAGE = C::kStageBytes;
+  constexpr uint32_t IDESC = instr_desc(128, BN, 1u);
+
+  TileInfo ti;
+  const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
+  if (!decode_tile(a, m_tiles, BN, ti)) return;
+  const int KB = (MODE == kGateUp ? a.H : a.I) / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + S * STAGE;  // full[S], empty[S], accf
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (S + s); };
+  const uint32_t accf = bars + 16u * S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + 16 * S + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(accf, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  const MapEntry* me = a.maps + ti.mapi;
+  const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
+
+  if (warp == 4) {
+    if (lane == 0) {
+      tensormap_acquire(wmap);
+      tma_prefetch_map(wmap);
+      tma_prefetch_map(&act_map);
+      const uint64_t pol_w = l2_policy_evict_first();
+      int kb = 0;
+      for (; kb < KB; ++kb) {
+        const int s = kb % S;
+        if (kb >= S && !mbar_wait(empty(s), ((kb / S) - 1) & 1)) {
+          *abort_flag = 1;
+          flag_status(a.status, MOE_DEV_TIMEOUT);
+          break;
+        }
+        if (*abort_flag) break;
+        const uint32_t st = base + s * STAGE;
+        mbar_arrive_expect_tx(full(s), STAGE);
+        tma_load_2d_hint(st, wmap, full(s), kb * 64, ti.mt * 128, pol_w);
+        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 64, a.I + ti.mt * 128, pol_w);
+        tma_load_2d(st + NA * kABytes, &act_map, full(s), kb * 64, ti.row0);
+      }
+      // every load this thread issued has landed before the CTA may exit
+      for (int j = kb - S < 0 ? 0 : kb - S; j < kb; ++j) mbar_wait(full(j % S), (j / S) & 1);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S;
+        if (!mbar_wait(full(s), (kb / S) & 1)) {
+          *abort_flag = 1;
+          flag_status(a.status, MOE_DEV_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = base + s * STAGE;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
+          const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
+          tc_mma_bf16(tmem, sw128_kmajor_desc(st + k * 32), bdesc, IDESC, acc);
+          if (MODE == kGateUp) tc_mma_bf16(tmem + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, IDESC, acc);
+        }
+        tc_commit(empty(s));
+      }
+      tc_commit(accf);
+    }
+  } else {
+    const bool ok = mbar_wait(accf, 0);
+    if (!ok) flag_status(a.status, MOE_DEV_TIMEOUT);
+    tc_fence_after();
+    __syncwarp();
+    if (ok && !*abort_flag) {
+      const int r = warp * 32 + lane;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+      if (MODE == kGateUp) {
+        const int j = ti.mt * 128 + r;
+        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          if (c >= ti.nvalid) break;
+          uint32_t g[16], u[16];
+          tmem_ld16(tl + c, g);
+          tmem_ld16(tl + BN + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            if (c + q < ti.nvalid) {
+              const float gv = __uint_as_float(g[q]);
+              const float uv = __uint_as_float(u[q]);
+              const float hv = gv / (1.0f + expf(-gv)) * uv;
+              hout[(size_t)(ti.row0 + c + q) * a.I + j] = __float2bfloat16_rn(hv);
+            }
+          }
+        }
+      } else {
+        const int o = ti.mt * 128 + r;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          if (c >= ti.nvalid) break;
+          uint32_t v[16];
+          tmem_ld16(tl + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            if (c + q < ti.nvalid) {
+              const int p = ti.row0 + c + q;
+              const float wgt = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
+              a.y_out[(size_t)p * a.H + o] = wgt * __uint_as_float(v[q]);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ======================================================================= fp8
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__ CUtensorMap act_map,
+                                                         const GemmArgs a) {
+  using C = Fp8Cfg<MODE, BN>;
+  constexpr int NA = C::NA, S = C::kStages;
+  constexpr uint32_t STAGE = C::kStageBytes;
+  constexpr uint32_t IDESC = instr_desc(128, BN, 0u);
+  constexpr int HALF = BN / 2;  // columns per epilogue warp
+  constexpr int NCH = HALF >= 16 ? HALF / 16 : 1;
+  constexpr int CW = HALF >= 16 ? 16 : HALF;  // columns per TMEM load
+
+  TileInfo ti;
+  const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
+  if (!decode_tile(a, m_tiles, BN, ti)) return;
+  const int KD = MODE == kGateUp ? a.H : a.I;  // reduction length
+  const int KB = KD / 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  float* s_act = reinterpret_cast<float*>(gbase + S * STAGE);  // [BN][KB]
+  const uint32_t bars = base + S * STAGE + C::kScaleBytes;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (S + s); };
+  auto pfull = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto pempty = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + C::kScaleBytes + 8 * (2 * S + 4));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(pfull(b), 1);
+      mbar_init(pempty(b), 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // activation scales of this tile's pairs -> shared memory
+  for (int i = threadIdx.x; i < BN * KB; i += blockDim.x) {
+    const int n = i / KB, kb = i - n * KB;
+    s_act[i] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  const MapEntry* me = a.maps + ti.mapi;
+  const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
+
+  if (warp == 8) {
+    if (lane == 0) {
+      tensormap_acquire(wmap);
+      tma_prefetch_map(wmap);
+      tma_prefetch_map(&act_map);
+      const uint64_t pol_w = l2_policy_evict_first();
+      int kb = 0;
+      for (; kb < KB; ++kb) {
+        const int s = kb % S;
+        if (kb >= S && !mbar_wait(empty(s), ((kb / S) - 1) & 1)) {
+          *abort_flag = 1;
+          flag_status(a.status, MOE_DEV_TIMEOUT);
+          break;
+        }
+        if (*abort_flag) break;
+        const uint32_t st = base + s * STAGE;
+        mbar_arrive_expect_tx(full(s), STAGE);
+        tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
+        tma_load_2d(st + NA * kABytes, &act_map, full(s), kb * 128, ti.row0);
+      }
+      for (int j = kb - S < 0 ? 0 : kb - S; j < kb; ++j) mbar_wait(full(j % S), (j / S) & 1);
+    }
+  } else if (warp == 9) {
+    if (lane == 0) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % S, b = kb & 1;
+        bool ok = mbar_wait(full(s), (kb / S) & 1);
+        if (ok && kb >= 2) ok = mbar_wait(pempty(b), ((kb >> 1) - 1) & 1);
+        if (!ok) {
+          *abort_flag = 1;
+          flag_status(a.status, MOE_DEV_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = base + s * STAGE;
+        const uint32_t d = tmem + static_cast<uint32_t>(b * NA * BN);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
+          const uint32_t acc = k != 0 ? 1u : 0u;
+          tc_mma_e4m3(d, sw128_kmajor_desc(st + k * 32), bdesc, IDESC, acc);
+          if (MODE == kGateUp) tc_mma_e4m3(d + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, IDESC, acc);
+        }
+        tc_commit(empty(s));
+        tc_commit(pfull(b));
+      }
+    }
+  } else {
+    // epilogue: warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int c0 = hf * HALF;
+    const int wrow_g = ti.mt;                // weight row block of this lane's gate (or down) row
+    const int wrow_u = a.I / 128 + ti.mt;    // weight row block of the up row
+    const float* sw = MODE == kGateUp ? me->s_gu : me->s_dn;
+    float accg[HALF], accu[MODE == kGateUp ? HALF : 1];
+#pragma unroll
+    for (int i = 0; i < HALF; ++i) accg[i] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < (MODE == kGateUp ? HALF : 1); ++i) accu[i] = 0.0f;
+    bool ok = true;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int b = kb & 1;
+      ok = mbar_wait(pfull(b), (kb >> 1) & 1);
+      if (!ok || *abort_flag) break;
+      tc_fence_after();
+      const float swg = __ldg(sw + (size_t)wrow_g * KB + kb);
+      const float swu = MODE == kGateUp ? __ldg(sw + (size_t)wrow_u * KB + kb) : 0.0f;
+      const uint32_t pb = tl + static_cast<uint32_t>(b * NA * BN + c0);
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        uint32_t pg[16], pu[16];
+        if (CW == 16) {
+          tmem_ld16(pb + ch * 16, pg);
+          if (MODE == kGateUp) tmem_ld16(pb + BN + ch * 16, pu);
+        } else {
+          // HALF == 8: load 16 columns starting at c0 (the other half is ignored)
+          tmem_ld16(tl + static_cast<uint32_t>(b * NA * BN), pg);
+          if (MODE == kGateUp) tmem_ld16(tl + static_cast<uint32_t>(b * NA * BN + BN), pu);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < CW; ++q) {
+          const int col = ch * 16 + q;             // index within this warp's half
+          const int n = c0 + col;                  // tile column
+          const int src = CW == 16 ? q : c0 + q;   // register holding column n
+          const float sa = s_act[n * KB + kb];
+          accg[col] = fmaf(__uint_as_float(pg[src]), sa * swg, accg[col]);
+          if (MODE == kGateUp) accu[col] = fmaf(__uint_as_float(pu[src]), sa * swu, accu[col]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pempty(b));
+    }
+    if (!ok) flag_status(a.status, MOE_DEV_TIMEOUT);
+    if (ok && !*abort_flag) {
+      if (MODE == kGateUp) {
+        const int j = ti.mt * 128 + r;
+        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
+#pragma unroll
+        for (int col = 0; col < HALF; ++col) {
+          const int n = c0 + col;
+          if (n < ti.nvalid) {
+            const float gv = accg[col], uv = accu[col];
+            const float hv = gv / (1.0f + expf(-gv)) * uv;
+            hout[(size_t)(ti.row0 + n) * a.I + j] = __float2bfloat16_rn(hv);
+          }
+        }
+      } else {
+        const int o = ti.mt * 128 + r;
+#pragma unroll
+        for (int col = 0; col < HALF; ++col) {
+          const int n = c0 + col;
+          if (n < ti.nvalid) {
+            const int p = ti.row0 + n;
+            const float wgt = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
+            a.y_out[(size_t)p * a.H + o] = wgt * accg[col];
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ==================================================================== launch
+
+template <typename Kern>
+static cudaError_t launch_kernel(Kern kern, size_t smem, int threads, int grid, const CUtensorMap& map,
+                                 const GemmArgs& a, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, threads, smem, s>>>(map, a);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const GemmArgs& a, int grid,
+                               cudaStream_t s) {
+  if (wdtype == MOE_BF16) {
+    switch (bn) {
+      case 16: return launch_kernel(ffn_bf16_kernel<MODE, 16>, Bf16Cfg<MODE, 16>::kSmem, 192, grid, map, a, s);
+      case 32: return launch_kernel(ffn_bf16_kernel<MODE, 32>, Bf16Cfg<MODE, 32>::kSmem, 192, grid, map, a, s);
+      case 64: return launch_kernel(ffn_bf16_kernel<MODE, 64>, Bf16Cfg<MODE, 64>::kSmem, 192, grid, map, a, s);
+      case 128: return launch_kernel(ffn_bf16_kernel<MODE, 128>, Bf16Cfg<MODE, 128>::kSmem, 192, grid, map, a, s);
+      case 256: return launch_kernel(ffn_bf16_kernel<MODE, 256>, Bf16Cfg<MODE, 256>::kSmem, 192, grid, map, a, s);
+    }
+  } else {
+    switch (bn) {
+      case 16: return launch_kernel(ffn_fp8_kernel<MODE, 16>, Fp8Cfg<MODE, 16>::kSmem, 320, grid, map, a, s);
+      case 32: return launch_kernel(ffn_fp8_kernel<MODE, 32>, Fp8Cfg<MODE, 32>::kSmem, 320, grid, map, a, s);
+      case 64: return launch_kernel(ffn_fp8_kernel<MODE, 64>, Fp8Cfg<MODE, 64>::kSmem, 320, grid, map, a, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+int ffn_block_n(int T, int wdtype) {
+  int bn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256;
+  if (wdtype == MOE_FP8_E4M3_B128 && bn > 64) bn = 64;
+  return bn;
+}
+
+size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
+  if (wdtype == MOE_BF16) {
+    if (mode == kGateUp) {
+      switch (bn) {
+        case 16: return Bf16Cfg<kGateUp, 16>::kSmem;
+        case 32: return Bf16Cfg<kGateUp, 32>::kSmem;
+        case 64: return Bf16Cfg<kGateUp, 64>::kSmem;
+        case 128: return Bf16Cfg<kGateUp, 128>::kSmem;
+        case 256: return Bf16Cfg<kGateUp, 256>::kSmem;
+      }
+    } else {
+      switch (bn) {
+        case 16: return Bf16Cfg<kDown, 16>::kSmem;
+        case 32: return Bf16Cfg<kDown, 32>::kSmem;
+        case 64: return Bf16Cfg<kDown, 64>::kSmem;
+        case 128: return Bf16Cfg<kDown, 128>::kSmem;
+        case 256: return Bf16Cfg<kDown, 256>::kSmem;
+      }
+    }
+  } else {
+    if (mode == kGateUp) {
+      switch (bn) {
+        case 16: return Fp8Cfg<kGateUp, 16>::kSmem;
+        case 32: return Fp8Cfg<kGateUp, 32>::kSmem;
+        case 64: return Fp8Cfg<kGateUp, 64>::kSmem;
+      }
+    } else {
+      switch (bn) {
+        case 16: return Fp8Cfg<kDown, 16>::kSmem;
+        case 32: return Fp8Cfg<kDown, 32>::kSmem;
+        case 64: return Fp8Cfg<kDown, 64>::kSmem;
+      }
+    }
+  }
+  return 0;
+}
+
+cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const GemmArgs& a,
+                            int max_tiles, cudaStream_t s) {
+  if (mode == kGateUp) return launch_mode<kGateUp>(wdtype, bn, act_map, a, max_tiles, s);
+  return launch_mode<kDown>(wdtype, bn, act_map, a, max_tiles, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,223 @@
+// permute.cu -- token-to-expert permutation ("compact MoE calls": the pairs
+// routed to one expert made contiguous; vLLM-Moet, topairepos.com page, hybrid
+// results table, row "identity") as a deterministic counting sort by
+// (expert asc, token asc), plus the FFN tile plan and the row gathers that
+// feed the grouped GEMMs.
+//
+//   rank:    one warp per chunk of tokens; the warp walks its chunk in token
+//            order, 32/K tokens per step, and gives each pair its rank among
+//            the chunk's earlier pairs of the same expert (match_any for
+//            pairs of one step, a per-warp shared counter across steps).
+//   scan:    one CTA: per-expert exclusive scan over chunks, counts, and the
+//            exclusive scan over experts (offsets).
+//   scatter: p = offsets[e] + chunk_base[c][e] + rank.
+// Integer arithmetic only: the result is bit-exact and run-to-run identical.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr int kRankWarps = 4;
+constexpr int kMaxChunks = 64;
+
+int permute_chunk_tokens(int T, int K) {
+  const int tps = 32 / K;
+  int c = (T + kMaxChunks - 1) / kMaxChunks;
+  if (c < 32) c = 32;
+  c = (c + tps - 1) / tps * tps;
+  return c;
+}
+
+__global__ void __launch_bounds__(kRankWarps * 32) permute_rank_kernel(const int32_t* __restrict__ idx, int T,
+                                                                        int K, int E, int chunk,
+                                                                        int32_t* __restrict__ rank,
+                                                                        int32_t* __restrict__ chunk_counts,
+                                                                        int* status) {
+  extern __shared__ int32_t cnt_all[];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * kRankWarps + w;
+  const int n_chunks = (T + chunk - 1) / chunk;
+  if (c >= n_chunks) return;  // warp-uniform
+  int32_t* cnt = cnt_all + (size_t)w * E;
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  __syncwarp();
+  const int tps = 32 / K;
+  const int tl = lane / K, k = lane - tl * K;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const int t_end = min(T, (c + 1) * chunk);
+  for (int t0 = c * chunk; t0 < t_end; t0 += tps) {
+    const int t = t0 + tl;
+    const bool active = tl < tps && t < t_end;
+    const int e = active ? idx[(size_t)t * K + k] : -1;
+    const bool valid = active && e >= 0 && e < E;
+    if (active && !valid) flag_status(status, MOE_DEV_BAD_EXPERT);
+    const int key = valid ? e : E + lane;  // invalid lanes match nobody
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    int r = -1;
+    if (valid) r = cnt[e] + __popc(peers & lt_mask);
+    __syncwarp();
+    if (valid && (peers >> lane) == 1u) cnt[e] += __popc(peers);  // highest peer lane updates
+    __syncwarp();
+    if (active) rank[(size_t)t * K + k] = r;
+  }
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) chunk_counts[(size_t)c * E + e] = cnt[e];
+}
+
+cudaError_t launch_permute_rank(const int32_t* idx, int T, int K, int E, int chunk, int32_t* rank,
+                                int32_t* chunk_counts, int* status, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  const int n_chunks = (T + chunk - 1) / chunk;
+  const int blocks = (n_chunks + kRankWarps - 1) / kRankWarps;
+  const size_t smem = sizeof(int32_t) * (size_t)E * kRankWarps;
+  permute_rank_kernel<<<blocks, kRankWarps * 32, smem, s>>>(idx, T, K, E, chunk, rank, chunk_counts, status);
+  return cudaGetLastError();
+}
+
+// Exclusive scan of up to 1024 values held one per thread (blockDim = 1024).
+__device__ int block_exclusive_scan_1024(int v, int* sh /* >= 32 ints */, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) sh[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int s = sh[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    sh[lane] = si - s;  // exclusive prefix of warp totals
+    if (lane == 31) sh[32] = si;
+  }
+  __syncthreads();
+  const int res = sh[w] + incl - v;
+  *total = sh[32];
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks,
+                                                             int E, int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ offsets) {
+  __shared__ int sh[33];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int c = 0; c < n_chunks; ++c) {
+      const int v = chunk_counts[(size_t)c * E + e];
+      chunk_counts[(size_t)c * E + e] = run;  // becomes this chunk's base within expert e
+      run += v;
+    }
+    counts[e] = run;
+  }
+  int total;
+  const int off = block_exclusive_scan_1024(e < E ? run : 0, sh, &total);
+  if (e < E) offsets[e] = off;
+  if (e == 0) offsets[E] = total;
+}
+
+cudaError_t launch_permute_scan(int32_t* chunk_counts, int n_chunks, int E, int32_t* counts, int32_t* offsets,
+                                cudaStream_t s) {
+  permute_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, n_chunks, E, counts, offsets);
+  return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __restrict__ idx,
+                                                               const int32_t* __restrict__ rank,
+                                                               const int32_t* __restrict__ chunk_base,
+                                                               const int32_t* __restrict__ offsets, int T, int K,
+                                                               int E, int chunk, int32_t* __restrict__ perm_src,
+                                                               int32_t* __restrict__ perm_k,
+                                                               int32_t* __restrict__ inv) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)T * K) return;
+  const int t = (int)(i / K), k = (int)(i - (int64_t)t * K);
+  const int e = idx[i];
+  const int r = rank[i];
+  if (e < 0 || e >= E || r < 0) {
+    inv[i] = -1;
+    return;
+  }
+  const int c = t / chunk;
+  const int p = offsets[e] + chunk_base[(size_t)c * E + e] + r;
+  perm_src[p] = t;
+  perm_k[p] = k;
+  inv[i] = p;
+}
+
+cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, const int32_t* chunk_base,
+                                   const int32_t* offsets, int T, int K, int E, int chunk, int32_t* perm_src,
+                                   int32_t* perm_k, int32_t* inv, cudaStream_t s) {
+  const int64_t n = (int64_t)T * K;
+  if (n <= 0) return cudaSuccess;
+  permute_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, rank, chunk_base, offsets, T, K, E,
+                                                                      chunk, perm_src, perm_k, inv);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- FFN plan --
+// List = every expert in index order; experts with pairs but no registered
+// weights are flagged and given no tiles.
+__global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restrict__ offsets,
+                                                         const int32_t* __restrict__ map_of, int E, int bn,
+                                                         int32_t* __restrict__ list_expert,
+                                                         int32_t* __restrict__ list_map,
+                                                         int32_t* __restrict__ nt_prefix, int* status) {
+  __shared__ int sh[33];
+  const int e = threadIdx.x;
+  int nt = 0;
+  if (e < E) {
+    const int cnt = offsets[e + 1] - offsets[e];
+    const int m = map_of[e];
+    nt = (cnt + bn - 1) / bn;
+    if (cnt > 0 && m < 0) {
+      flag_status(status, MOE_DEV_NO_SLOT);
+      nt = 0;
+    }
+    list_expert[e] = e;
+    list_map[e] = m < 0 ? 0 : m;
+  }
+  int total;
+  const int pre = block_exclusive_scan_1024(nt, sh, &total);
+  if (e < E) nt_prefix[e] = pre;
+  if (e == 0) nt_prefix[E] = total;
+}
+
+cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s) {
+  ffn_plan_kernel<<<1, 1024, 0, s>>>(offsets, map_of, E, bn, list_expert, list_map, nt_prefix, status);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------- gather --
+// x_perm[p, :] = x[perm_src[p], :] for the offsets[E] valid pairs; one warp per
+// row, 16-byte vectors.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                           const int32_t* __restrict__ perm_src,
+                                                           const int32_t* __restrict__ offsets, int E, int P,
+                                                           int vec_per_row, uint4* __restrict__ xp) {
+  const int lane = threadIdx.x & 31;
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (p >= P || p >= offsets[E]) return;
+  const int t = perm_src[p];
+  const uint4* src = x + (size_t)t * vec_per_row;
+  uint4* dst = xp + (size_t)p * vec_per_row;
+  for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+}
+
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
+                               int H, void* x_perm, cudaStream_t s) {
+  if (P <= 0) return cudaSuccess;
+  gather_rows_kernel<<<(P + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm_src, offsets, E, P,
+                                                 H * 2 / 16, static_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -94,16 +94,51 @@ def _irwin_hall8(idx: torch.Tensor, seed: int, tensor_id: int) -> torch.Tensor:
     return s - 262140
 
 
+_clib = None
+
+
+def _c_generator():
+    """ctypes handle of _gen.c (built on first use with gcc), or None."""
+    global _clib
+    if _clib is None:
+        import ctypes
+        import os
+        import subprocess
+        here = os.path.dirname(os.path.abspath(__file__))
+        src, so = os.path.join(here, "_gen.c"), os.path.join(here, "_gen.so")
+        try:
+            if not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(src):
+                subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-shared", "-fPIC",
+                                       "-o", so + ".tmp", src])
+                os.replace(so + ".tmp", so)
+            lib = ctypes.CDLL(so)
+            lib.synth_normal.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_void_p, ctypes.c_uint32, ctypes.c_float]
+            _clib = lib
+        except Exception:  # no compiler: the torch path below gives the same bits
+            _clib = False
+    return _clib or None
+
+
 def normal(shape, seed: int, tensor_id: int, sigma: float, dtype: torch.dtype,
-           device="cpu", offset: int = 0) -> torch.Tensor:
+           device="cpu", offset: int = 0, use_c: bool = True) -> torch.Tensor:
     """Seeded approx-N(0, sigma^2) tensor; element i uses counter ``offset + i``."""
     shape = tuple(int(s) for s in shape)
     n = 1
     for s in shape:
         n *= s
+    cval = float(np.float32(sigma * math.sqrt(1.5) / 65536.0))
+    if use_c and torch.device(device).type == "cpu" and dtype in (torch.float32, torch.bfloat16) \
+            and _c_generator() is not None:
+        import ctypes
+        kj, khi = _keys(seed, tensor_id)
+        keys = (ctypes.c_uint32 * 4)(*kj)
+        out = torch.empty(n, dtype=dtype)
+        _c_generator().synth_normal(ctypes.c_void_p(out.data_ptr()), 0 if dtype == torch.float32 else 1, n,
+                                    offset, keys, khi, cval)
+        return out.view(shape)
     out = torch.empty(n, dtype=dtype, device=device)
-    c = torch.tensor(float(np.float32(sigma * math.sqrt(1.5) / 65536.0)),
-                     dtype=torch.float32, device=device)
+    c = torch.tensor(cval, dtype=torch.float32, device=device)
     for start in range(0, n, _CHUNK):
         stop = min(n, start + _CHUNK)
         idx = torch.arange(offset + start, offset + stop, dtype=torch.int64, device=device)
