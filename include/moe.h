@@ -156,6 +156,28 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* slots, const void* x, cons
 moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                                moe_stream_t stream);
 
+/* moe_route_noalloc -- the router (logits, top-k, weights; same kernels, same
+ * order and results as moe_route) for callers that cannot allocate device
+ * memory: engines that reserve HBM up front and hand it out only through
+ * their own pool, latency-critical paths that cannot take cudaMalloc's
+ * device-wide synchronisation, and plug-ins whose host process owns the
+ * device allocator. There is no counterpart on the pages this library
+ * follows; it is an interface convenience.
+ *   x [T, H] bf16, w_router [E, H] fp32, logit_bias [E] or NULL (device),
+ *   topk_idx [T, K] int32 out, topk_w [T, K] fp32 out (device).
+ * Needs no context and allocates nothing: its only scratch, the [T, E] fp32
+ * logits, is a fixed array of MOE_ROUTE_NOALLOC_MAX_LOGITS floats (256 KiB)
+ * compiled into the library, present on every GPU that loads it until the
+ * process exits. T * E above that limit returns MOE_ERR_UNSUPPORTED. The
+ * first call on each device looks up the array's device address (make it
+ * before any stream capture). All calls share the array: calls that overlap
+ * on the GPU (two streams, two host threads) race and must be serialised by
+ * the caller. Size limits otherwise as above; errors do not set a status word
+ * (there is no context). */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS 65536
+moe_status_t moe_route_noalloc(const void* x, const float* w_router, const float* logit_bias, int T, int H, int E,
+                               int K, int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
 /* ---- expert-slot table (residency) ------------------------------------ */
 
 /* Creates the slot table of `ctx` with n_spare_slots spare HBM slots

@@ -33,6 +33,7 @@ from .binding import (  # noqa: F401
     moe_profile_read,
     moe_quantize_e4m3,
     moe_route,
+    moe_route_noalloc,
     moe_slots_create,
     moe_slots_destroy,
     moe_slots_query,

@@ -31,7 +31,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_e4m3", "moe_slots_create",
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_read"]
+           "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine"]
 
@@ -85,6 +85,7 @@ def lib():
         "moe_launch_count": ([P], ctypes.c_int64),
         "moe_profile_enable": ([P, I], S),
         "moe_profile_read": ([P, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], S),
+        "moe_route_noalloc": ([P, P, P, I, I, I, I, P, P, P], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -151,6 +152,12 @@ def moe_permute(ctx, topk_idx, T, counts, offsets, perm_src, perm_k, inv, ws, st
 def moe_expert_ffn(ctx, slots, x, perm_src, perm_k, offsets, topk_w, T, y_pair, ws, stream=None):
     _check(lib().moe_expert_ffn(ctx, slots, _p(x), _p(perm_src), _p(perm_k), _p(offsets), _p(topk_w), T,
                                 _p(y_pair), _p(ws), _nbytes(ws), _s(stream)), "moe_expert_ffn")
+
+
+def moe_route_noalloc(x, w_router, logit_bias, T, H, E, K, topk_idx, topk_w, stream=None):
+    """Router without a context or workspace (static scratch inside libmoe)."""
+    _check(lib().moe_route_noalloc(_p(x), _p(w_router), _p(logit_bias), T, H, E, K, _p(topk_idx), _p(topk_w),
+                                   _s(stream)), "moe_route_noalloc")
 
 
 def moe_combine(ctx, y_pair, inv, T, out, stream=None):

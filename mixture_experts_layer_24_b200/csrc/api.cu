@@ -49,6 +49,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+void moe::record_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 struct moe_ctx {
   moe_config_t cfg;
   int device = 0;

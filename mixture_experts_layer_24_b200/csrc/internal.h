@@ -79,6 +79,9 @@ cudaError_t launch_gather_quant_rows(const void* x, const int32_t* perm_src, con
 cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s);
 cudaError_t launch_quant_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                               cudaStream_t s);
+// Sets the text moe_last_error() returns on this thread.
+void record_error(const char* msg);
+
 cudaError_t launch_quant_rows_e4m3_count(const void* src, const int32_t* offsets, int E, int rows, int cols,
                                          uint8_t* q, float* scales, cudaStream_t s);
 
