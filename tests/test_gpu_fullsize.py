@@ -1,0 +1,227 @@
+"""Full-size parity: the 384-expert layer (hidden 4096, top-8, intermediate 2048)
+in the launch configuration bench.py times.
+
+- Routing and permutation: bit-exact for ALL tokens of every batch.
+- Outputs: checked on a seeded sample of tokens against the oracle (a token's
+  output depends on that token alone, which the invariance tests check).
+- Batch invariance across the decode/prefill tile-width switch.
+- Hot/cold residency: bit-identical to the all-resident run, over a chain of
+  layers (vLLM-Moet page, hybrid results table, row "identity": calls, rows,
+  0 differ).
+- FP8 block-scaled experts at full size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import assert_close_out
+
+pytestmark = pytest.mark.gpu
+
+H, E, K, I = 4096, 384, 8, 2048
+ZIPF = 1.1
+TOL_BF16, TOL_FP8 = 2e-2, 4e-2
+
+
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+class FullLayer:
+    def __init__(self, seed, wdtype=0, hot=None, n_spare=0, store=None):
+        import mixture_experts_layer_24_b200 as M
+        self.M, self.seed, self.wdtype = M, seed, wdtype
+        dev = torch.device("cuda")
+        self.dev = dev
+        self.wr = synth.router_weight(E, H, seed=seed, device=dev)
+        self.bias = synth.zipf_logit_bias(E, ZIPF, seed=seed).to(dev)
+        self.layer = M.MoeLayer(H, E, K, I, wdtype=wdtype, n_spare_slots=n_spare, device=dev)
+        self.keep = []
+        for e in range(E):
+            if store is not None:
+                w = store[e]
+            else:
+                g, d = synth.expert_weights(e, H, I, seed=seed, device=dev)
+                if wdtype == 1:
+                    qg = torch.empty((2 * I, H), dtype=torch.uint8, device=dev)
+                    sg = torch.empty((2 * I // 128, H // 128), dtype=torch.float32, device=dev)
+                    qd = torch.empty((H, I), dtype=torch.uint8, device=dev)
+                    sd = torch.empty((H // 128, I // 128), dtype=torch.float32, device=dev)
+                    M.moe_quantize_e4m3(g, 2 * I, H, 128, qg, sg)
+                    M.moe_quantize_e4m3(d, H, I, 128, qd, sd)
+                    w = (qg, qd, sg, sd)
+                else:
+                    w = (g, d, None, None)
+            resident = hot is None or e in hot
+            if resident:
+                self.layer.register(e, w[0], w[1], w[2], w[3], M.MOE_LOC_HBM)
+                self.keep.append(w)
+            else:
+                hw = tuple(None if t is None else t.cpu().pin_memory() for t in w)
+                self.layer.register(e, hw[0], hw[1], hw[2], hw[3], M.MOE_LOC_HOST_PINNED)
+                self.keep.append(hw)
+        torch.cuda.synchronize()
+
+    def forward(self, x):
+        return self.layer.forward(x, self.wr, self.bias)
+
+    def oracle_tokens(self, x, tokens):
+        """Oracle outputs of the given token rows (CPU-generated weights, same bits)."""
+        xu = oracle.as_u16(x)
+        wr = self.wr.cpu().numpy()
+        bias = self.bias.cpu().numpy()
+        sub = xu[np.asarray(tokens)]
+        _, idx, _ = oracle.route(sub, wr, bias, K)
+        gu, dn, sgu, sdn = {}, {}, {}, {}
+        for e in np.unique(idx):
+            e = int(e)
+            g, d = synth.expert_weights(e, H, I, seed=self.seed)
+            if self.wdtype == 1:
+                gu[e], sgu[e] = oracle.quant_e4m3(oracle.as_u16(g), 128)
+                dn[e], sdn[e] = oracle.quant_e4m3(oracle.as_u16(d), 128)
+            else:
+                gu[e], dn[e] = oracle.as_u16(g), oracle.as_u16(d)
+        if self.wdtype == 1:
+            return oracle.forward(sub, wr, bias, K, E, gu, dn, dtype="fp8", scales=(sgu, sdn))["out"]
+        return oracle.forward(sub, wr, bias, K, E, gu, dn)["out"]
+
+    def close(self):
+        self.layer.close()
+        self.keep = []
+
+
+@pytest.fixture(scope="module")
+def full_bf16():
+    _need_cuda()
+    L = FullLayer(seed=0)
+    yield L
+    L.close()
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 512, 4096])
+def test_routing_and_permutation_bit_exact_full(full_bf16, T):
+    L = full_bf16
+    x = synth.tokens(T, H, seed=0, device=L.dev, first_token=7000)
+    idx, w = L.layer.route(x, L.wr, L.bias)
+    counts, offsets, ps, pk, inv = L.layer.permute(idx)
+    torch.cuda.synchronize()
+    _, io, wo = oracle.route(oracle.as_u16(x), L.wr.cpu().numpy(), L.bias.cpu().numpy(), K)
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert np.max(np.abs(w.cpu().numpy() - wo)) < 1e-6
+    ref = oracle.permute(io, E)
+    for g, r in zip((counts, offsets, ps, pk, inv), ref):
+        assert np.array_equal(g.cpu().numpy().reshape(-1), np.asarray(r).reshape(-1))
+
+
+@pytest.mark.parametrize("T,n_sample", [(1, 1), (8, 8), (64, 16), (4096, 24), (16384, 8)])
+def test_outputs_full_size_sampled(full_bf16, T, n_sample):
+    L = full_bf16
+    x = synth.tokens(T, H, seed=0, device=L.dev, first_token=20000)
+    out = L.forward(x)
+    torch.cuda.synchronize()
+    assert L.layer.status() == 0
+    rng = np.random.default_rng(T)
+    tok = np.sort(rng.choice(T, size=n_sample, replace=False))
+    if T > 1:
+        tok[-1] = T - 1  # the ragged tail
+    ref = L.oracle_tokens(x, tok)
+    assert_close_out(oracle.as_u16(out)[tok], ref, TOL_BF16)
+
+
+def test_batch_invariance_across_tile_widths(full_bf16):
+    """Tokens 0..63 of a 4096-token chunk: the same bits in batches of 1..64
+    (tile width 16 and 64), in a 512-token chunk and in the 4096 chunk (256)."""
+    L = full_bf16
+    xb = synth.tokens(4096, H, seed=0, device=L.dev, first_token=50000)
+    ref = oracle.as_u16(L.forward(xb))
+    for T in (1, 2, 4, 8, 16, 64, 512):
+        out = oracle.as_u16(L.forward(xb[:T].contiguous()))
+        assert np.array_equal(out, ref[:T]), f"batch {T} differs from the 4096 chunk"
+    # the same tokens at other positions of another batch
+    perm = torch.arange(63, -1, -1, device=L.dev)
+    out = oracle.as_u16(L.forward(xb[perm].contiguous()))
+    assert np.array_equal(out, ref[:64][perm.cpu().numpy()])
+
+
+def test_hot_cold_bit_identical_to_all_resident():
+    """Two chained layers with 120 hot experts each (picked greedily from a
+    seeded routing histogram), the other 264 in pinned host memory staged
+    through 32 spare slots: decode B=1, B=4 and a 4096-token prefill chunk."""
+    _need_cuda()
+    import mixture_experts_layer_24_b200 as M
+    dev = torch.device("cuda")
+    n_layers, n_hot, n_spare = 2, 120, 32
+    inputs = {T: synth.tokens(T, H, seed=3, device=dev, first_token=90000 + 5000 * i)
+              for i, T in enumerate((1, 4, 4096))}
+    calls = rows = differ = 0
+    cold_total = 0
+    for layer_i in range(n_layers):
+        seed = 10 + layer_i
+        full = FullLayer(seed=seed)
+        # seeded routing histogram -> hot set
+        hx = synth.tokens(2048, H, seed=seed, device=dev, first_token=700000)
+        idx, _ = full.layer.route(hx, full.wr, full.bias)
+        hist = torch.bincount(idx.reshape(-1).long(), minlength=E).cpu()
+        hot = set(M.moe_plan_hot_set(hist, n_hot).tolist())
+        ref = {T: full.forward(x) for T, x in inputs.items()}
+        torch.cuda.synchronize()
+        store = [tuple(full.keep[e]) for e in range(E)]
+        split = FullLayer(seed=seed, hot=hot, n_spare=n_spare, store=store)
+        for e in range(E):
+            loc, slot = M.moe_slots_query(split.layer.slots, e)
+            assert loc == (M.MOE_LOC_HBM if e in hot else M.MOE_LOC_HOST_PINNED)
+        outs = {}
+        for T, x in inputs.items():
+            outs[T] = split.forward(x)
+            torch.cuda.synchronize()
+            st = split.layer.stats()
+            cold_total += st["last_cold"]
+            assert split.layer.status() == 0
+            a, b = oracle.as_u16(outs[T]), oracle.as_u16(ref[T])
+            calls += 1
+            rows += T
+            differ += int(np.sum(np.any(a != b, axis=1)))
+        split.close()
+        full.close()
+        inputs = {T: outs[T] for T in inputs}  # chain: this layer's output feeds the next
+        del store
+        torch.cuda.empty_cache()
+    assert cold_total > 0, "no cold expert was exercised"
+    assert differ == 0, f"{differ} of {rows} rows differ over {calls} calls"
+
+
+@pytest.fixture(scope="module")
+def full_fp8():
+    _need_cuda()
+    L = FullLayer(seed=4, wdtype=1)
+    yield L
+    L.close()
+
+
+@pytest.mark.parametrize("T,n_sample", [(1, 1), (8, 8), (64, 8), (4096, 12)])
+def test_fp8_full_size_sampled(full_fp8, T, n_sample):
+    L = full_fp8
+    x = synth.tokens(T, H, seed=4, device=L.dev, first_token=3000)
+    out = L.forward(x)
+    torch.cuda.synchronize()
+    assert L.layer.status() == 0
+    rng = np.random.default_rng(T + 1)
+    tok = np.sort(rng.choice(T, size=n_sample, replace=False))
+    ref = L.oracle_tokens(x, tok)
+    assert_close_out(oracle.as_u16(out)[tok], ref, TOL_FP8)
+    # FP8 routing is the bf16 router: bit-exact
+    idx, _ = L.layer.route(x, L.wr, L.bias)
+    _, io, _ = oracle.route(oracle.as_u16(x), L.wr.cpu().numpy(), L.bias.cpu().numpy(), K)
+    assert np.array_equal(idx.cpu().numpy(), io)
+
+
+def test_fp8_batch_invariance(full_fp8):
+    L = full_fp8
+    xb = synth.tokens(512, H, seed=4, device=L.dev, first_token=60000)
+    ref = oracle.as_u16(L.forward(xb))
+    for T in (1, 8, 64):
+        assert np.array_equal(oracle.as_u16(L.forward(xb[:T].contiguous())), ref[:T]), T
