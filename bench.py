@@ -165,17 +165,36 @@ def touched_experts(layer, x, wr, bias):
     return int(torch.unique(idx).numel())
 
 
-def time_forwards(layer, xs, wr, bias, flush, stream, steps):
-    """Device ms of `steps` passes over xs (one forward each), L2 flushed before each."""
+_GRAPHS = {}
+
+
+def graph_for(layer, x, wr, bias):
+    """One CUDA graph per input tensor: the whole forward (route, permute, FFN,
+    combine) replays as one launch of the captured kernels."""
+    key = (id(layer), x.data_ptr(), x.shape[0])
+    if key not in _GRAPHS:
+        _GRAPHS[key] = layer.capture(x, wr, bias)
+    return _GRAPHS[key][0]
+
+
+def time_forwards(layer, xs, wr, bias, flush, stream, steps, graphs=False):
+    """Device ms of `steps` passes over xs (one forward each), L2 flushed before each.
+    Inputs are made on the default stream: `stream` (a torch stream, which does
+    not wait for the default stream by itself) is made to wait for them first."""
+    stream.wait_stream(torch.cuda.current_stream())
+    gs = [graph_for(layer, x, wr, bias) for x in xs] if graphs else None
     pairs = []
     with torch.cuda.stream(stream):
         for _ in range(steps):
-            for x in xs:
+            for i, x in enumerate(xs):
                 flush.fill_(1)
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                layer.forward(x, wr, bias, stream=stream)
+                if graphs:
+                    gs[i].replay()
+                else:
+                    layer.forward(x, wr, bias, stream=stream)
                 b.record(stream)
                 pairs.append((a, b))
     torch.cuda.synchronize()
@@ -270,21 +289,24 @@ def run_ours(args):
     layer.workspace(16384 if (world == 1 and not args.no_extras) else max(batches))  # no allocation while timing
     tokens_per_step = sum(batches)
 
-    # warm-up
-    time_forwards(layer, xs, wr, bias, flush, stream, max(args.warmup, 0))
+    use_graphs = not args.eager
+    clocks = ClockSampler(local)
+    clocks.start()  # sampled through warm-up and the timed region (the timed region alone is short)
+    # warm-up (also captures the graphs)
+    launches0 = layer.launches()
+    time_forwards(layer, xs, wr, bias, flush, stream, 1, graphs=False)
+    per_forward_launches = (layer.launches() - launches0) / len(xs)
+    time_forwards(layer, xs, wr, bias, flush, stream, max(args.warmup, 0), graphs=use_graphs)
     status = layer.status()
     if status:
         raise SystemExit(f"device status {status} after warm-up")
 
-    clocks = ClockSampler(local)
     dist_barrier(world)
     torch.cuda.synchronize()
-    launches0 = layer.launches()
-    clocks.start()
-    ms = time_forwards(layer, xs, wr, bias, flush, stream, args.steps)
+    ms = time_forwards(layer, xs, wr, bias, flush, stream, args.steps, graphs=use_graphs)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    launches = layer.launches() - launches0
+    launches = int(round(per_forward_launches * len(xs) * args.steps))
     dist_barrier(world)
     ms_max = dist_max(world, ms, device)
     total_tokens = dist_sum(world, tokens_per_step * args.steps, device)
@@ -296,6 +318,8 @@ def run_ours(args):
             "config": {"workload": workload, "hidden": H, "experts": E, "top_k": K, "intermediate": I,
                        "batches": batches, "zipf_s": ZIPF_S, "weights": "bf16, seeded N(0,0.02)",
                        "l2": "flushed (256 MiB write) before every forward, outside the timed events",
+                       "launch": "CUDA graph per batch (kernels chained with programmatic dependent launch)"
+                       if use_graphs else "eager (kernels chained with programmatic dependent launch)",
                        "parallelism": f"replicas x{world}"},
             "gpu_launches": launches, "gpu_launches_per_step": launches / max(args.steps, 1), "clocks": clk}
 
@@ -338,21 +362,36 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
     out["kernels"]["down"]["achieved_GBps"] = (dn_bytes * steps) / (dn_ms / 1000.0) / 1e9 if dn_ms else None
 
     # --- per-batch / prefill breakdown ---
+    def kernel_profile(x, reps):
+        M.moe_profile_enable(layer.ctx, True)
+        M.moe_profile_read(layer.ctx, reset=True)
+        time_forwards(layer, [x], wr, bias, flush, stream, reps)
+        pr = M.moe_profile_read(layer.ctx, reset=True)
+        M.moe_profile_enable(layer.ctx, False)
+        return {k: round(1000 * v[0] / reps, 2) for k, v in pr.items() if v[1]}
+
     br = {}
+    use_graphs = not args.eager
     for b, x, t in zip(batches, xs, touched):
-        ms = time_forwards(layer, [x], wr, bias, flush, stream, 5) / 5
+        time_forwards(layer, [x], wr, bias, flush, stream, 2, graphs=use_graphs)  # warm-up
+        ms = time_forwards(layer, [x], wr, bias, flush, stream, 5, graphs=use_graphs) / 5
+        ms_eager = time_forwards(layer, [x], wr, bias, flush, stream, 5) / 5
         nbytes = t * EXPERT_BYTES + E * H * 4 + b * H * 2 * 2
-        br[f"B{b}"] = {"us_per_layer": 1000 * ms, "tokens_per_s": b / (ms / 1000), "touched_experts": t,
-                       "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+        br[f"B{b}"] = {"us_per_layer": 1000 * ms, "us_per_layer_eager": 1000 * ms_eager,
+                       "tokens_per_s": b / (ms / 1000), "touched_experts": t,
+                       "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm,
+                       "kernel_us": kernel_profile(x, 3)}
     if args.workload == "decode":
         for T in (512, 4096, 16384):
             x = synth.tokens(T, H, seed=SEED, device=device, first_token=500000)
             reps = 3 if T < 16384 else 2
+            time_forwards(layer, [x], wr, bias, flush, stream, 1)  # warm-up
             ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
             t = touched_experts(layer, x, wr, bias)
             flops = 2.0 * T * K * (2 * I * H + H * I) + 2.0 * T * E * H
             nbytes = t * EXPERT_BYTES + E * H * 4 + T * H * 4
             br[f"prefill{T}"] = {"us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
+                                 "kernel_us": kernel_profile(x, 2),
                                  "tensor_frac": (flops / (ms / 1000) / 1e12) / tf_burst,
                                  "hbm_frac": (nbytes / (ms / 1000) / 1e9) / hbm,
                                  "combined_roofline_frac": max(flops / (tf_burst * 1e12), nbytes / (hbm * 1e9)) /
@@ -363,6 +402,7 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
     hx = [x.cpu().pin_memory() for x in xs]
     hout = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
     dx = [torch.empty_like(x) for x in xs]
+    stream.wait_stream(torch.cuda.current_stream())
     pairs = []
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
@@ -393,6 +433,30 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
     return out
 
 
+def run_profile_case():
+    """Small case for ncu captures of the FFN kernels: the same layer shape with 32
+    experts (1.6 GB of bf16 weights, all touched) and 64 tokens, three forwards."""
+    import mixture_experts_layer_24_b200 as M
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    E_s = 32
+    layer = M.MoeLayer(H, E_s, K, I, device=device)
+    keep = []
+    for e in range(E_s):
+        g, d = synth.expert_weights(e, H, I, seed=SEED, device=device)
+        layer.register(e, g, d)
+        keep.append((g, d))
+    wr = synth.router_weight(E_s, H, seed=SEED, device=device)
+    x = synth.tokens(64, H, seed=SEED, device=device)
+    for _ in range(3):
+        layer.forward(x, wr, None)
+    torch.cuda.synchronize()
+    st = layer.status()
+    print(json.dumps({"profile_case": "E=32 H=4096 I=2048 K=8 T=64 bf16", "status": st}))
+    layer.close()
+    return 1 if st else 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,7 +465,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="small ncu case: 32 experts, 64 tokens, 3 forwards (no timing)")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

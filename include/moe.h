@@ -89,8 +89,15 @@ typedef struct {
   int top_k;        /* K */
   int intermediate; /* I */
   int wdtype;       /* moe_wdtype_t */
-  int flags;        /* reserved, must be 0 */
+  int flags;        /* MOE_FLAG_* bits, 0 = defaults */
 } moe_config_t;
+
+/* Config flags. */
+enum {
+  /* Launch every kernel in plain stream order instead of chaining the
+   * kernels of one call with programmatic dependent launch. */
+  MOE_FLAG_NO_PDL = 1
+};
 
 /* Creates a context on the CURRENT CUDA device (which must be sm_100).
  * Allocates the device status word. Synchronous. */

@@ -124,8 +124,11 @@ def _nbytes(t):
 
 # ------------------------------------------------------------ C entry points --
 
-def moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16):
-    cfg = MoeConfig(hidden, n_experts, top_k, intermediate, wdtype, 0)
+MOE_FLAG_NO_PDL = 1
+
+
+def moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16, flags=0):
+    cfg = MoeConfig(hidden, n_experts, top_k, intermediate, wdtype, flags)
     h = ctypes.c_void_p()
     _check(lib().moe_ctx_create(ctypes.byref(h), ctypes.byref(cfg)), "moe_ctx_create")
     return h
@@ -241,11 +244,12 @@ class MoeLayer:
     Registered weight tensors are kept referenced here because the library
     borrows them."""
 
-    def __init__(self, hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16, n_spare_slots=0, device=None):
+    def __init__(self, hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16, n_spare_slots=0, device=None,
+                 flags=0):
         self.H, self.E, self.K, self.I, self.wdtype = hidden, n_experts, top_k, intermediate, wdtype
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         with torch.cuda.device(self.device):
-            self.ctx = moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype)
+            self.ctx = moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype, flags)
             self.slots = moe_slots_create(self.ctx, n_spare_slots)
         self._keep = {}
         self._ws = None
@@ -260,11 +264,12 @@ class MoeLayer:
             self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
         return self._ws
 
-    def forward(self, x, w_router, logit_bias=None, out=None, stream=None):
+    def forward(self, x, w_router, logit_bias=None, out=None, stream=None, ws=None):
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
-        moe_forward(self.ctx, self.slots, x, w_router, logit_bias, T, out, self.workspace(T), stream)
+        moe_forward(self.ctx, self.slots, x, w_router, logit_bias, T, out, self.workspace(T) if ws is None else ws,
+                    stream)
         return out
 
     def route(self, x, w_router, logit_bias=None, stream=None):
@@ -297,6 +302,24 @@ class MoeLayer:
         out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
         moe_combine(self.ctx, y_pair, inv, T, out, stream)
         return out
+
+    def capture(self, x, w_router, logit_bias=None):
+        """Captures one forward over the fixed tensor x into a CUDA graph.
+
+        Returns (graph, out): graph.replay() recomputes out from the current
+        contents of x. Valid while x, w_router, logit_bias and the registered
+        weights stay where they are; residency must be all-HBM (the hot/cold
+        path synchronises with the host and cannot be captured)."""
+        T = x.shape[0]
+        ws = torch.empty(max(moe_workspace_size(self.ctx, T), 256), dtype=torch.uint8, device=self.device)
+        out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        self.forward(x, w_router, logit_bias, out=out, ws=ws)  # first call outside capture (kernel attributes)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.forward(x, w_router, logit_bias, out=out, ws=ws)
+        g.moe_workspace = ws  # the graph's own workspace lives as long as the graph
+        return g, out
 
     def status(self, reset=True) -> int:
         return moe_get_device_status(self.ctx, reset)

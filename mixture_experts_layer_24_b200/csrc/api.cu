@@ -55,6 +55,9 @@ struct moe_ctx {
   moe_config_t cfg;
   int device = 0;
   int* d_status = nullptr;
+  int num_sms = 148;
+  bool chain = true;  // programmatic dependent launch between this library's kernels
+  unsigned int* d_counters = nullptr;  // arrival counters of the decode router (self-resetting)
   int host_status = 0;
   EncodeTiledFn encode = nullptr;
   std::atomic<int64_t> launches{0};
@@ -178,7 +181,7 @@ moe_status_t check_cfg(const moe_config_t& c) {
   if (c.hidden <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.intermediate <= 0)
     return fail(MOE_ERR_INVALID_ARG, "config sizes must be positive");
   if (c.wdtype != MOE_BF16 && c.wdtype != MOE_FP8_E4M3_B128) return fail(MOE_ERR_INVALID_ARG, "unknown wdtype");
-  if (c.flags != 0) return fail(MOE_ERR_INVALID_ARG, "flags must be 0");
+  if (c.flags & ~MOE_FLAG_NO_PDL) return fail(MOE_ERR_INVALID_ARG, "unknown flag bits");
   if (c.hidden % 128 || c.intermediate % 128) return fail(MOE_ERR_UNSUPPORTED, "H and I must be multiples of 128");
   if (c.hidden > 8192 || c.intermediate > 8192) return fail(MOE_ERR_UNSUPPORTED, "H and I must be <= 8192");
   if (c.top_k > 32 || c.top_k > c.n_experts || c.n_experts > 1024)
@@ -240,7 +243,7 @@ moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void
 moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void* ws, int T, int bn,
                        const int32_t* perm_src, const int32_t* perm_k, const int32_t* offsets, const float* topk_w,
                        float* y_pair, const int32_t* list_expert, const int32_t* list_map, const int32_t* nt_prefix,
-                       int L, int max_ntiles, cudaStream_t s) {
+                       int L, int max_ntiles, cudaStream_t s, bool pdl, bool plan_ready_gu) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
@@ -266,21 +269,27 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   a.perm_k = perm_k;
   a.status = ctx->d_status;
   a.act_scale = fp8 ? at<float>(ws, W.x_scale) : nullptr;
+  a.plan_ready = (pdl && plan_ready_gu) ? 1 : 0;
+  a.num_sms = ctx->num_sms;
+  const int max_experts = std::min(L, P);  // experts that can hold a pair
+  a.est_tiles = (c.intermediate / 128) * std::min(max_ntiles, max_experts * ((P + bn - 1) / bn));
   {
     Prof p(ctx, MOE_PROF_GATE_UP, s);
-    MOE_CUDA(launch_ffn_gemm(kGateUp, c.wdtype, bn, xmap, a, (c.intermediate / 128) * max_ntiles, s));
+    MOE_CUDA(launch_ffn_gemm(kGateUp, c.wdtype, bn, xmap, a, (c.intermediate / 128) * max_ntiles, s, pdl));
   }
   if (fp8) {
     {
       Prof p(ctx, MOE_PROF_QUANT, s);
       MOE_CUDA(launch_quant_rows_e4m3_count(at<void>(ws, W.h), offsets, c.n_experts, P, c.intermediate,
-                                            at<uint8_t>(ws, W.hq), at<float>(ws, W.h_scale), s));
+                                            at<uint8_t>(ws, W.hq), at<float>(ws, W.h_scale), s, pdl));
     }
     a.act_scale = at<float>(ws, W.h_scale);
   }
+  a.plan_ready = pdl ? 1 : 0;  // the plan is at least two launches back from the down GEMM
+  a.est_tiles = (c.hidden / 128) * std::min(max_ntiles, max_experts * ((P + bn - 1) / bn));
   {
     Prof p(ctx, MOE_PROF_DOWN, s);
-    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, a, (c.hidden / 128) * max_ntiles, s));
+    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, a, (c.hidden / 128) * max_ntiles, s, pdl));
   }
   return MOE_OK;
 }
@@ -310,12 +319,17 @@ moe_status_t moe_ctx_create(moe_ctx_t** out, const moe_config_t* cfg) {
   moe_ctx_t* ctx = new moe_ctx_t();
   ctx->cfg = *cfg;
   ctx->device = dev;
+  ctx->num_sms = prop.multiProcessorCount;
+  ctx->chain = !(cfg->flags & MOE_FLAG_NO_PDL);
   ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
-  if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess) {
+  if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&ctx->d_counters, sizeof(unsigned int) * kRouteSmallMaxT) != cudaSuccess) {
+    cudaFree(ctx->d_status);
     delete ctx;
-    return fail(MOE_ERR_OOM, "cudaMalloc of the status word failed");
+    return fail(MOE_ERR_OOM, "cudaMalloc of the context's device words failed");
   }
   cudaMemset(ctx->d_status, 0, sizeof(int));
+  cudaMemset(ctx->d_counters, 0, sizeof(unsigned int) * kRouteSmallMaxT);
   cudaDeviceSynchronize();
   *out = ctx;
   return MOE_OK;
@@ -329,6 +343,7 @@ moe_status_t moe_ctx_destroy(moe_ctx_t* ctx) {
   }
   for (auto e : ctx->ev_pool) cudaEventDestroy(e);
   cudaFree(ctx->d_status);
+  cudaFree(ctx->d_counters);
   delete ctx;
   return MOE_OK;
 }
@@ -383,77 +398,85 @@ moe_status_t moe_get_device_status(moe_ctx_t* ctx, int32_t* status, int reset) {
   return MOE_OK;
 }
 
-moe_status_t moe_route(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
-                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
-  moe_status_t st = check_T(ctx, T);
-  if (st != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
-  if (!x || !w_router || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
-  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+}  // extern "C"
+
+namespace {
+
+// ---- step implementations; `pdl` = launch the first kernel with programmatic
+// stream serialisation (only when the preceding launch is this library's own
+// kernel of the same forward).
+
+moe_status_t route_impl(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
+                        int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s) {
   const moe_config_t& c = ctx->cfg;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(c, T);
   float* logits = at<float>(ws, W.logits);
+  if (T <= kRouteSmallMaxT) {
+    Prof p(ctx, MOE_PROF_ROUTER, s);
+    MOE_CUDA(launch_route_small(x, w_router, logit_bias, T, c.hidden, c.n_experts, c.top_k, logits, topk_idx,
+                                topk_w, ctx->d_counters, ctx->d_status, s, ctx->chain));
+    return MOE_OK;
+  }
   {
     Prof p(ctx, MOE_PROF_ROUTER, s);
-    MOE_CUDA(launch_router_logits(x, w_router, logit_bias, T, c.hidden, c.n_experts, logits, s));
+    MOE_CUDA(launch_route_gemm(x, w_router, logit_bias, T, c.hidden, c.n_experts, logits, s));
   }
   {
     Prof p(ctx, MOE_PROF_TOPK, s);
-    MOE_CUDA(launch_topk(logits, T, c.n_experts, c.top_k, topk_idx, topk_w, ctx->d_status, s));
+    MOE_CUDA(launch_topk_warp(logits, T, c.n_experts, c.top_k, topk_idx, topk_w, s, ctx->chain));
   }
   return MOE_OK;
 }
 
-moe_status_t moe_permute(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
-                         int32_t* perm_src, int32_t* perm_k, int32_t* inv, void* ws, size_t ws_bytes,
-                         moe_stream_t stream) {
-  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
-  moe_status_t st = check_T(ctx, T);
-  if (st != MOE_OK) return st;
-  if (!counts || !offsets) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
-  if (T > 0 && (!topk_idx || !perm_src || !perm_k || !inv)) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
-  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+// Small batches: one launch (plus, with map_of, the FFN tile plan and, with
+// x_perm, the sorted activation rows). Otherwise rank -> scan -> scatter.
+moe_status_t permute_impl(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
+                          int32_t* perm_src, int32_t* perm_k, int32_t* inv, void* ws, cudaStream_t s, bool pdl,
+                          const int32_t* map_of = nullptr, int bn = 0, const void* x = nullptr,
+                          void* x_perm = nullptr, bool* planned = nullptr) {
   const moe_config_t& c = ctx->cfg;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(c, T);
+  if (planned) *planned = false;
+  if ((long long)T * c.top_k <= kPermuteSmallMaxPairs) {
+    Prof p(ctx, MOE_PROF_PERMUTE, s);
+    MOE_CUDA(launch_permute_small(topk_idx, T, c.top_k, c.n_experts, counts, offsets, perm_src, perm_k, inv, map_of,
+                                  bn, at<int32_t>(ws, W.list_expert), at<int32_t>(ws, W.list_map),
+                                  at<int32_t>(ws, W.nt_prefix), x, c.hidden, x_perm, ctx->d_status, s, pdl));
+    if (planned) *planned = map_of != nullptr;
+    return MOE_OK;
+  }
   const int chunk = permute_chunk_tokens(T, c.top_k);
   const int n_chunks = T > 0 ? (T + chunk - 1) / chunk : 0;
   int32_t* cc = at<int32_t>(ws, W.chunk_counts);
   if (T > 0) {
     Prof p(ctx, MOE_PROF_PERMUTE, s);
     MOE_CUDA(launch_permute_rank(topk_idx, T, c.top_k, c.n_experts, chunk, at<int32_t>(ws, W.rank), cc,
-                                 ctx->d_status, s));
+                                 ctx->d_status, s, pdl));
+    pdl = ctx->chain;
   }
   {
     Prof p(ctx, MOE_PROF_PERMUTE, s);
-    MOE_CUDA(launch_permute_scan(cc, n_chunks, c.n_experts, counts, offsets, s));
+    MOE_CUDA(launch_permute_scan(cc, n_chunks, c.n_experts, counts, offsets, s, pdl));
   }
   if (T > 0) {
     Prof p(ctx, MOE_PROF_PERMUTE, s);
     MOE_CUDA(launch_permute_scatter(topk_idx, at<int32_t>(ws, W.rank), cc, offsets, T, c.top_k, c.n_experts, chunk,
-                                    perm_src, perm_k, inv, s));
+                                    perm_src, perm_k, inv, s, ctx->chain));
   }
   return MOE_OK;
 }
 
-moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
-                            const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T,
-                            float* y_pair, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  if (!ctx || !sl) return fail(MOE_ERR_INVALID_ARG, "NULL context or slot table");
-  if (sl->ctx != ctx) return fail(MOE_ERR_SLOT, "slot table belongs to another context");
-  moe_status_t st = check_T(ctx, T);
-  if (st != MOE_OK) return st;
-  if (T == 0) return MOE_OK;
-  if (!x || !perm_src || !perm_k || !offsets || !topk_w || !y_pair) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
-  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+// Expert FFN. `planned`: the permutation step already wrote the tile plan and
+// (bf16) the sorted rows; `pdl`: the previous launch is this forward's own.
+moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
+                      const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T, float* y_pair,
+                      void* ws, cudaStream_t s, bool pdl, bool planned) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const WsLayout W = ws_layout(c, T);
   const int E = c.n_experts, P = T * c.top_k;
   const int bn = ffn_block_n(T, c.wdtype);
+  moe_status_t st = MOE_OK;
   std::lock_guard<std::mutex> lock(sl->mu);
   sl->stats.calls++;
 
@@ -462,26 +485,42 @@ moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, cons
   int32_t* np = at<int32_t>(ws, W.nt_prefix);
   const int ntile_bound = (P + bn - 1) / bn + std::min(E, P);
 
-  // activation rows in sorted-pair order (quantised for FP8)
-  {
-  Prof pg(ctx, MOE_PROF_GATHER, s);
-  if (fp8) {
-    MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
-                                      at<float>(ws, W.x_scale), s));
-  } else {
-    MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s));
-  }
-  }
-
   if (sl->n_host == 0) {
-    {
-      Prof p(ctx, MOE_PROF_PERMUTE, s);
-      MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s));
-    }
     sl->stats.last_cold = 0;
     sl->stats.last_touched = -1;
+    bool plan_ready_gu = false;
+    if (!planned) {
+      {
+        Prof p(ctx, MOE_PROF_PERMUTE, s);
+        MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl));
+      }
+      Prof pg(ctx, MOE_PROF_GATHER, s);
+      if (fp8) {
+        MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                          at<float>(ws, W.x_scale), s, ctx->chain));
+      } else {
+        MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s, ctx->chain));
+      }
+      plan_ready_gu = true;  // plan -> gather -> gate/up
+    } else if (fp8) {
+      Prof pg(ctx, MOE_PROF_GATHER, s);
+      MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                        at<float>(ws, W.x_scale), s, pdl));
+      plan_ready_gu = pdl;  // permutation+plan -> quantiser -> gate/up
+    }
     return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
-                     s);
+                     s, ctx->chain, plan_ready_gu);
+  }
+
+  // activation rows in sorted-pair order (quantised for FP8); no PDL on the host-synchronised path
+  {
+    Prof pg(ctx, MOE_PROF_GATHER, s);
+    if (fp8) {
+      MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                        at<float>(ws, W.x_scale), s, false));
+    } else {
+      MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s, false));
+    }
   }
 
   // ---- hot/cold: read the per-expert offsets back, stage the routed cold experts
@@ -544,7 +583,7 @@ moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, cons
   if (!hot.empty()) {
     const ListRef& r = lists[li++];
     st = run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le + r.e_off, lm + r.e_off,
-                   np + r.p_off, r.L, ntile_bound, s);
+                   np + r.p_off, r.L, ntile_bound, s, false, false);
     if (st != MOE_OK) return st;
   }
   for (int b = 0; b < n_batches; ++b) {
@@ -568,11 +607,54 @@ moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, cons
     MOE_CUDA(cudaEventRecord(sl->ev_ready[buf], sl->copy_stream));
     MOE_CUDA(cudaStreamWaitEvent(s, sl->ev_ready[buf], 0));
     st = run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le + r.e_off, lm + r.e_off,
-                   np + r.p_off, r.L, ntile_bound, s);
+                   np + r.p_off, r.L, ntile_bound, s, false, false);
     if (st != MOE_OK) return st;
     MOE_CUDA(cudaEventRecord(sl->ev_free[buf], s));
   }
   return MOE_OK;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  return route_impl(ctx, x, w_router, logit_bias, T, topk_idx, topk_w, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_t* counts, int32_t* offsets,
+                         int32_t* perm_src, int32_t* perm_k, int32_t* inv, void* ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if (T > 0 && (!topk_idx || !perm_src || !perm_k || !inv)) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  return permute_impl(ctx, topk_idx, T, counts, offsets, perm_src, perm_k, inv, ws, static_cast<cudaStream_t>(stream),
+                      false);
+}
+
+moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
+                            const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T,
+                            float* y_pair, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ctx || !sl) return fail(MOE_ERR_INVALID_ARG, "NULL context or slot table");
+  if (sl->ctx != ctx) return fail(MOE_ERR_SLOT, "slot table belongs to another context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !perm_src || !perm_k || !offsets || !topk_w || !y_pair) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
+  return ffn_impl(ctx, sl, x, perm_src, perm_k, offsets, topk_w, T, y_pair, ws, static_cast<cudaStream_t>(stream),
+                  false, false);
 }
 
 moe_status_t moe_combine(moe_ctx_t* ctx, const float* y_pair, const int32_t* inv, int T, void* out,
@@ -583,7 +665,8 @@ moe_status_t moe_combine(moe_ctx_t* ctx, const float* y_pair, const int32_t* inv
   if (T == 0) return MOE_OK;
   if (!y_pair || !inv || !out) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
   Prof p(ctx, MOE_PROF_COMBINE, static_cast<cudaStream_t>(stream));
-  MOE_CUDA(launch_combine(y_pair, inv, T, ctx->cfg.top_k, ctx->cfg.hidden, out, static_cast<cudaStream_t>(stream)));
+  MOE_CUDA(launch_combine(y_pair, inv, T, ctx->cfg.top_k, ctx->cfg.hidden, out, static_cast<cudaStream_t>(stream),
+                          false));
   return MOE_OK;
 }
 
@@ -591,24 +674,38 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
                          const float* logit_bias, int T, void* out, void* ws, size_t ws_bytes,
                          moe_stream_t stream) {
   if (!ctx || !sl) return fail(MOE_ERR_INVALID_ARG, "NULL context or slot table");
+  if (sl->ctx != ctx) return fail(MOE_ERR_SLOT, "slot table belongs to another context");
   moe_status_t st = check_T(ctx, T);
   if (st != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   if (!x || !w_router || !out) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
   if ((st = check_ws(ctx, T, ws, ws_bytes)) != MOE_OK) return st;
-  const WsLayout W = ws_layout(ctx->cfg, T);
+  const moe_config_t& c = ctx->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const WsLayout W = ws_layout(c, T);
   int32_t* idx = at<int32_t>(ws, W.topk_idx);
   float* w = at<float>(ws, W.topk_w);
-  if ((st = moe_route(ctx, x, w_router, logit_bias, T, idx, w, ws, ws_bytes, stream)) != MOE_OK) return st;
   int32_t* counts = at<int32_t>(ws, W.counts);
   int32_t* offsets = at<int32_t>(ws, W.offsets);
   int32_t* ps = at<int32_t>(ws, W.perm_src);
   int32_t* pk = at<int32_t>(ws, W.perm_k);
   int32_t* inv = at<int32_t>(ws, W.inv);
-  if ((st = moe_permute(ctx, idx, T, counts, offsets, ps, pk, inv, ws, ws_bytes, stream)) != MOE_OK) return st;
   float* y = at<float>(ws, W.y_pair);
-  if ((st = moe_expert_ffn(ctx, sl, x, ps, pk, offsets, w, T, y, ws, ws_bytes, stream)) != MOE_OK) return st;
-  return moe_combine(ctx, y, inv, T, out, stream);
+  const bool resident = sl->n_host == 0;
+  const bool chain = ctx->chain;
+  // route (first kernel: ordinary stream order with whatever came before)
+  if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s)) != MOE_OK) return st;
+  // permutation (+ tile plan + sorted bf16 rows when the batch is small)
+  bool planned = false;
+  const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  if ((st = permute_impl(ctx, idx, T, counts, offsets, ps, pk, inv, ws, s, chain, resident ? sl->d_map_of : nullptr,
+                         ffn_block_n(T, c.wdtype), x, (resident && !fp8) ? at<void>(ws, W.x_perm) : nullptr,
+                         &planned)) != MOE_OK)
+    return st;
+  if ((st = ffn_impl(ctx, sl, x, ps, pk, offsets, w, T, y, ws, s, chain, planned)) != MOE_OK) return st;
+  Prof p(ctx, MOE_PROF_COMBINE, s);
+  MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, resident && chain));
+  return MOE_OK;
 }
 
 moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,

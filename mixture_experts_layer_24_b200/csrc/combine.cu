@@ -12,6 +12,8 @@ namespace moe {
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y,
                                                        const int32_t* __restrict__ inv, int K, int H4,
                                                        uint2* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int v = blockIdx.y * blockDim.x + threadIdx.x;
   if (v >= H4) return;
@@ -41,12 +43,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   out[(size_t)t * H4 + v] = o;
 }
 
-cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s) {
+cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s,
+                           bool pdl) {
   if (T <= 0) return cudaSuccess;
   const int H4 = H / 4;
   dim3 grid(T, (H4 + 255) / 256);
-  combine_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(y), inv, K, H4, static_cast<uint2*>(out));
-  return cudaGetLastError();
+  return launch_ex(combine_kernel, grid, dim3(256), 0, s, pdl, reinterpret_cast<const float4*>(y), inv, K, H4,
+                   static_cast<uint2*>(out));
 }
 
 }  // namespace moe

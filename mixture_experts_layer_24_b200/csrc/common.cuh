@@ -186,6 +186,32 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N, uint32_t fmt) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// Kernels of one forward are chained with programmatic stream serialisation.
+// Each kernel calls pdl_wait() before touching what its immediate predecessor
+// wrote, and pdl_trigger() only AFTER its own pdl_wait(): so when a kernel
+// starts, every kernel two or more launches back has completed, and data they
+// wrote (the permutation, the tile plan) may be read before pdl_wait().
+// Launched without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// 1-D bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// ------------------------------------------------------------- cp.async --
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc --
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }

@@ -42,10 +42,13 @@ template <int MODE, int BN>
 struct Bf16Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
   static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;
-  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // Pipeline depth is chosen per launch: the deepest that fits one CTA per SM
+  // when the grid is at most one wave, else (narrow tiles) the depth that fits
+  // two CTAs per SM so that more tiles stream at once.
+  static constexpr int kStagesMax = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kStagesTwo = BN <= 32 ? (104 * 1024) / kStageBytes : kStagesMax;
   static constexpr uint32_t kTmemCols = tmem_cols_for(NA * BN);
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + 256;
+  static constexpr size_t smem(int stages) { return 1024 + (size_t)stages * kStageBytes + 256; }
 };
 
 template <int MODE, int BN>
@@ -98,13 +101,21 @@ template <int MODE, int BN>
 __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ CUtensorMap act_map,
                                                           const GemmArgs a) {
   using C = Bf16Cfg<MODE, BN>;
-  constexpr int NA = C::NA, S = C::kStages;
+  constexpr int NA = C::NA;
+  const int S = a.stages;
   constexpr uint32_t STAGE = C::kStageBytes;
   constexpr uint32_t IDESC = instr_desc(128, BN, 1u);
 
   TileInfo ti;
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
-  if (!decode_tile(a, m_tiles, BN, ti)) return;
+  if (!a.plan_ready) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  if (!decode_tile(a, m_tiles, BN, ti)) {
+    pdl_wait();
+    return;
+  }
   const int KB = (MODE == kGateUp ? a.H : a.I) / 64;
 
   extern __shared__ uint8_t smem_raw[];
@@ -146,7 +157,22 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
       tma_prefetch_map(wmap);
       tma_prefetch_map(&act_map);
       const uint64_t pol_w = l2_policy_evict_first();
-      int kb = 0;
+      // with the plan already complete, weight tiles for the first stages go
+      // out before waiting for the kernel that writes the activations
+      const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
+      for (int kb = 0; kb < npre; ++kb) {
+        const uint32_t st = base + kb * STAGE;
+        mbar_arrive_expect_tx(full(kb), STAGE);
+        tma_load_2d_hint(st, wmap, full(kb), kb * 64, ti.mt * 128, pol_w);
+        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(kb), kb * 64, a.I + ti.mt * 128, pol_w);
+      }
+      if (a.plan_ready) {
+        pdl_wait();
+        pdl_trigger();
+      }
+      for (int kb = 0; kb < npre; ++kb) tma_load_2d(base + kb * STAGE + NA * kABytes, &act_map, full(kb), kb * 64,
+                                                    ti.row0);
+      int kb = npre;
       for (; kb < KB; ++kb) {
         const int s = kb % S;
         if (kb >= S && !mbar_wait(empty(s), ((kb / S) - 1) & 1)) {
@@ -163,8 +189,15 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
       }
       // every load this thread issued has landed before the CTA may exit
       for (int j = kb - S < 0 ? 0 : kb - S; j < kb; ++j) mbar_wait(full(j % S), (j / S) & 1);
+    } else if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
     }
   } else if (warp == 5) {
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     if (lane == 0) {
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % S;
@@ -187,6 +220,10 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
       tc_commit(accf);
     }
   } else {
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     const bool ok = mbar_wait(accf, 0);
     if (!ok) flag_status(a.status, MOE_DEV_TIMEOUT);
     tc_fence_after();
@@ -257,7 +294,14 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
 
   TileInfo ti;
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
-  if (!decode_tile(a, m_tiles, BN, ti)) return;
+  if (!a.plan_ready) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  if (!decode_tile(a, m_tiles, BN, ti)) {
+    pdl_wait();
+    return;
+  }
   const int KD = MODE == kGateUp ? a.H : a.I;  // reduction length
   const int KB = KD / 128;
 
@@ -287,7 +331,12 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // activation scales of this tile's pairs -> shared memory
+  // activation scales of this tile's pairs -> shared memory (they come from the
+  // immediately preceding kernel)
+  if (a.plan_ready) {
+    pdl_wait();
+    pdl_trigger();
+  }
   for (int i = threadIdx.x; i < BN * KB; i += blockDim.x) {
     const int n = i / KB, kb = i - n * KB;
     s_act[i] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
@@ -441,30 +490,36 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
 
 template <typename Kern>
 static cudaError_t launch_kernel(Kern kern, size_t smem, int threads, int grid, const CUtensorMap& map,
-                                 const GemmArgs& a, cudaStream_t s) {
+                                 const GemmArgs& a, cudaStream_t s, bool pdl) {
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, threads, smem, s>>>(map, a);
-  return cudaGetLastError();
+  return launch_ex(kern, dim3(grid), dim3(threads), smem, s, pdl, map, a);
+}
+
+template <int MODE, int BN>
+static cudaError_t launch_bf16(const CUtensorMap& map, GemmArgs a, int grid, cudaStream_t s, bool pdl) {
+  using C = Bf16Cfg<MODE, BN>;
+  a.stages = a.est_tiles <= a.num_sms ? C::kStagesMax : C::kStagesTwo;
+  return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 192, grid, map, a, s, pdl);
 }
 
 template <int MODE>
 static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const GemmArgs& a, int grid,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool pdl) {
   if (wdtype == MOE_BF16) {
     switch (bn) {
-      case 16: return launch_kernel(ffn_bf16_kernel<MODE, 16>, Bf16Cfg<MODE, 16>::kSmem, 192, grid, map, a, s);
-      case 32: return launch_kernel(ffn_bf16_kernel<MODE, 32>, Bf16Cfg<MODE, 32>::kSmem, 192, grid, map, a, s);
-      case 64: return launch_kernel(ffn_bf16_kernel<MODE, 64>, Bf16Cfg<MODE, 64>::kSmem, 192, grid, map, a, s);
-      case 128: return launch_kernel(ffn_bf16_kernel<MODE, 128>, Bf16Cfg<MODE, 128>::kSmem, 192, grid, map, a, s);
-      case 256: return launch_kernel(ffn_bf16_kernel<MODE, 256>, Bf16Cfg<MODE, 256>::kSmem, 192, grid, map, a, s);
+      case 16: return launch_bf16<MODE, 16>(map, a, grid, s, pdl);
+      case 32: return launch_bf16<MODE, 32>(map, a, grid, s, pdl);
+      case 64: return launch_bf16<MODE, 64>(map, a, grid, s, pdl);
+      case 128: return launch_bf16<MODE, 128>(map, a, grid, s, pdl);
+      case 256: return launch_bf16<MODE, 256>(map, a, grid, s, pdl);
     }
   } else {
     switch (bn) {
-      case 16: return launch_kernel(ffn_fp8_kernel<MODE, 16>, Fp8Cfg<MODE, 16>::kSmem, 320, grid, map, a, s);
-      case 32: return launch_kernel(ffn_fp8_kernel<MODE, 32>, Fp8Cfg<MODE, 32>::kSmem, 320, grid, map, a, s);
-      case 64: return launch_kernel(ffn_fp8_kernel<MODE, 64>, Fp8Cfg<MODE, 64>::kSmem, 320, grid, map, a, s);
+      case 16: return launch_kernel(ffn_fp8_kernel<MODE, 16>, Fp8Cfg<MODE, 16>::kSmem, 320, grid, map, a, s, pdl);
+      case 32: return launch_kernel(ffn_fp8_kernel<MODE, 32>, Fp8Cfg<MODE, 32>::kSmem, 320, grid, map, a, s, pdl);
+      case 64: return launch_kernel(ffn_fp8_kernel<MODE, 64>, Fp8Cfg<MODE, 64>::kSmem, 320, grid, map, a, s, pdl);
     }
   }
   return cudaErrorInvalidValue;
@@ -480,19 +535,19 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
   if (wdtype == MOE_BF16) {
     if (mode == kGateUp) {
       switch (bn) {
-        case 16: return Bf16Cfg<kGateUp, 16>::kSmem;
-        case 32: return Bf16Cfg<kGateUp, 32>::kSmem;
-        case 64: return Bf16Cfg<kGateUp, 64>::kSmem;
-        case 128: return Bf16Cfg<kGateUp, 128>::kSmem;
-        case 256: return Bf16Cfg<kGateUp, 256>::kSmem;
+        case 16: return Bf16Cfg<kGateUp, 16>::smem(Bf16Cfg<kGateUp, 16>::kStagesMax);
+        case 32: return Bf16Cfg<kGateUp, 32>::smem(Bf16Cfg<kGateUp, 32>::kStagesMax);
+        case 64: return Bf16Cfg<kGateUp, 64>::smem(Bf16Cfg<kGateUp, 64>::kStagesMax);
+        case 128: return Bf16Cfg<kGateUp, 128>::smem(Bf16Cfg<kGateUp, 128>::kStagesMax);
+        case 256: return Bf16Cfg<kGateUp, 256>::smem(Bf16Cfg<kGateUp, 256>::kStagesMax);
       }
     } else {
       switch (bn) {
-        case 16: return Bf16Cfg<kDown, 16>::kSmem;
-        case 32: return Bf16Cfg<kDown, 32>::kSmem;
-        case 64: return Bf16Cfg<kDown, 64>::kSmem;
-        case 128: return Bf16Cfg<kDown, 128>::kSmem;
-        case 256: return Bf16Cfg<kDown, 256>::kSmem;
+        case 16: return Bf16Cfg<kDown, 16>::smem(Bf16Cfg<kDown, 16>::kStagesMax);
+        case 32: return Bf16Cfg<kDown, 32>::smem(Bf16Cfg<kDown, 32>::kStagesMax);
+        case 64: return Bf16Cfg<kDown, 64>::smem(Bf16Cfg<kDown, 64>::kStagesMax);
+        case 128: return Bf16Cfg<kDown, 128>::smem(Bf16Cfg<kDown, 128>::kStagesMax);
+        case 256: return Bf16Cfg<kDown, 256>::smem(Bf16Cfg<kDown, 256>::kStagesMax);
       }
     }
   } else {
@@ -514,9 +569,9 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
 }
 
 cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const GemmArgs& a,
-                            int max_tiles, cudaStream_t s) {
-  if (mode == kGateUp) return launch_mode<kGateUp>(wdtype, bn, act_map, a, max_tiles, s);
-  return launch_mode<kDown>(wdtype, bn, act_map, a, max_tiles, s);
+                            int max_tiles, cudaStream_t s, bool pdl) {
+  if (mode == kGateUp) return launch_mode<kGateUp>(wdtype, bn, act_map, a, max_tiles, s, pdl);
+  return launch_mode<kDown>(wdtype, bn, act_map, a, max_tiles, s, pdl);
 }
 
 }  // namespace moe

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -21,6 +23,24 @@ struct alignas(64) MapEntry {
 };
 
 enum FfnMode { kGateUp = 0, kDown = 1 };
+
+// Launches `kern` on `s`, with programmatic stream serialisation when pdl is
+// true (the kernel must then follow the pdl_wait / pdl_trigger rule).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // The token-column tile width the FFN GEMMs use for a batch of T tokens. It
 // depends on T only, so the tile that computes a given pair does not depend on
@@ -44,13 +64,18 @@ struct GemmArgs {
   const int32_t* perm_k;      // [P]
   const float* act_scale;     // FP8: scales of the activation operand [P, Kdim/128]
   int* status;
+  int plan_ready;             // 1: the tile plan was written two or more launches back
+                              // (read it, and start streaming weights, before pdl_wait)
+  int stages;                 // pipeline depth (set by the launcher)
+  int est_tiles;              // host-side bound on the tiles of this launch
+  int num_sms;
 };
 
 // Launches one FFN GEMM (gate/up+SwiGLU or down*weight) over the tile list.
 // act_map is the TMA descriptor of the activation operand (x_perm or h);
 // max_tiles bounds the grid (CTAs past the real tile count exit at once).
 cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const GemmArgs& a,
-                            int max_tiles, cudaStream_t s);
+                            int max_tiles, cudaStream_t s, bool pdl);
 size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn);
 
 cudaError_t launch_router_logits(const void* x, const float* wr, const float* bias, int T, int H, int E,
@@ -58,31 +83,55 @@ cudaError_t launch_router_logits(const void* x, const float* wr, const float* bi
 cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, float* w, int* status,
                         cudaStream_t s);
 
+// Decode-regime router (T <= kRouteSmallMaxT): logits and top-k in one launch.
+// counters: >= kRouteSmallMaxT zero-initialised words owned by the caller's
+// context (each is returned to zero by the kernel that uses it).
+constexpr int kRouteSmallMaxT = 64;
+cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
+                               float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
+                               cudaStream_t s, bool pdl);
+// Prefill-regime router logits (register-tiled fp32 GEMM in the same order).
+cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias, int T, int H, int E,
+                              float* logits, cudaStream_t s);
+// Top-k + weights for any T, one warp per token (logits read through L2).
+cudaError_t launch_topk_warp(const float* logits, int T, int E, int K, int32_t* idx, float* w, cudaStream_t s,
+                             bool pdl);
+
+// Small-batch permutation (T*K <= kPermuteSmallMaxPairs): counts, offsets, the
+// sorted pairs, optionally the FFN tile plan (map_of != nullptr) and the row
+// gather of x (x_perm != nullptr), in one launch of n_ctas CTAs.
+constexpr int kPermuteSmallMaxPairs = 1024;
+cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_t* counts, int32_t* offsets,
+                                 int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
+                                 int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
+                                 void* x_perm, int* status, cudaStream_t s, bool pdl);
+
 // Permutation: rank -> scan -> scatter. chunk = tokens per warp-chunk.
 int permute_chunk_tokens(int T, int K);
 cudaError_t launch_permute_rank(const int32_t* idx, int T, int K, int E, int chunk, int32_t* rank,
-                                int32_t* chunk_counts, int* status, cudaStream_t s);
+                                int32_t* chunk_counts, int* status, cudaStream_t s, bool pdl);
 cudaError_t launch_permute_scan(int32_t* chunk_counts, int n_chunks, int E, int32_t* counts, int32_t* offsets,
-                                cudaStream_t s);
+                                cudaStream_t s, bool pdl);
 cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, const int32_t* chunk_base,
                                    const int32_t* offsets, int T, int K, int E, int chunk, int32_t* perm_src,
-                                   int32_t* perm_k, int32_t* inv, cudaStream_t s);
+                                   int32_t* perm_k, int32_t* inv, cudaStream_t s, bool pdl);
 
 // FFN tile plan for the all-resident case: every expert with pairs, in order.
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
-                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s);
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl);
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
-                               int H, void* x_perm, cudaStream_t s);
+                               int H, void* x_perm, cudaStream_t s, bool pdl);
 cudaError_t launch_gather_quant_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E,
-                                     int P, int H, uint8_t* xq, float* xs, cudaStream_t s);
-cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s);
+                                     int P, int H, uint8_t* xq, float* xs, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s,
+                           bool pdl);
 cudaError_t launch_quant_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                               cudaStream_t s);
 // Sets the text moe_last_error() returns on this thread.
 void record_error(const char* msg);
 
 cudaError_t launch_quant_rows_e4m3_count(const void* src, const int32_t* offsets, int E, int rows, int cols,
-                                         uint8_t* q, float* scales, cudaStream_t s);
+                                         uint8_t* q, float* scales, cudaStream_t s, bool pdl);
 
 }  // namespace moe

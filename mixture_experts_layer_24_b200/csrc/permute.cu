@@ -12,6 +12,8 @@
 //            exclusive scan over experts (offsets).
 //   scatter: p = offsets[e] + chunk_base[c][e] + rank.
 // Integer arithmetic only: the result is bit-exact and run-to-run identical.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -34,6 +36,8 @@ __global__ void __launch_bounds__(kRankWarps * 32) permute_rank_kernel(const int
                                                                         int32_t* __restrict__ chunk_counts,
                                                                         int* status) {
   extern __shared__ int32_t cnt_all[];
+  pdl_wait();
+  pdl_trigger();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x * kRankWarps + w;
   const int n_chunks = (T + chunk - 1) / chunk;
@@ -65,13 +69,13 @@ __global__ void __launch_bounds__(kRankWarps * 32) permute_rank_kernel(const int
 }
 
 cudaError_t launch_permute_rank(const int32_t* idx, int T, int K, int E, int chunk, int32_t* rank,
-                                int32_t* chunk_counts, int* status, cudaStream_t s) {
+                                int32_t* chunk_counts, int* status, cudaStream_t s, bool pdl) {
   if (T <= 0) return cudaSuccess;
   const int n_chunks = (T + chunk - 1) / chunk;
   const int blocks = (n_chunks + kRankWarps - 1) / kRankWarps;
   const size_t smem = sizeof(int32_t) * (size_t)E * kRankWarps;
-  permute_rank_kernel<<<blocks, kRankWarps * 32, smem, s>>>(idx, T, K, E, chunk, rank, chunk_counts, status);
-  return cudaGetLastError();
+  return launch_ex(permute_rank_kernel, dim3(blocks), dim3(kRankWarps * 32), smem, s, pdl, idx, T, K, E, chunk,
+                   rank, chunk_counts, status);
 }
 
 // Exclusive scan of up to 1024 values held one per thread (blockDim = 1024).
@@ -107,13 +111,21 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
                                                              int E, int32_t* __restrict__ counts,
                                                              int32_t* __restrict__ offsets) {
   __shared__ int sh[33];
+  pdl_wait();
+  pdl_trigger();
   const int e = threadIdx.x;
   int run = 0;
   if (e < E) {
-    for (int c = 0; c < n_chunks; ++c) {
-      const int v = chunk_counts[(size_t)c * E + e];
-      chunk_counts[(size_t)c * E + e] = run;  // becomes this chunk's base within expert e
-      run += v;
+    // 16 independent loads in flight per round, then the running sum
+    for (int c0 = 0; c0 < n_chunks; c0 += 16) {
+      int v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = c0 + j < n_chunks ? chunk_counts[(size_t)(c0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (c0 + j < n_chunks) chunk_counts[(size_t)(c0 + j) * E + e] = run;  // chunk's base within expert e
+        run += v[j];
+      }
     }
     counts[e] = run;
   }
@@ -124,9 +136,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
 }
 
 cudaError_t launch_permute_scan(int32_t* chunk_counts, int n_chunks, int E, int32_t* counts, int32_t* offsets,
-                                cudaStream_t s) {
-  permute_scan_kernel<<<1, 1024, 0, s>>>(chunk_counts, n_chunks, E, counts, offsets);
-  return cudaGetLastError();
+                                cudaStream_t s, bool pdl) {
+  return launch_ex(permute_scan_kernel, dim3(1), dim3(1024), 0, s, pdl, chunk_counts, n_chunks, E, counts, offsets);
 }
 
 __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __restrict__ idx,
@@ -136,6 +147,8 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
                                                                int E, int chunk, int32_t* __restrict__ perm_src,
                                                                int32_t* __restrict__ perm_k,
                                                                int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)T * K) return;
   const int t = (int)(i / K), k = (int)(i - (int64_t)t * K);
@@ -154,12 +167,11 @@ __global__ void __launch_bounds__(256) permute_scatter_kernel(const int32_t* __r
 
 cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, const int32_t* chunk_base,
                                    const int32_t* offsets, int T, int K, int E, int chunk, int32_t* perm_src,
-                                   int32_t* perm_k, int32_t* inv, cudaStream_t s) {
+                                   int32_t* perm_k, int32_t* inv, cudaStream_t s, bool pdl) {
   const int64_t n = (int64_t)T * K;
   if (n <= 0) return cudaSuccess;
-  permute_scatter_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(idx, rank, chunk_base, offsets, T, K, E,
-                                                                      chunk, perm_src, perm_k, inv);
-  return cudaGetLastError();
+  return launch_ex(permute_scatter_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, pdl, idx, rank,
+                   chunk_base, offsets, T, K, E, chunk, perm_src, perm_k, inv);
 }
 
 // --------------------------------------------------------------- FFN plan --
@@ -171,6 +183,8 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
                                                          int32_t* __restrict__ list_map,
                                                          int32_t* __restrict__ nt_prefix, int* status) {
   __shared__ int sh[33];
+  pdl_wait();
+  pdl_trigger();
   const int e = threadIdx.x;
   int nt = 0;
   if (e < E) {
@@ -191,9 +205,9 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
 }
 
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
-                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s) {
-  ffn_plan_kernel<<<1, 1024, 0, s>>>(offsets, map_of, E, bn, list_expert, list_map, nt_prefix, status);
-  return cudaGetLastError();
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl) {
+  return launch_ex(ffn_plan_kernel, dim3(1), dim3(1024), 0, s, pdl, offsets, map_of, E, bn, list_expert, list_map,
+                   nt_prefix, status);
 }
 
 // ----------------------------------------------------------------- gather --
@@ -203,6 +217,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                            const int32_t* __restrict__ perm_src,
                                                            const int32_t* __restrict__ offsets, int E, int P,
                                                            int vec_per_row, uint4* __restrict__ xp) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (p >= P || p >= offsets[E]) return;
@@ -213,11 +229,117 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
-                               int H, void* x_perm, cudaStream_t s) {
+                               int H, void* x_perm, cudaStream_t s, bool pdl) {
   if (P <= 0) return cudaSuccess;
-  gather_rows_kernel<<<(P + 7) / 8, 256, 0, s>>>(static_cast<const uint4*>(x), perm_src, offsets, E, P,
-                                                 H * 2 / 16, static_cast<uint4*>(x_perm));
-  return cudaGetLastError();
+  return launch_ex(gather_rows_kernel, dim3((P + 7) / 8), dim3(256), 0, s, pdl, static_cast<const uint4*>(x),
+                   perm_src, offsets, E, P, H * 2 / 16, static_cast<uint4*>(x_perm));
+}
+
+// ------------------------------------------------------ small batches --
+// Whole permutation of T*K <= 1024 pairs in one launch: every CTA builds it in
+// shared memory (a counting sort: order-free counts, one block scan, then each
+// pair's rank among earlier pairs of its expert), CTA 0 writes counts,
+// offsets, the sorted pairs and (optionally) the FFN tile plan, and all CTAs
+// copy their share of the sorted x rows. Same result as rank/scan/scatter.
+__global__ void __launch_bounds__(1024) permute_small_kernel(
+    const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_k,
+    int32_t* __restrict__ inv, const int32_t* __restrict__ map_of, int bn, int32_t* __restrict__ list_expert,
+    int32_t* __restrict__ list_map, int32_t* __restrict__ nt_prefix, const uint4* __restrict__ x, int vec_per_row,
+    uint4* __restrict__ x_perm, int* status) {
+  __shared__ __align__(16) int s_e[kPermuteSmallMaxPairs];
+  __shared__ int s_cnt[1024];
+  __shared__ int s_off[1024];
+  __shared__ int s_src[kPermuteSmallMaxPairs];
+  __shared__ int sh[33];
+  pdl_wait();
+  pdl_trigger();
+  const int P = T * K;
+  const int i = threadIdx.x;
+  int e = -1;
+  if (i < P) {
+    e = idx[i];
+    if (e < 0 || e >= E) {
+      if (blockIdx.x == 0) flag_status(status, MOE_DEV_BAD_EXPERT);
+      e = -1;
+    }
+  }
+  s_e[i] = e;
+  s_cnt[i] = 0;
+  __syncthreads();
+  if (e >= 0) atomicAdd(&s_cnt[e], 1);
+  __syncthreads();
+  const int cnt = i < E ? s_cnt[i] : 0;
+  int total;
+  const int off = block_exclusive_scan_1024(cnt, sh, &total);
+  s_off[i] = off;
+  __syncthreads();
+  int p = -1;
+  if (e >= 0) {
+    int r = 0;
+    const int4* e4 = reinterpret_cast<const int4*>(s_e);
+    const int n4 = i >> 2;
+    for (int j = 0; j < n4; ++j) {
+      const int4 v = e4[j];
+      r += (v.x == e) + (v.y == e) + (v.z == e) + (v.w == e);
+    }
+    for (int j = n4 << 2; j < i; ++j) r += s_e[j] == e;
+    p = s_off[e] + r;
+    s_src[p] = i;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    if (i < E) {
+      counts[i] = cnt;
+      offsets[i] = off;
+    }
+    if (i == 0) offsets[E] = total;
+    if (i < P) {
+      inv[i] = p;
+      if (p >= 0) {
+        perm_src[p] = i / K;
+        perm_k[p] = i - (i / K) * K;
+      }
+    }
+    if (map_of) {
+      int nt = 0;
+      if (i < E) {
+        const int m = map_of[i];
+        nt = (cnt + bn - 1) / bn;
+        if (cnt > 0 && m < 0) {
+          flag_status(status, MOE_DEV_NO_SLOT);
+          nt = 0;
+        }
+        list_expert[i] = i;
+        list_map[i] = m < 0 ? 0 : m;
+      }
+      int nt_total;
+      const int pre = block_exclusive_scan_1024(nt, sh, &nt_total);
+      if (i < E) nt_prefix[i] = pre;
+      if (i == 0) nt_prefix[E] = nt_total;
+    }
+  }
+  if (x_perm) {
+    const int warp = i >> 5, lane = i & 31, nw = blockDim.x >> 5;
+    for (int row = blockIdx.x * nw + warp; row < total; row += gridDim.x * nw) {
+      const int t = s_src[row] / K;
+      const uint4* src = x + (size_t)t * vec_per_row;
+      uint4* dst = x_perm + (size_t)row * vec_per_row;
+      for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+    }
+  }
+}
+
+cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_t* counts, int32_t* offsets,
+                                 int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
+                                 int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
+                                 void* x_perm, int* status, cudaStream_t s, bool pdl) {
+  const int P = T * K;
+  int ctas = 1;
+  if (x_perm) ctas = std::max(1, std::min(64, (P + 31) / 32));
+  return launch_ex(permute_small_kernel, dim3(ctas), dim3(1024), 0, s, pdl, idx, T, K, E, counts, offsets, perm_src,
+                   perm_k, inv, map_of, bn, list_expert, list_map, nt_prefix, static_cast<const uint4*>(x), H / 8,
+                   static_cast<uint4*>(x_perm), status);
 }
 
 }  // namespace moe

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
                                                           const int32_t* __restrict__ offsets, int E, int rows,
                                                           int cols, uint8_t* __restrict__ q,
                                                           float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int groups = cols / 128;
@@ -99,21 +101,20 @@ cudaError_t launch_quant_e4m3(const void* src, int rows, int cols, int block_row
 }
 
 cudaError_t launch_gather_quant_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
-                                     int H, uint8_t* xq, float* xs, cudaStream_t s) {
+                                     int H, uint8_t* xq, float* xs, cudaStream_t s, bool pdl) {
   if (P <= 0) return cudaSuccess;
   const int64_t warps = (int64_t)P * (H / 128);
-  quant_rows_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(static_cast<const uint16_t*>(x), perm_src,
-                                                                 offsets, E, P, H, xq, xs);
-  return cudaGetLastError();
+  return launch_ex(quant_rows_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl,
+                   static_cast<const uint16_t*>(x), perm_src, offsets, E, P, H, xq, xs);
 }
 
 cudaError_t launch_quant_rows_e4m3_count(const void* src, const int32_t* offsets, int E, int rows, int cols,
-                                         uint8_t* q, float* scales, cudaStream_t s) {
+                                         uint8_t* q, float* scales, cudaStream_t s, bool pdl) {
   if (rows <= 0) return cudaSuccess;
   const int64_t warps = (int64_t)rows * (cols / 128);
-  quant_rows_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(static_cast<const uint16_t*>(src), nullptr,
-                                                                 offsets, E, rows, cols, q, scales);
-  return cudaGetLastError();
+  return launch_ex(quant_rows_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl,
+                   static_cast<const uint16_t*>(src), static_cast<const int32_t*>(nullptr), offsets, E, rows, cols,
+                   q, scales);
 }
 
 }  // namespace moe

@@ -77,6 +77,10 @@ def test_config_validation(lib):
     import mixture_experts_layer_24_b200 as M
     bad = [(100, 8, 2, 256, 0, 2), (256, 8, 2, 100, 0, 2), (256, 8, 40, 256, 0, 2), (256, 4, 8, 256, 0, 2),
            (256, 8, 2, 256, 5, 1), (256, 2000, 2, 256, 0, 2)]
+    # unknown flag bits are rejected before any device call
+    cfg = M.binding.MoeConfig(256, 8, 2, 256, 0, 8)
+    h = ctypes.c_void_p()
+    assert lib.moe_ctx_create(ctypes.byref(h), ctypes.byref(cfg)) == 1
     for H, E, K, I, dt, want in bad:
         cfg = M.binding.MoeConfig(H, E, K, I, dt, 0)
         h = ctypes.c_void_p()

@@ -225,3 +225,34 @@ def test_fp8_batch_invariance(full_fp8):
     ref = oracle.as_u16(L.forward(xb))
     for T in (1, 8, 64):
         assert np.array_equal(oracle.as_u16(L.forward(xb[:T].contiguous())), ref[:T]), T
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 512, 4096])
+def test_side_stream_chained_launches_match_plain_order(full_bf16, T):
+    """The same forward on a non-default stream (kernels chained by
+    programmatic dependent launch, the configuration bench.py times) and in
+    plain stream order (MOE_FLAG_NO_PDL) give identical bits; both are checked
+    on sampled tokens against the oracle."""
+    import mixture_experts_layer_24_b200 as M
+    L = full_bf16
+    x = synth.tokens(T, H, seed=0, device=L.dev, first_token=800000)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())  # torch's streams do not wait for the default stream by themselves
+    outs = []
+    for rep in range(3):
+        with torch.cuda.stream(side):
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=L.dev)
+            L.layer.forward(x, L.wr, L.bias, out=out, stream=side)
+        side.synchronize()
+        outs.append(oracle.as_u16(out))
+    plain = M.MoeLayer(H, E, K, I, device=L.dev, flags=M.binding.MOE_FLAG_NO_PDL)
+    for e in range(E):
+        plain.register(e, L.keep[e][0], L.keep[e][1])
+    ref = oracle.as_u16(plain.forward(x, L.wr, L.bias))
+    torch.cuda.synchronize()
+    for o in outs:
+        assert np.array_equal(o, ref)
+    assert L.layer.status() == 0 and plain.status() == 0
+    tok = np.unique(np.array([0, T // 2, T - 1]))
+    assert_close_out(ref[tok], L.oracle_tokens(x, tok), TOL_BF16)
+    plain.close()

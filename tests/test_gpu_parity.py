@@ -225,3 +225,44 @@ def test_empty_batch_is_a_no_op():
     torch.cuda.synchronize()
     assert case.layer.status() == 0
     case.close()
+
+
+def test_graph_replay_matches_eager():
+    """A forward captured in a CUDA graph (kernels chained by programmatic
+    dependent launch) gives the eager bits, replay after replay."""
+    case = LayerCase(64, 512, 16, 4, 256, seed=12)
+    ref = oracle.as_u16(case.forward())
+    g, out = case.layer.capture(case.x, case.wr, case.bias)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(oracle.as_u16(out), ref)
+    # new input contents, same buffer
+    case.x.copy_(synth.tokens(64, 512, seed=13, device="cuda"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(oracle.as_u16(out), oracle.as_u16(case.forward()))
+    assert case.layer.status() == 0
+    case.close()
+
+
+@pytest.mark.parametrize("T", [1, 5, 64, 65, 129])
+def test_small_and_large_paths_agree(T):
+    """Batches around the decode/prefill switch of the router (64 tokens) and of
+    the single-launch permutation (1024 pairs) give the oracle's routing and
+    the same bits as the same tokens inside a bigger batch."""
+    H, E, K, I = 1024, 64, 8, 256
+    big = LayerCase(160, H, E, K, I, seed=31, zipf=1.1)
+    ref = oracle.as_u16(big.forward())
+    x = big.x[:T].contiguous()
+    idx, w = big.layer.route(x, big.wr, big.bias)
+    _, io, wo = oracle.route(oracle.as_u16(x), big.wr.cpu().numpy(), big.bias.cpu().numpy(), K)
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert np.max(np.abs(w.cpu().numpy() - wo)) < 1e-6
+    got = big.layer.permute(idx)
+    for g, r in zip(got, oracle.permute(io, E)):
+        assert np.array_equal(g.cpu().numpy().reshape(-1), np.asarray(r).reshape(-1))
+    out = oracle.as_u16(big.layer.forward(x, big.wr, big.bias))
+    assert np.array_equal(out, ref[:T])
+    big.close()
