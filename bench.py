@@ -324,7 +324,7 @@ def run_ours(args):
             "gpu_launches": launches, "gpu_launches_per_step": launches / max(args.steps, 1), "clocks": clk}
 
     if world == 1 and not args.no_extras:
-        line.update(extras(layer, wr, bias, xs, batches, flush, stream, args, device))
+        line.update(extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -333,7 +333,7 @@ def run_ours(args):
     return 0
 
 
-def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
+def extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep):
     import mixture_experts_layer_24_b200 as M
     hbm, tf_burst, tf_sust, peak_kind = peaks()
     out = {}
@@ -398,6 +398,10 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
                                  (ms / 1000)}
     out["breakdown"] = br
 
+    if args.workload == "decode" and not args.quick:
+        br.update(fp8_breakdown(keep, wr, bias, flush, stream, device, hbm))
+        br.update(hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm))
+
     # --- end to end through the public API, host buffers ---
     hx = [x.cpu().pin_memory() for x in xs]
     hout = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
@@ -433,13 +437,15 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device):
     return out
 
 
-def run_profile_case():
-    """Small case for ncu captures of the FFN kernels: the same layer shape with 32
-    experts (1.6 GB of bf16 weights, all touched) and 64 tokens, three forwards."""
+def run_profile_case(kind):
+    """Small cases for ncu captures of the FFN kernels, three forwards each:
+    "t64": the layer shape with 32 experts (1.6 GB of bf16 weights, all
+    touched) and 64 tokens; "t1": 8 experts (top-8 of 8, all touched, 400 MB)
+    and one token -- the per-launch shape of batch-1 decode."""
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    E_s = 32
+    E_s, T_s = (32, 64) if kind == "t64" else (8, 1)
     layer = M.MoeLayer(H, E_s, K, I, device=device)
     keep = []
     for e in range(E_s):
@@ -447,14 +453,109 @@ def run_profile_case():
         layer.register(e, g, d)
         keep.append((g, d))
     wr = synth.router_weight(E_s, H, seed=SEED, device=device)
-    x = synth.tokens(64, H, seed=SEED, device=device)
+    x = synth.tokens(T_s, H, seed=SEED, device=device)
     for _ in range(3):
         layer.forward(x, wr, None)
     torch.cuda.synchronize()
     st = layer.status()
-    print(json.dumps({"profile_case": "E=32 H=4096 I=2048 K=8 T=64 bf16", "status": st}))
+    print(json.dumps({"profile_case": f"E={E_s} H=4096 I=2048 K=8 T={T_s} bf16", "status": st}))
     layer.close()
     return 1 if st else 0
+
+
+def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
+    """The same layer with e4m3 experts (128x128 block scales, quantised on the
+    GPU from the bf16 weights): decode B=1, 8, 64 and a 4096-token chunk."""
+    import mixture_experts_layer_24_b200 as M
+    layer = M.MoeLayer(H, E, K, I, wdtype=M.MOE_FP8_E4M3_B128, device=device)
+    qkeep = []
+    for e in range(E):
+        g, d = keep[e]
+        qg = torch.empty((2 * I, H), dtype=torch.uint8, device=device)
+        sg = torch.empty((2 * I // 128, H // 128), dtype=torch.float32, device=device)
+        qd = torch.empty((H, I), dtype=torch.uint8, device=device)
+        sd = torch.empty((H // 128, I // 128), dtype=torch.float32, device=device)
+        M.moe_quantize_e4m3(g, 2 * I, H, 128, qg, sg)
+        M.moe_quantize_e4m3(d, H, I, 128, qd, sd)
+        layer.register(e, qg, qd, sg, sd)
+        qkeep.append((qg, sg, qd, sd))
+    torch.cuda.synchronize()
+    layer.workspace(4096)
+    fp8_bytes = 3 * I * H + 2 * (2 * I // 128) * (H // 128) * 4 + 2 * (H // 128) * (I // 128) * 4
+    out = {}
+    for T in (1, 8, 64, 4096):
+        x = synth.tokens(T, H, seed=SEED, device=device, first_token=600000)
+        time_forwards(layer, [x], wr, bias, flush, stream, 2)
+        reps = 5 if T < 4096 else 3
+        ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
+        t = touched_experts(layer, x, wr, bias)
+        nbytes = t * fp8_bytes + E * H * 4 + T * H * 4
+        out[f"fp8_B{T}" if T < 4096 else "fp8_prefill4096"] = {
+            "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
+            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+    if layer.status():
+        out["fp8_device_status"] = layer.status()
+    layer.close()
+    del qkeep
+    torch.cuda.empty_cache()
+    return out
+
+
+def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_spare=32):
+    """120 of the 384 experts resident (greedy hot set from a seeded 2048-token
+    routing histogram), the other 264 in pinned host memory staged through 32
+    spare HBM slots on demand: decode B=1, B=4 and a 4096-token chunk. Bound:
+    max(resident bytes / HBM, staged bytes / measured pinned H2D rate)."""
+    import mixture_experts_layer_24_b200 as M
+    probe = M.MoeLayer(H, E, K, I, device=device)
+    for e in range(E):
+        probe.register(e, *keep[e])
+    hx = synth.tokens(2048, H, seed=SEED, device=device, first_token=700000)
+    idx, _ = probe.route(hx, wr, bias)
+    hist = torch.bincount(idx.reshape(-1).long(), minlength=E).cpu()
+    hot = set(M.moe_plan_hot_set(hist, n_hot).tolist())
+    probe.close()
+    layer = M.MoeLayer(H, E, K, I, n_spare_slots=n_spare, device=device)
+    host = {}
+    for e in range(E):
+        g, d = keep[e]
+        if e in hot:
+            layer.register(e, g, d)
+        else:
+            hg, hd = g.cpu().pin_memory(), d.cpu().pin_memory()
+            host[e] = (hg, hd)
+            layer.register(e, hg, hd, None, None, M.MOE_LOC_HOST_PINNED)
+    # pinned host -> HBM rate on this box (one 400 MB copy)
+    src = torch.empty(200 << 20, dtype=torch.bfloat16).pin_memory()
+    dst = torch.empty_like(src, device=device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    dst.copy_(src, non_blocking=True)
+    b.record()
+    torch.cuda.synchronize()
+    h2d_gbs = src.numel() * 2 / (a.elapsed_time(b) / 1000) / 1e9
+    del src, dst
+    out = {"hotcold_h2d_GBps": h2d_gbs}
+    for T in (1, 4, 4096):
+        x = synth.tokens(T, H, seed=SEED, device=device, first_token=610000)
+        time_forwards(layer, [x], wr, bias, flush, stream, 1)
+        reps = 3
+        ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
+        st = layer.stats()
+        cold = st["last_cold"]
+        touched = st["last_touched"]
+        hot_bytes = (touched - cold) * EXPERT_BYTES
+        cold_bytes = cold * EXPERT_BYTES
+        bound_s = max(hot_bytes / (hbm * 1e9), cold_bytes / (h2d_gbs * 1e9))
+        out[f"hotcold_B{T}" if T < 4096 else "hotcold_prefill4096"] = {
+            "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": touched,
+            "cold_experts_staged": cold, "cold_bytes": cold_bytes,
+            "roofline_frac": bound_s / (ms / 1000) if ms > 0 else None}
+    if layer.status():
+        out["hotcold_device_status"] = layer.status()
+    layer.close()
+    del host
+    return out
 
 
 def main():
@@ -466,11 +567,12 @@ def main():
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
-    ap.add_argument("--profile-case", action="store_true",
-                    help="small ncu case: 32 experts, 64 tokens, 3 forwards (no timing)")
+    ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1"],
+                    help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:
-        return run_profile_case()
+        return run_profile_case(args.profile_case)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

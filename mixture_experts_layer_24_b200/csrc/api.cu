@@ -223,11 +223,35 @@ moe_status_t encode_2d(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, bool fp8
   return MOE_OK;
 }
 
+// bf16 operand as (64 elements, rows, K/64 chunks): one copy of box
+// {64, box_rows, kc} brings kc K chunks, each a swizzled box_rows x 128 B block.
+moe_status_t encode_3d_bf16(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                            uint32_t box_rows, uint32_t kc) {
+  const cuuint64_t dims[3] = {64, rows, inner / 64};
+  const cuuint64_t strides[2] = {inner * 2, 128};
+  const cuuint32_t box[3] = {64u, box_rows, kc};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
 moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void* dn, const float* sgu,
                         const float* sdn) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   std::memset(me, 0, sizeof(*me));
+  if (!fp8) {
+    for (int kc = 1; kc <= 2; ++kc) {
+      moe_status_t st = encode_3d_bf16(ctx, kc == 1 ? &me->gu : &me->gu2, gu, c.hidden, 2ull * c.intermediate, 128, kc);
+      if (st != MOE_OK) return st;
+      st = encode_3d_bf16(ctx, kc == 1 ? &me->dn : &me->dn2, dn, c.intermediate, c.hidden, 128, kc);
+      if (st != MOE_OK) return st;
+    }
+    return MOE_OK;
+  }
   moe_status_t st = encode_2d(ctx, &me->gu, gu, fp8, c.hidden, 2ull * c.intermediate, 128);
   if (st != MOE_OK) return st;
   st = encode_2d(ctx, &me->dn, dn, fp8, c.intermediate, c.hidden, 128);
@@ -248,9 +272,24 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
   CUtensorMap xmap, hmap;
-  moe_status_t st = encode_2d(ctx, &xmap, at<void>(ws, W.x_perm), fp8, c.hidden, P, bn);
-  if (st != MOE_OK) return st;
-  st = encode_2d(ctx, &hmap, fp8 ? at<void>(ws, W.hq) : at<void>(ws, W.h), fp8, c.intermediate, P, bn);
+  ActMaps xmaps, hmaps;  // bf16: one map per tile box height 16 .. bn
+  moe_status_t st = MOE_OK;
+  if (fp8) {
+    st = encode_2d(ctx, &xmap, at<void>(ws, W.x_perm), true, c.hidden, P, bn);
+    if (st != MOE_OK) return st;
+    st = encode_2d(ctx, &hmap, at<void>(ws, W.hq), true, c.intermediate, P, bn);
+  } else {
+    std::memset(&xmaps, 0, sizeof(xmaps));
+    std::memset(&hmaps, 0, sizeof(hmaps));
+    for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
+      st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, ffn_k_chunks(kGateUp, bn));
+      if (st != MOE_OK) return st;
+      st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, ffn_k_chunks(kDown, bn));
+      if (st != MOE_OK) return st;
+    }
+    xmap = xmaps.m[0];
+    hmap = hmaps.m[0];
+  }
   if (st != MOE_OK) return st;
   GemmArgs a{};
   a.maps = sl->d_maps;
@@ -275,7 +314,7 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   a.est_tiles = (c.intermediate / 128) * std::min(max_ntiles, max_experts * ((P + bn - 1) / bn));
   {
     Prof p(ctx, MOE_PROF_GATE_UP, s);
-    MOE_CUDA(launch_ffn_gemm(kGateUp, c.wdtype, bn, xmap, a, (c.intermediate / 128) * max_ntiles, s, pdl));
+    MOE_CUDA(launch_ffn_gemm(kGateUp, c.wdtype, bn, xmap, &xmaps, a, (c.intermediate / 128) * max_ntiles, s, pdl));
   }
   if (fp8) {
     {
@@ -289,7 +328,7 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   a.est_tiles = (c.hidden / 128) * std::min(max_ntiles, max_experts * ((P + bn - 1) / bn));
   {
     Prof p(ctx, MOE_PROF_DOWN, s);
-    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, a, (c.hidden / 128) * max_ntiles, s, pdl));
+    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, &hmaps, a, (c.hidden / 128) * max_ntiles, s, pdl));
   }
   return MOE_OK;
 }

@@ -38,17 +38,23 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
   return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
 }
 
+// bf16: one pipeline stage holds kKC consecutive 64-wide K chunks, fetched by
+// one 3-D TMA copy per operand (the per-copy cost of the TMA unit, not the
+// bytes, bounds a single SM's streaming rate for small boxes).
 template <int MODE, int BN>
 struct Bf16Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;
-  // Pipeline depth is chosen per launch: the deepest that fits one CTA per SM
-  // when the grid is at most one wave, else (narrow tiles) the depth that fits
-  // two CTAs per SM so that more tiles stream at once.
-  static constexpr int kStagesMax = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-  static constexpr int kStagesTwo = BN <= 32 ? (104 * 1024) / kStageBytes : kStagesMax;
-  static constexpr uint32_t kTmemCols = tmem_cols_for(NA * BN);
-  static constexpr size_t smem(int stages) { return 1024 + (size_t)stages * kStageBytes + 256; }
+  static constexpr int KC = ffn_k_chunks(MODE, BN);
+  static constexpr uint32_t kChunkA = kABytes;     // 128 rows x 128 B
+  static constexpr uint32_t kChunkB = BN * 128;    // BN rows x 128 B
+  static constexpr uint32_t kStageBytes = KC * (NA * kChunkA + kChunkB);
+  static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
+  static constexpr int kStagesMax = kStagesFit > 8 ? 8 : kStagesFit;
+  // two accumulator buffers whenever both fit in TMEM's 512 columns
+  static constexpr int NBUF = 2 * NA * BN <= 512 ? 2 : 1;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(NBUF * NA * BN);
+  static constexpr size_t smem(int stages) { return 1024 + (size_t)stages * kStageBytes + 256 + 4 * BN; }
+  static_assert(kStagesMax >= 2, "a pipeline needs two stages");
 };
 
 template <int MODE, int BN>
@@ -91,52 +97,99 @@ __device__ __forceinline__ bool decode_tile(const GemmArgs& a, int m_tiles, int 
   return true;
 }
 
+// Same as decode_tile for an explicit tile index (no range or status checks).
+__device__ __forceinline__ void decode_tile_at(const GemmArgs& a, int m_tiles, int bn, int tile, TileInfo& ti) {
+  int lo = 0, hi = a.L;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.nt_prefix[mid] * m_tiles <= tile) lo = mid;
+    else hi = mid;
+  }
+  const int nti = a.nt_prefix[lo + 1] - a.nt_prefix[lo];
+  const int local = tile - a.nt_prefix[lo] * m_tiles;
+  const int mt = local / nti, nt = local - mt * nti;
+  ti.e = a.list_expert[lo];
+  ti.mapi = a.list_map[lo];
+  ti.mt = mt;
+  ti.row0 = a.offsets[ti.e] + nt * bn;
+  ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
+}
+
 __device__ __forceinline__ void tensormap_acquire(const void* map) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
 }
 
 // ====================================================================== bf16
+// Persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ... The
+// shared-memory pipeline runs on across tile boundaries (stage and phase come
+// from one running K-step count), and the accumulator lives in one of NBUF
+// TMEM buffers so that the epilogue of tile j overlaps the MMAs of tile j+1.
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Per-tile MMA width: the smallest of 16, 32, 64, 128, 256 (<= BN) that holds
+// the tile's pairs; its index selects the activation map of that box height.
+__device__ __forceinline__ int tile_width_index(int nvalid, int bn) {
+  int w = 16, i = 0;
+  while (w < nvalid && w < bn) {
+    w <<= 1;
+    ++i;
+  }
+  return i;
+}
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ CUtensorMap act_map,
+__global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ ActMaps act,
                                                           const GemmArgs a) {
   using C = Bf16Cfg<MODE, BN>;
-  constexpr int NA = C::NA;
-  const int S = a.stages;
+  constexpr int NA = C::NA, kKC = C::KC, NBUF = C::NBUF;
   constexpr uint32_t STAGE = C::kStageBytes;
-  constexpr uint32_t IDESC = instr_desc(128, BN, 1u);
-
-  TileInfo ti;
+  constexpr uint32_t A_OP = kKC * C::kChunkA;  // bytes of one A operand per stage
+  constexpr uint32_t B_OFF = NA * A_OP;        // stage: [A gate][A up][B], kKC chunks each
+  constexpr uint32_t ACC = NA * BN;            // TMEM columns of one accumulator buffer
+  const int S = a.stages;
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
+  const int KB = (MODE == kGateUp ? a.H : a.I) / (64 * kKC);  // K steps per tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
   if (!a.plan_ready) {
     pdl_wait();
     pdl_trigger();
   }
-  if (!decode_tile(a, m_tiles, BN, ti)) {
+  const int total = a.nt_prefix[a.L] * m_tiles;
+  const bool stand_down = a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT);
+  if ((int)blockIdx.x >= total || stand_down) {
     pdl_wait();
     return;
   }
-  const int KB = (MODE == kGateUp ? a.H : a.I) / 64;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t bars = base + S * STAGE;  // full[S], empty[S], accf
+  const uint32_t bars = base + S * STAGE;  // full[S], empty[S], tfull[2], tempty[2]
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
-  const uint32_t accf = bars + 16u * S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + 16 * S + 8);
+  auto tfull = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto tempty = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + 8 * (2 * S + 4));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ep_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);  // written by epilogue warps only
+  float* wcol = reinterpret_cast<float*>(tmem_slot + 4);  // [BN] routing weights of the tile's pairs (down)
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull(b), 1);
+      mbar_init(tempty(b), 4);
+    }
     *abort_flag = 0;
+    *ep_abort = 0;
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -148,127 +201,190 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  const MapEntry* me = a.maps + ti.mapi;
-  const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
-
   if (warp == 4) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tensormap_acquire(wmap);
-      tma_prefetch_map(wmap);
-      tma_prefetch_map(&act_map);
       const uint64_t pol_w = l2_policy_evict_first();
-      // with the plan already complete, weight tiles for the first stages go
-      // out before waiting for the kernel that writes the activations
-      const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
-      for (int kb = 0; kb < npre; ++kb) {
-        const uint32_t st = base + kb * STAGE;
-        mbar_arrive_expect_tx(full(kb), STAGE);
-        tma_load_2d_hint(st, wmap, full(kb), kb * 64, ti.mt * 128, pol_w);
-        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(kb), kb * 64, a.I + ti.mt * 128, pol_w);
-      }
-      if (a.plan_ready) {
-        pdl_wait();
-        pdl_trigger();
-      }
-      for (int kb = 0; kb < npre; ++kb) tma_load_2d(base + kb * STAGE + NA * kABytes, &act_map, full(kb), kb * 64,
-                                                    ti.row0);
-      int kb = npre;
-      for (; kb < KB; ++kb) {
-        const int s = kb % S;
-        if (kb >= S && !mbar_wait(empty(s), ((kb / S) - 1) & 1)) {
-          *abort_flag = 1;
-          flag_status(a.status, MOE_DEV_TIMEOUT);
-          break;
+      int issued = 0;  // K steps issued so far (all tiles)
+      bool first = true;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile_at(a, m_tiles, BN, tile, ti);
+        const int wi = tile_width_index(ti.nvalid, BN);
+        const void* amap = &act.m[wi];
+        const uint32_t stage_tx = NA * A_OP + kKC * ((16u << wi) * 128u);
+        const MapEntry* me = a.maps + ti.mapi;
+        const void* wmap = MODE == kGateUp ? static_cast<const void*>(kKC == 1 ? &me->gu : &me->gu2)
+                                           : static_cast<const void*>(kKC == 1 ? &me->dn : &me->dn2);
+        tensormap_acquire(wmap);
+        int kb = 0;
+        if (first) {
+          first = false;
+          // the plan is complete: the first weight stages go out before waiting
+          // for the kernel that writes the activations
+          const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
+          for (int j = 0; j < npre; ++j) {
+            const uint32_t st = base + j * STAGE;
+            mbar_arrive_expect_tx(full(j), stage_tx);
+            tma_load_3d_hint(st, wmap, full(j), 0, ti.mt * 128, j * kKC, pol_w);
+            if (MODE == kGateUp) tma_load_3d_hint(st + A_OP, wmap, full(j), 0, a.I + ti.mt * 128, j * kKC, pol_w);
+          }
+          if (a.plan_ready) {
+            pdl_wait();
+            pdl_trigger();
+          }
+          for (int j = 0; j < npre; ++j) tma_load_3d(base + j * STAGE + B_OFF, amap, full(j), 0, ti.row0, j * kKC);
+          kb = npre;
+          issued = npre;
         }
-        if (*abort_flag) break;
-        const uint32_t st = base + s * STAGE;
-        mbar_arrive_expect_tx(full(s), STAGE);
-        tma_load_2d_hint(st, wmap, full(s), kb * 64, ti.mt * 128, pol_w);
-        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 64, a.I + ti.mt * 128, pol_w);
-        tma_load_2d(st + NA * kABytes, &act_map, full(s), kb * 64, ti.row0);
+        for (; kb < KB; ++kb, ++issued) {
+          const int s = issued % S;
+          if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
+            *abort_flag = 1;
+            flag_status(a.status, MOE_DEV_TIMEOUT);
+            break;
+          }
+          const uint32_t st = base + s * STAGE;
+          mbar_arrive_expect_tx(full(s), stage_tx);
+          tma_load_3d_hint(st, wmap, full(s), 0, ti.mt * 128, kb * kKC, pol_w);
+          if (MODE == kGateUp) tma_load_3d_hint(st + A_OP, wmap, full(s), 0, a.I + ti.mt * 128, kb * kKC, pol_w);
+          tma_load_3d(st + B_OFF, amap, full(s), 0, ti.row0, kb * kKC);
+        }
       }
-      // every load this thread issued has landed before the CTA may exit
-      for (int j = kb - S < 0 ? 0 : kb - S; j < kb; ++j) mbar_wait(full(j % S), (j / S) & 1);
+      // every copy this thread issued has landed before the CTA may exit
+      for (int g = issued - S < 0 ? 0 : issued - S; g < issued; ++g) mbar_wait(full(g % S), (g / S) & 1);
     } else if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
   } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
     if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
     if (lane == 0) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S;
-        if (!mbar_wait(full(s), (kb / S) & 1)) {
+      int consumed = 0, j = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+        const int buf = j % NBUF;
+        if (j >= NBUF && !mbar_wait(tempty(buf), ((j / NBUF) - 1) & 1)) {
           *abort_flag = 1;
           flag_status(a.status, MOE_DEV_TIMEOUT);
           break;
         }
         tc_fence_after();
-        const uint32_t st = base + s * STAGE;
+        const uint32_t d = tmem + buf * ACC;
+        TileInfo ti;
+        decode_tile_at(a, m_tiles, BN, tile, ti);
+        const int width = 16 << tile_width_index(ti.nvalid, BN);
+        const uint32_t idesc = instr_desc(128, width, 1u);
+        const uint32_t chunk_b = (uint32_t)width * 128u;  // a 3-D box lands its K chunks densely
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb, ++consumed) {
+          const int s = consumed % S;
+          if (!mbar_wait(full(s), (consumed / S) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = base + s * STAGE;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
-          const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
-          tc_mma_bf16(tmem, sw128_kmajor_desc(st + k * 32), bdesc, IDESC, acc);
-          if (MODE == kGateUp) tc_mma_bf16(tmem + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, IDESC, acc);
+          for (int c = 0; c < kKC; ++c) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t bdesc = sw128_kmajor_desc(st + B_OFF + c * chunk_b + k * 32);
+              const uint32_t acc = (kb | c | k) != 0 ? 1u : 0u;
+              tc_mma_bf16(d, sw128_kmajor_desc(st + c * C::kChunkA + k * 32), bdesc, idesc, acc);
+              if (MODE == kGateUp)
+                tc_mma_bf16(d + BN, sw128_kmajor_desc(st + A_OP + c * C::kChunkA + k * 32), bdesc, idesc, acc);
+            }
+          }
+          tc_commit(empty(s));
         }
-        tc_commit(empty(s));
+        tc_commit(tfull(buf));
+        if (!ok) {
+          *abort_flag = 1;
+          flag_status(a.status, MOE_DEV_TIMEOUT);
+          break;
+        }
       }
-      tc_commit(accf);
     }
   } else {
+    // ------------------------------------------------------------ epilogue (warps 0..3)
     if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
-    const bool ok = mbar_wait(accf, 0);
-    if (!ok) flag_status(a.status, MOE_DEV_TIMEOUT);
-    tc_fence_after();
-    __syncwarp();
-    if (ok && !*abort_flag) {
-      const int r = warp * 32 + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-      if (MODE == kGateUp) {
-        const int j = ti.mt * 128 + r;
-        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
+    const int r = warp * 32 + lane;
+    int j = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
+      const int buf = j % NBUF;
+      TileInfo ti;
+      decode_tile_at(a, m_tiles, BN, tile, ti);
+      if (MODE == kDown) {
+        // routing weights of this tile's pairs, once per tile
+        named_bar_sync(1, 128);  // previous tile's readers are done with wcol
+        for (int n = r; n < BN; n += 128) {
+          float wv = 0.0f;
+          if (n < ti.nvalid) {
+            const int p = ti.row0 + n;
+            wv = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
+          }
+          wcol[n] = wv;
+        }
+        named_bar_sync(1, 128);
+      }
+      int okv = 1;
+      if (lane == 0) okv = mbar_wait(tfull(buf), (j / NBUF) & 1) ? 1 : 0;
+      if (lane == 0 && !okv) *ep_abort = 1;
+      named_bar_sync(2, 128);  // the four epilogue warps leave the loop together or not at all
+      if (*ep_abort) {
+        flag_status(a.status, MOE_DEV_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int skip = __shfl_sync(0xffffffffu, *abort_flag ? 1 : 0, 0);  // warp-uniform around tcgen05.ld
+      if (!skip) {
+        const uint32_t tl = tmem + buf * ACC + (static_cast<uint32_t>(warp * 32) << 16);
+        if (MODE == kGateUp) {
+          const int jj = ti.mt * 128 + r;
+          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          if (c >= ti.nvalid) break;
-          uint32_t g[16], u[16];
-          tmem_ld16(tl + c, g);
-          tmem_ld16(tl + BN + c, u);
-          tmem_wait_ld();
+          for (int c = 0; c < BN; c += 16) {
+            if (c >= ti.nvalid) break;
+            uint32_t g[16], u[16];
+            tmem_ld16(tl + c, g);
+            tmem_ld16(tl + BN + c, u);
+            tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            if (c + q < ti.nvalid) {
-              const float gv = __uint_as_float(g[q]);
-              const float uv = __uint_as_float(u[q]);
-              const float hv = gv / (1.0f + expf(-gv)) * uv;
-              hout[(size_t)(ti.row0 + c + q) * a.I + j] = __float2bfloat16_rn(hv);
+            for (int q = 0; q < 16; ++q) {
+              if (c + q < ti.nvalid) {
+                const float gv = __uint_as_float(g[q]);
+                const float uv = __uint_as_float(u[q]);
+                const float hv = gv / (1.0f + expf(-gv)) * uv;
+                hout[(size_t)(ti.row0 + c + q) * a.I + jj] = __float2bfloat16_rn(hv);
+              }
             }
           }
-        }
-      } else {
-        const int o = ti.mt * 128 + r;
+        } else {
+          const int o = ti.mt * 128 + r;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          if (c >= ti.nvalid) break;
-          uint32_t v[16];
-          tmem_ld16(tl + c, v);
-          tmem_wait_ld();
+          for (int c = 0; c < BN; c += 16) {
+            if (c >= ti.nvalid) break;
+            uint32_t v[16];
+            tmem_ld16(tl + c, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            if (c + q < ti.nvalid) {
-              const int p = ti.row0 + c + q;
-              const float wgt = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
-              a.y_out[(size_t)p * a.H + o] = wgt * __uint_as_float(v[q]);
+            for (int q = 0; q < 16; ++q) {
+              if (c + q < ti.nvalid) a.y_out[(size_t)(ti.row0 + c + q) * a.H + o] = wcol[c + q] * __uint_as_float(v[q]);
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty(buf));
     }
   }
   tc_fence_before();
@@ -488,9 +604,9 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
 
 // ==================================================================== launch
 
-template <typename Kern>
-static cudaError_t launch_kernel(Kern kern, size_t smem, int threads, int grid, const CUtensorMap& map,
-                                 const GemmArgs& a, cudaStream_t s, bool pdl) {
+template <typename Kern, typename MapT>
+static cudaError_t launch_kernel(Kern kern, size_t smem, int threads, int grid, const MapT& map, const GemmArgs& a,
+                                 cudaStream_t s, bool pdl) {
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
@@ -498,22 +614,23 @@ static cudaError_t launch_kernel(Kern kern, size_t smem, int threads, int grid, 
 }
 
 template <int MODE, int BN>
-static cudaError_t launch_bf16(const CUtensorMap& map, GemmArgs a, int grid, cudaStream_t s, bool pdl) {
+static cudaError_t launch_bf16(const ActMaps& maps, GemmArgs a, int grid, cudaStream_t s, bool pdl) {
   using C = Bf16Cfg<MODE, BN>;
-  a.stages = a.est_tiles <= a.num_sms ? C::kStagesMax : C::kStagesTwo;
-  return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 192, grid, map, a, s, pdl);
+  a.stages = C::kStagesMax;
+  const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
+  return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 192, persistent, maps, a, s, pdl);
 }
 
 template <int MODE>
-static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const GemmArgs& a, int grid,
-                               cudaStream_t s, bool pdl) {
+static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const ActMaps* maps, const GemmArgs& a,
+                               int grid, cudaStream_t s, bool pdl) {
   if (wdtype == MOE_BF16) {
     switch (bn) {
-      case 16: return launch_bf16<MODE, 16>(map, a, grid, s, pdl);
-      case 32: return launch_bf16<MODE, 32>(map, a, grid, s, pdl);
-      case 64: return launch_bf16<MODE, 64>(map, a, grid, s, pdl);
-      case 128: return launch_bf16<MODE, 128>(map, a, grid, s, pdl);
-      case 256: return launch_bf16<MODE, 256>(map, a, grid, s, pdl);
+      case 16: return launch_bf16<MODE, 16>(*maps, a, grid, s, pdl);
+      case 32: return launch_bf16<MODE, 32>(*maps, a, grid, s, pdl);
+      case 64: return launch_bf16<MODE, 64>(*maps, a, grid, s, pdl);
+      case 128: return launch_bf16<MODE, 128>(*maps, a, grid, s, pdl);
+      case 256: return launch_bf16<MODE, 256>(*maps, a, grid, s, pdl);
     }
   } else {
     switch (bn) {
@@ -568,10 +685,10 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
   return 0;
 }
 
-cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const GemmArgs& a,
-                            int max_tiles, cudaStream_t s, bool pdl) {
-  if (mode == kGateUp) return launch_mode<kGateUp>(wdtype, bn, act_map, a, max_tiles, s, pdl);
-  return launch_mode<kDown>(wdtype, bn, act_map, a, max_tiles, s, pdl);
+cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const ActMaps* act_maps,
+                            const GemmArgs& a, int max_tiles, cudaStream_t s, bool pdl) {
+  if (mode == kGateUp) return launch_mode<kGateUp>(wdtype, bn, act_map, act_maps, a, max_tiles, s, pdl);
+  return launch_mode<kDown>(wdtype, bn, act_map, act_maps, a, max_tiles, s, pdl);
 }
 
 }  // namespace moe

@@ -16,13 +16,22 @@ namespace moe {
 // Per-slot TMA descriptors of one expert's weights (and FP8 scales), kept in
 // a device array that the FFN kernels index by slot.
 struct alignas(64) MapEntry {
-  CUtensorMap gu;  // w_gu [2I, H]: box {128 B of K, 128 rows}
-  CUtensorMap dn;  // w_dn [H, I]:  box {128 B of K, 128 rows}
+  // bf16: 3-D maps (64 elements, rows, K/64 chunks), box {64, 128, kc} with
+  //       kc = 1 (gu, dn) and kc = 2 (gu2, dn2);
+  // FP8:  2-D maps in gu / dn, box {128 B of K, 128 rows}.
+  CUtensorMap gu;   // w_gu [2I, H]
+  CUtensorMap dn;   // w_dn [H, I]
+  CUtensorMap gu2;
+  CUtensorMap dn2;
   const float* s_gu;
   const float* s_dn;
 };
 
 enum FfnMode { kGateUp = 0, kDown = 1 };
+
+// K chunks (of 64 bf16) per TMA copy in the bf16 FFN GEMMs: 2, except the
+// widest gate/up tile, whose stage would not fit twice in shared memory.
+constexpr int ffn_k_chunks(int mode, int bn) { return (mode == 0 && bn == 256) ? 1 : 2; }
 
 // Launches `kern` on `s`, with programmatic stream serialisation when pdl is
 // true (the kernel must then follow the pdl_wait / pdl_trigger rule).
@@ -71,11 +80,17 @@ struct GemmArgs {
   int num_sms;
 };
 
+// Activation-operand TMA descriptors for box heights 16, 32, 64, 128, 256
+// rows (the bf16 GEMMs pick, per tile, the smallest that holds its pairs).
+struct alignas(64) ActMaps {
+  CUtensorMap m[5];
+};
+
 // Launches one FFN GEMM (gate/up+SwiGLU or down*weight) over the tile list.
 // act_map is the TMA descriptor of the activation operand (x_perm or h);
 // max_tiles bounds the grid (CTAs past the real tile count exit at once).
-cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const GemmArgs& a,
-                            int max_tiles, cudaStream_t s, bool pdl);
+cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const ActMaps* act_maps,
+                            const GemmArgs& a, int max_tiles, cudaStream_t s, bool pdl);
 size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn);
 
 cudaError_t launch_router_logits(const void* x, const float* wr, const float* bias, int T, int H, int E,
