@@ -4,71 +4,95 @@
 // layers of 384 routed experts, top-k routing; "identical requests return
 // identical logits at any batch size" is the results-table "quality" row).
 //
-// Logit order (the contract both this kernel and the CPU oracle follow):
-// H is cut into 16 contiguous segments of L = H/16; segment s accumulates
-// fmaf(x[h], Wr[e][h], acc) from +0 over its h in increasing order; the 16
-// partials are summed by the pairwise tree p[s] += p[s+o], o = 8, 4, 2, 1,
-// which is exactly what an xor-butterfly over 16 lanes leaves in every lane;
-// then one fp32 add of bias[e]. A token's logits therefore depend on that
-// token alone, whatever the batch.
+// Logit order (the contract both these kernels and the CPU oracle follow):
+// h is cut into chunks of 8 (chunk c = h 8c..8c+7); lane j of a warp owns the
+// chunks c = j, j+32, j+64, ... and runs fmaf(x[h], Wr[e][h], acc) from +0
+// over them in increasing c (h increasing inside a chunk); the 32 lane
+// partials are then summed by the xor butterfly (offsets 16, 8, 4, 2, 1),
+// which leaves p[j] += p[j+o] (o = 16 .. 1) in every lane; then one fp32 add
+// of bias[e]. Every warp load of Wr or x is 32 consecutive 16-byte pieces,
+// and a token's logits depend on that token alone, whatever the batch.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-// One 16-lane group per (expert, token group); lane s owns segment s.
-// EPC experts per CTA, TG tokens per thread.
-template <int EPC, int TG>
-__global__ void __launch_bounds__(EPC * 16) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                                  const float* __restrict__ wr,
-                                                                  const float* __restrict__ bias, int T, int H,
-                                                                  int E, float* __restrict__ logits) {
-  const int s = threadIdx.x & 15;
-  const int e = blockIdx.x * EPC + (threadIdx.x >> 4);
-  const int t0 = blockIdx.y * TG;
-  const int L = H >> 4;
-  float acc[TG];
+// One warp per expert, TG tokens per warp; lane j owns chunks j, j+32, ...
+// U chunks per lane are loaded before any is used, so a warp keeps
+// U x (32 + 16 TG) bytes per lane in flight. Wr streams once per token
+// group with coalesced 512-byte warp loads; x comes through L1 (shared by
+// the CTA's warps, which all read the same tokens).
+template <int TG, int U>
+__device__ __forceinline__ void logits_warp(const uint16_t* __restrict__ x, const float* __restrict__ wrow, int T,
+                                            int H, int t0, float (&acc)[TG]) {
+  const int lane = threadIdx.x & 31;
+  const int ntok = min(TG, T - t0);
 #pragma unroll
   for (int i = 0; i < TG; ++i) acc[i] = 0.0f;
-
-  if (e < E) {
-    const float* w = wr + (size_t)e * H + (size_t)s * L;
-    const uint16_t* xs = x + (size_t)t0 * H + (size_t)s * L;
-    const int ntok = min(TG, T - t0);
-#pragma unroll 2
-    for (int h = 0; h < L; h += 8) {
-      const float4 wa = __ldg(reinterpret_cast<const float4*>(w + h));
-      const float4 wb = __ldg(reinterpret_cast<const float4*>(w + h + 4));
+  for (int hb = lane * 8; hb < H; hb += 256 * U) {
+    float4 wa[U], wb[U];
+    uint4 xv[U][TG];
 #pragma unroll
-      for (int i = 0; i < TG; ++i) {
-        if (i < ntok) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xs + (size_t)i * H + h));
-          float a = acc[i];
-          a = fmaf(__uint_as_float(xv.x << 16), wa.x, a);
-          a = fmaf(__uint_as_float(xv.x & 0xffff0000u), wa.y, a);
-          a = fmaf(__uint_as_float(xv.y << 16), wa.z, a);
-          a = fmaf(__uint_as_float(xv.y & 0xffff0000u), wa.w, a);
-          a = fmaf(__uint_as_float(xv.z << 16), wb.x, a);
-          a = fmaf(__uint_as_float(xv.z & 0xffff0000u), wb.y, a);
-          a = fmaf(__uint_as_float(xv.w << 16), wb.z, a);
-          a = fmaf(__uint_as_float(xv.w & 0xffff0000u), wb.w, a);
-          acc[i] = a;
+    for (int u = 0; u < U; ++u) {
+      const int h = hb + 256 * u;
+      if (h < H) {
+        wa[u] = __ldg(reinterpret_cast<const float4*>(wrow + h));
+        wb[u] = __ldg(reinterpret_cast<const float4*>(wrow + h + 4));
+#pragma unroll
+        for (int i = 0; i < TG; ++i)
+          if (i < ntok) xv[u][i] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + i) * H + h));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (hb + 256 * u < H) {
+#pragma unroll
+        for (int i = 0; i < TG; ++i) {
+          if (i < ntok) {
+            const uint4 v = xv[u][i];
+            float a = acc[i];
+            a = fmaf(__uint_as_float(v.x << 16), wa[u].x, a);
+            a = fmaf(__uint_as_float(v.x & 0xffff0000u), wa[u].y, a);
+            a = fmaf(__uint_as_float(v.y << 16), wa[u].z, a);
+            a = fmaf(__uint_as_float(v.y & 0xffff0000u), wa[u].w, a);
+            a = fmaf(__uint_as_float(v.z << 16), wb[u].x, a);
+            a = fmaf(__uint_as_float(v.z & 0xffff0000u), wb[u].y, a);
+            a = fmaf(__uint_as_float(v.w << 16), wb[u].z, a);
+            a = fmaf(__uint_as_float(v.w & 0xffff0000u), wb[u].w, a);
+            acc[i] = a;
+          }
         }
       }
     }
   }
-  // pairwise tree over the 16 segments (xor offsets stay inside the 16-lane group)
 #pragma unroll
   for (int i = 0; i < TG; ++i) {
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) acc[i] = acc[i] + __shfl_xor_sync(0xffffffffu, acc[i], o);
+    for (int o = 16; o >= 1; o >>= 1) acc[i] = acc[i] + __shfl_xor_sync(0xffffffffu, acc[i], o);
   }
-  if (s == 0 && e < E) {
+}
+
+// Loads in flight per lane for a token group of TG (registers: U (8 + 4 TG)).
+template <int TG>
+struct LogitsUnroll {
+  static constexpr int value = TG <= 2 ? 8 : (TG <= 4 ? 4 : 2);
+};
+
+template <int TG>
+__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                             const float* __restrict__ wr,
+                                                             const float* __restrict__ bias, int T, int H, int E,
+                                                             float* __restrict__ logits) {
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int t0 = blockIdx.y * TG;
+  if (e >= E) return;  // warp-uniform
+  float acc[TG];
+  logits_warp<TG, LogitsUnroll<TG>::value>(x, wr + (size_t)e * H, T, H, t0, acc);
+  if ((threadIdx.x & 31) == 0) {
     const float b = bias ? bias[e] : 0.0f;
 #pragma unroll
-    for (int i = 0; i < TG; ++i) {
+    for (int i = 0; i < TG; ++i)
       if (t0 + i < T) logits[(size_t)(t0 + i) * E + e] = bias ? acc[i] + b : acc[i];
-    }
   }
 }
 
@@ -76,15 +100,11 @@ cudaError_t launch_router_logits(const void* x, const float* wr, const float* bi
                                  float* logits, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   const uint16_t* xb = static_cast<const uint16_t*>(x);
+  const dim3 block(256);
   if (T <= 4) {
-    dim3 grid((E + 3) / 4, (T + 3) / 4);
-    router_logits_kernel<4, 4><<<grid, 64, 0, s>>>(xb, wr, bias, T, H, E, logits);
-  } else if (T <= 64) {
-    dim3 grid((E + 7) / 8, (T + 7) / 8);
-    router_logits_kernel<8, 8><<<grid, 128, 0, s>>>(xb, wr, bias, T, H, E, logits);
+    router_logits_kernel<4><<<dim3((E + 7) / 8, (T + 3) / 4), block, 0, s>>>(xb, wr, bias, T, H, E, logits);
   } else {
-    dim3 grid((E + 15) / 16, (T + 15) / 16);
-    router_logits_kernel<16, 16><<<grid, 256, 0, s>>>(xb, wr, bias, T, H, E, logits);
+    router_logits_kernel<8><<<dim3((E + 7) / 8, (T + 7) / 8), block, 0, s>>>(xb, wr, bias, T, H, E, logits);
   }
   return cudaGetLastError();
 }
@@ -244,136 +264,84 @@ cudaError_t launch_topk_warp(const float* logits, int T, int E, int K, int32_t* 
 }
 
 // ------------------------------------------------- decode-regime router --
-// One CTA per (EPC experts, TG tokens). The CTA's Wr segments (1 KB each at
-// H = 4096) and token segments are staged in padded shared memory by TMA bulk
-// copies -- one request per segment, all in flight at once -- then thread
-// (expert el, segment s) runs the segment's fma chain for every token of the
-// group and the 16-lane tree sums the partials (the same order as
-// router_logits_kernel). With fuse_topk, the last CTA of a token group (an
-// arrival counter) selects the group's top-k, one warp per token, and returns
-// the counter to zero; otherwise a top-k kernel follows.
-template <int EPC, int TG>
-__global__ void __launch_bounds__(EPC * 16) route_small_kernel(const uint16_t* __restrict__ x,
-                                                                const float* __restrict__ wr,
-                                                                const float* __restrict__ bias, int T, int H,
-                                                                int E, int K, float* __restrict__ logits,
-                                                                int32_t* __restrict__ idx, float* __restrict__ w,
-                                                                unsigned int* __restrict__ counters, int fuse_topk,
-                                                                int* status) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ __align__(8) uint64_t bar;
+// Same warp-per-expert logits (WPC experts per CTA, TG tokens per group); with
+// fuse_topk, the last CTA of each token group (an arrival counter) selects the
+// group's top-k, one warp per token, and returns the counter to zero;
+// otherwise a top-k kernel follows.
+template <int TG, int WPC>
+__global__ void __launch_bounds__(WPC * 32) route_small_kernel(const uint16_t* __restrict__ x,
+                                                           const float* __restrict__ wr,
+                                                           const float* __restrict__ bias, int T, int H, int E, int K,
+                                                           float* __restrict__ logits, int32_t* __restrict__ idx,
+                                                           float* __restrict__ w, unsigned int* __restrict__ counters,
+                                                           int fuse_topk) {
   __shared__ int s_last;
   pdl_trigger();  // first kernel of a forward: the next one may launch (it waits for us)
-  const int L = H >> 4;
-  const int wst = L + 4;  // padded floats per Wr segment row
-  const int xst = L + 8;  // padded bf16 per x segment row
-  float* sw = reinterpret_cast<float*>(sm);
-  uint16_t* sx = reinterpret_cast<uint16_t*>(sm + (size_t)EPC * 16 * wst * 4);
-  const int s = threadIdx.x & 15, el = threadIdx.x >> 4;
-  const int e0 = blockIdx.x * EPC;
-  const int e = e0 + el;
+  const int warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * WPC + warp;
   const int t0 = blockIdx.y * TG;
   const int ntok = min(TG, T - t0);
-  const int nexp = min(EPC, E - e0);
-  const uint32_t b = smem_u32(&bar);
-  if (threadIdx.x == 0) {
-    mbar_init(b, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(b, (uint32_t)(nexp * 16 * L * 4 + ntok * 16 * L * 2));
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < (nexp + ntok) * 16; i += blockDim.x) {
-    if (i < nexp * 16) {
-      const int ee = i >> 4, ss = i & 15;
-      bulk_load(smem_u32(sw + (size_t)i * wst), wr + (size_t)(e0 + ee) * H + (size_t)ss * L, L * 4, b);
-    } else {
-      const int j = i - nexp * 16, tt = j >> 4, ss = j & 15;
-      bulk_load(smem_u32(sx + (size_t)j * xst), x + (size_t)(t0 + tt) * H + (size_t)ss * L, L * 2, b);
+  if (e < E) {
+    float acc[TG];
+    logits_warp<TG, LogitsUnroll<TG>::value>(x, wr + (size_t)e * H, T, H, t0, acc);
+    if ((threadIdx.x & 31) == 0) {
+      const float b = bias ? bias[e] : 0.0f;
+#pragma unroll
+      for (int i = 0; i < TG; ++i)
+        if (i < ntok) logits[(size_t)(t0 + i) * E + e] = bias ? acc[i] + b : acc[i];
     }
-  }
-  if (!mbar_wait(b, 0)) flag_status(status, MOE_DEV_TIMEOUT);
-
-  float acc[TG];
-#pragma unroll
-  for (int i = 0; i < TG; ++i) acc[i] = 0.0f;
-  if (el < nexp) {
-    const float* wseg = sw + (size_t)(el * 16 + s) * wst;
-#pragma unroll 2
-    for (int h = 0; h < L; h += 8) {
-      const float4 wa = *reinterpret_cast<const float4*>(wseg + h);
-      const float4 wb = *reinterpret_cast<const float4*>(wseg + h + 4);
-#pragma unroll
-      for (int i = 0; i < TG; ++i) {
-        if (i < ntok) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(sx + (size_t)(i * 16 + s) * xst + h);
-          float a = acc[i];
-          a = fmaf(__uint_as_float(xv.x << 16), wa.x, a);
-          a = fmaf(__uint_as_float(xv.x & 0xffff0000u), wa.y, a);
-          a = fmaf(__uint_as_float(xv.y << 16), wa.z, a);
-          a = fmaf(__uint_as_float(xv.y & 0xffff0000u), wa.w, a);
-          a = fmaf(__uint_as_float(xv.z << 16), wb.x, a);
-          a = fmaf(__uint_as_float(xv.z & 0xffff0000u), wb.y, a);
-          a = fmaf(__uint_as_float(xv.w << 16), wb.z, a);
-          a = fmaf(__uint_as_float(xv.w & 0xffff0000u), wb.w, a);
-          acc[i] = a;
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < TG; ++i) {
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) acc[i] = acc[i] + __shfl_xor_sync(0xffffffffu, acc[i], o);
-  }
-  if (s == 0 && e < E) {
-    const float bv = bias ? bias[e] : 0.0f;
-#pragma unroll
-    for (int i = 0; i < TG; ++i)
-      if (i < ntok) logits[(size_t)(t0 + i) * E + e] = bias ? acc[i] + bv : acc[i];
   }
   if (!fuse_topk) return;
-  // ---- arrival: the last CTA of this token group runs the group's top-k
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = atomicAdd(counters + blockIdx.y, 1u) == gridDim.x - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int i = warp; i < ntok; i += nw) {
+  for (int i = warp; i < ntok; i += WPC) {
     const int t = t0 + i;
     topk_warp_any(logits + (size_t)t * E, E, K, idx + (size_t)t * K, w + (size_t)t * K);
   }
   if (threadIdx.x == 0) counters[blockIdx.y] = 0u;
 }
 
-template <int EPC, int TG>
+// Four warps per CTA: a 384-expert router spreads over 96 SMs.
+constexpr int kRsWarps = 4;
+
+template <int TG>
 static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
-                             float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, int* status,
-                             cudaStream_t s) {
-  const int L = H >> 4;
-  const size_t smem = (size_t)EPC * 16 * (L + 4) * 4 + (size_t)TG * 16 * (L + 8) * 2;
-  auto kern = route_small_kernel<EPC, TG>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                             float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, cudaStream_t s) {
+  dim3 grid((E + kRsWarps - 1) / kRsWarps, (T + TG - 1) / TG);
+  return launch_ex(route_small_kernel<TG, kRsWarps>, grid, dim3(kRsWarps * 32), 0, s, false, static_cast<const uint16_t*>(x), wr, bias,
+                   T, H, E, K, logits, idx, w, counters, fuse);
+}
+
+// T <= 8: logits + fused top-k in one launch; up to 64 tokens: logits in
+// 8-token groups, then the warp top-k kernel (programmatic launch).
+cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
+                               float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
+                               cudaStream_t s, bool pdl) {
+  (void)status;
+  if (T <= 0) return cudaSuccess;
+  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
+  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
+  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
+  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
+  cudaError_t err = launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, s);
   if (err != cudaSuccess) return err;
-  dim3 grid((E + EPC - 1) / EPC, (T + TG - 1) / TG);
-  return launch_ex(kern, grid, dim3(EPC * 16), smem, s, false, static_cast<const uint16_t*>(x), wr, bias, T, H, E,
-                   K, logits, idx, w, counters, fuse, status);
+  return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
 }
 
 // ------------------------------------------------ prefill-regime router --
-// Logits as a register-tiled fp32 GEMM in the same order. CTA tile: 32 tokens
-// x 32 experts, 256 threads. Lane s = segment (two 16-lane groups per warp);
-// group g = 2 warp + lane/16 owns an 8-token x 8-expert tile of segment-s
-// partials (64 accumulators). Each stage brings RC consecutive h of every
-// segment, for the CTA's 32 tokens and 32 experts, into padded shared memory
-// (cp.async, two buffers); the h loop runs in increasing order inside each
-// segment, so every partial is the same fma chain as in router_logits_kernel,
-// and the 16-lane tree at the end sums them the same way.
-constexpr int kRgT = 32, kRgE = 32, kRgC = 16;
-constexpr int kRgXs = kRgC + 8;  // bf16 per padded (token, segment) row
-constexpr int kRgWs = kRgC + 4;  // floats per padded (expert, segment) row
-constexpr size_t kRgStageBytes = (size_t)kRgT * 16 * kRgXs * 2 + (size_t)kRgE * 16 * kRgWs * 4;
+// Register-tiled fp32 GEMM in the same order. CTA tile: 32 tokens x 16
+// experts, 8 warps as 4 token groups x 2 expert groups; a warp owns 8 tokens
+// x 8 experts and its lane j keeps the 64 lane-j partials (chunks j, j+32,
+// ...). Each stage holds 256 consecutive h of the tile's tokens and experts
+// in shared memory (cp.async, two buffers): token rows as stored, each Wr row
+// split into its chunks' first halves then second halves so that the 32
+// lanes' 16-byte reads are consecutive.
+constexpr int kRgT = 32, kRgE = 16;
+constexpr size_t kRgStageBytes = (size_t)kRgT * 256 * 2 + (size_t)kRgE * 256 * 4;
 
 __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
                                                              const float* __restrict__ wr,
@@ -382,29 +350,24 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
   extern __shared__ __align__(16) uint8_t sm[];
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int s = lane & 15, g = warp * 2 + (lane >> 4);
-  const int tt0 = (g >> 2) * 8, ee0 = (g & 3) * 8;
+  const int tt0 = (warp >> 1) * 8, ee0 = (warp & 1) * 8;
   const int tb = blockIdx.y * kRgT, eb = blockIdx.x * kRgE;
-  const int L = H >> 4, nsteps = L / kRgC;
+  const int nsteps = H / 256;
   auto xs = [&](int buf) { return reinterpret_cast<uint16_t*>(sm + buf * kRgStageBytes); };
-  auto ws = [&](int buf) {
-    return reinterpret_cast<float*>(sm + buf * kRgStageBytes + (size_t)kRgT * 16 * kRgXs * 2);
-  };
+  auto ws = [&](int buf) { return reinterpret_cast<float*>(sm + buf * kRgStageBytes + (size_t)kRgT * 256 * 2); };
   auto load_stage = [&](int st, int buf) {
-    const int h0 = st * kRgC;
+    const int h0 = st * 256;
     uint16_t* xd = xs(buf);
     float* wd = ws(buf);
-    // x: (token, segment, 2 x 16-byte parts); rows past T re-read row T-1 (results discarded)
-    for (int c = tid; c < kRgT * 16 * 2; c += 256) {
-      const int part = c & 1, ts = c >> 1, ss = ts & 15, t = ts >> 4;
-      const int row = min(tb + t, T - 1);
-      cp_async16(xd + (size_t)ts * kRgXs + part * 8, x + (size_t)row * H + (size_t)ss * L + h0 + part * 8);
+    for (int c = tid; c < kRgT * 32; c += 256) {  // token row: 32 x 16 B
+      const int t = c >> 5, part = c & 31;
+      const int row = min(tb + t, T - 1);  // rows past T re-read row T-1 (results discarded)
+      cp_async16(xd + (size_t)t * 256 + part * 8, x + (size_t)row * H + h0 + part * 8);
     }
-    // Wr: (expert, segment, 4 x 16-byte parts)
-    for (int c = tid; c < kRgE * 16 * 4; c += 256) {
-      const int part = c & 3, es = c >> 2, ss = es & 15, e = es >> 4;
+    for (int c = tid; c < kRgE * 64; c += 256) {  // expert row: 64 x 16 B (32 chunks x 2 halves)
+      const int e = c >> 6, q = c & 63, chunk = q >> 1, half = q & 1;
       const int row = min(eb + e, E - 1);
-      cp_async16(wd + (size_t)es * kRgWs + part * 4, wr + (size_t)row * H + (size_t)ss * L + h0 + part * 4);
+      cp_async16(wd + (size_t)e * 256 + half * 128 + chunk * 4, wr + (size_t)row * H + h0 + q * 4);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
@@ -427,27 +390,36 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
     __syncthreads();
     const uint16_t* xb = xs(buf);
     const float* wb = ws(buf);
+    float xf[8][8];
 #pragma unroll
-    for (int hh = 0; hh < kRgC; hh += 4) {
-      uint2 xv[8];
-      float4 wv[8];
+    for (int i = 0; i < 8; ++i) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xb + (size_t)(tt0 + i) * 256 + lane * 8);
+      xf[i][0] = __uint_as_float(v.x << 16);
+      xf[i][1] = __uint_as_float(v.x & 0xffff0000u);
+      xf[i][2] = __uint_as_float(v.y << 16);
+      xf[i][3] = __uint_as_float(v.y & 0xffff0000u);
+      xf[i][4] = __uint_as_float(v.z << 16);
+      xf[i][5] = __uint_as_float(v.z & 0xffff0000u);
+      xf[i][6] = __uint_as_float(v.w << 16);
+      xf[i][7] = __uint_as_float(v.w & 0xffff0000u);
+    }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) xv[i] = *reinterpret_cast<const uint2*>(xb + (size_t)((tt0 + i) * 16 + s) * kRgXs + hh);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) wv[j] = *reinterpret_cast<const float4*>(wb + (size_t)((ee0 + j) * 16 + s) * kRgWs + hh);
+    for (int j = 0; j < 8; ++j) {
+      const float* wrow = wb + (size_t)(ee0 + j) * 256;
+      const float4 wa = *reinterpret_cast<const float4*>(wrow + lane * 4);
+      const float4 wc = *reinterpret_cast<const float4*>(wrow + 128 + lane * 4);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float x0 = __uint_as_float(xv[i].x << 16), x1 = __uint_as_float(xv[i].x & 0xffff0000u);
-        const float x2 = __uint_as_float(xv[i].y << 16), x3 = __uint_as_float(xv[i].y & 0xffff0000u);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float a = acc[i][j];
-          a = fmaf(x0, wv[j].x, a);
-          a = fmaf(x1, wv[j].y, a);
-          a = fmaf(x2, wv[j].z, a);
-          a = fmaf(x3, wv[j].w, a);
-          acc[i][j] = a;
-        }
+        float a = acc[i][j];
+        a = fmaf(xf[i][0], wa.x, a);
+        a = fmaf(xf[i][1], wa.y, a);
+        a = fmaf(xf[i][2], wa.z, a);
+        a = fmaf(xf[i][3], wa.w, a);
+        a = fmaf(xf[i][4], wc.x, a);
+        a = fmaf(xf[i][5], wc.y, a);
+        a = fmaf(xf[i][6], wc.z, a);
+        a = fmaf(xf[i][7], wc.w, a);
+        acc[i][j] = a;
       }
     }
     __syncthreads();
@@ -457,8 +429,8 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
 #pragma unroll
     for (int j = 0; j < 8; ++j)
 #pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) acc[i][j] = acc[i][j] + __shfl_xor_sync(0xffffffffu, acc[i][j], o);
-  if (s == 0) {
+      for (int o = 16; o >= 1; o >>= 1) acc[i][j] = acc[i][j] + __shfl_xor_sync(0xffffffffu, acc[i][j], o);
+  if (lane == 0) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int t = tb + tt0 + i;
@@ -475,28 +447,13 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
 cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias, int T, int H, int E,
                               float* logits, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  if ((H >> 4) % kRgC != 0) return launch_router_logits(x, wr, bias, T, H, E, logits, s);
+  if (H % 256 != 0) return launch_router_logits(x, wr, bias, T, H, E, logits, s);
   const size_t smem = 2 * kRgStageBytes;
   cudaError_t err = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((E + kRgE - 1) / kRgE, (T + kRgT - 1) / kRgT);
   return launch_ex(route_gemm_kernel, grid, dim3(256), smem, s, false, static_cast<const uint16_t*>(x), wr, bias, T,
                    H, E, logits);
-}
-
-// T <= 4: logits + fused top-k in one launch; up to 64 tokens: logits in
-// 16-token groups, then the warp top-k kernel (programmatic launch).
-cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
-                               float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl) {
-  if (T <= 0) return cudaSuccess;
-  if (T <= 2) return launch_rs<2, 2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
-  if (T <= 4) return launch_rs<4, 4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
-  cudaError_t err;
-  if (T <= 8) err = launch_rs<4, 8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, status, s);
-  else err = launch_rs<4, 16>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, status, s);
-  if (err != cudaSuccess) return err;
-  return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
 }
 
 }  // namespace moe

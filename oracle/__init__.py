@@ -78,11 +78,11 @@ def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------- steps --
 
 def router_logits(x_u16: np.ndarray, wr: np.ndarray, bias=None, threads: int = 0) -> np.ndarray:
-    """fp32 logits [T, E] in the specified 16-segment order (+ bias)."""
+    """fp32 logits [T, E] in the specified 32-lane interleaved order (+ bias)."""
     lib = _load()
     T, H = x_u16.shape
     E = wr.shape[0]
-    assert H % 16 == 0
+    assert H % 8 == 0
     wr = np.ascontiguousarray(wr, dtype=np.float32)
     out = np.empty((T, E), dtype=np.float32)
     b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)

@@ -27,10 +27,11 @@
  * Reading of the layer where the definition leaves a step open (each one is
  * listed with its reason in the design notes):
  *   - Logit reduction order (needed for bit-exact top-k across two
- *     implementations): H is cut into 16 contiguous segments of H/16; segment
- *     s accumulates fmaf(f32(x[h]), Wr[e][h], acc) from +0 over its h in
- *     increasing order; the 16 partials are then summed pairwise,
- *     p[s] += p[s+o] for o = 8, 4, 2, 1 (s < o); the logit is p[0], then
+ *     implementations): h is cut into chunks of 8 (chunk c = h 8c..8c+7);
+ *     lane j of 32 owns the chunks c = j, j+32, j+64, ... and accumulates
+ *     fmaf(f32(x[h]), Wr[e][h], acc) from +0 over its chunks in increasing c,
+ *     h increasing inside a chunk; the 32 partials are then summed pairwise,
+ *     p[j] += p[j+o] for o = 16, 8, 4, 2, 1 (j < o); the logit is p[0], then
  *     + bias[e] (one fp32 add) when a bias is given.
  *   - Top-k runs on the logits (softmax is monotone, so the set is the same
  *     in exact arithmetic, and no exp() rounding can flip an index).
@@ -146,23 +147,24 @@ void oracle_quant_e4m3(const uint16_t* src, int rows, int cols, int br, uint8_t*
 
 /* ------------------------------------------------------------- router -- */
 
-#define SEGMENTS 16
+#define LANES 32
+#define CHUNK 8
 
 /* One logit in the specified order (see the header comment). */
 static float logit_one(const uint16_t* xrow, const float* wrow, int H) {
-  float p[SEGMENTS];
-  int L = H / SEGMENTS;
-  for (int s = 0; s < SEGMENTS; ++s) {
+  float p[LANES];
+  for (int j = 0; j < LANES; ++j) {
     float acc = 0.0f;
-    for (int h = s * L; h < (s + 1) * L; ++h) acc = fmaf(bf16_to_f32(xrow[h]), wrow[h], acc);
-    p[s] = acc;
+    for (int c = j; c * CHUNK < H; c += LANES)
+      for (int h = c * CHUNK; h < (c + 1) * CHUNK; ++h) acc = fmaf(bf16_to_f32(xrow[h]), wrow[h], acc);
+    p[j] = acc;
   }
-  for (int o = SEGMENTS / 2; o >= 1; o /= 2)
-    for (int s = 0; s < o; ++s) p[s] = p[s] + p[s + o];
+  for (int o = LANES / 2; o >= 1; o /= 2)
+    for (int j = 0; j < o; ++j) p[j] = p[j] + p[j + o];
   return p[0];
 }
 
-/* logits [T, E] fp32. H must be a multiple of 16. bias may be NULL. */
+/* logits [T, E] fp32. H must be a multiple of 8. bias may be NULL. */
 void oracle_router_logits(const uint16_t* x, const float* wr, const float* bias, int T, int H, int E,
                           float* logits, int threads) {
 #ifdef _OPENMP
