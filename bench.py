@@ -445,7 +445,7 @@ def run_profile_case(kind):
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    E_s, T_s = (32, 64) if kind == "t64" else (8, 1)
+    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048)}[kind]
     layer = M.MoeLayer(H, E_s, K, I, device=device)
     keep = []
     for e in range(E_s):
@@ -453,9 +453,10 @@ def run_profile_case(kind):
         layer.register(e, g, d)
         keep.append((g, d))
     wr = synth.router_weight(E_s, H, seed=SEED, device=device)
+    bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind == "p2048" else None
     x = synth.tokens(T_s, H, seed=SEED, device=device)
     for _ in range(3):
-        layer.forward(x, wr, None)
+        layer.forward(x, wr, bias)
     torch.cuda.synchronize()
     st = layer.status()
     print(json.dumps({"profile_case": f"E={E_s} H=4096 I=2048 K=8 T={T_s} bf16", "status": st}))
@@ -568,7 +569,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:

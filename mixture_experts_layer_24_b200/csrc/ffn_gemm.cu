@@ -70,7 +70,7 @@ struct Fp8Cfg {
 };
 
 struct TileInfo {
-  int e, mapi, mt, row0, nvalid;
+  int e, mapi, mt, row0, nvalid, nti;  // nti: N tiles of this expert (readers of each weight tile)
 };
 
 // Finds this CTA's (expert, M tile, N tile); false if the CTA has no tile.
@@ -94,6 +94,7 @@ __device__ __forceinline__ bool decode_tile(const GemmArgs& a, int m_tiles, int 
   ti.mt = mt;
   ti.row0 = a.offsets[ti.e] + nt * bn;
   ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
+  ti.nti = nti;
   return true;
 }
 
@@ -113,6 +114,7 @@ __device__ __forceinline__ void decode_tile_at(const GemmArgs& a, int m_tiles, i
   ti.mt = mt;
   ti.row0 = a.offsets[ti.e] + nt * bn;
   ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
+  ti.nti = nti;
 }
 
 __device__ __forceinline__ void tensormap_acquire(const void* map) {
@@ -204,7 +206,11 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
+      // Weights: evict-first when the tile is the weight rows' only reader;
+      // an expert with several N tiles has each weight tile read by all of
+      // them (close together in time), so there the lines keep the normal
+      // policy and the later readers hit L2.
+      const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
       int issued = 0;  // K steps issued so far (all tiles)
       bool first = true;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -213,6 +219,7 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
         const int wi = tile_width_index(ti.nvalid, BN);
         const void* amap = &act.m[wi];
         const uint32_t stage_tx = NA * A_OP + kKC * ((16u << wi) * 128u);
+        const uint64_t pol_w = ti.nti > 1 ? pol_shared : pol_once;
         const MapEntry* me = a.maps + ti.mapi;
         const void* wmap = MODE == kGateUp ? static_cast<const void*>(kKC == 1 ? &me->gu : &me->gu2)
                                            : static_cast<const void*>(kKC == 1 ? &me->dn : &me->dn2);
@@ -474,7 +481,8 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
       tensormap_acquire(wmap);
       tma_prefetch_map(wmap);
       tma_prefetch_map(&act_map);
-      const uint64_t pol_w = l2_policy_evict_first();
+      // evict-first only when this tile is the weight rows' sole reader
+      const uint64_t pol_w = ti.nti > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
       int kb = 0;
       for (; kb < KB; ++kb) {
         const int s = kb % S;
@@ -643,7 +651,9 @@ static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const
 }
 
 int ffn_block_n(int T, int wdtype) {
-  int bn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256;
+  // 128 at most: gate/up at 128 keeps two TMEM accumulators (the epilogue of
+  // one tile overlaps the next tile's MMAs) and four pipeline stages.
+  int bn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
   if (wdtype == MOE_FP8_E4M3_B128 && bn > 64) bn = 64;
   return bn;
 }

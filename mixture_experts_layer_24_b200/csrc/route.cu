@@ -333,17 +333,18 @@ cudaError_t launch_route_small(const void* x, const float* wr, const float* bias
 }
 
 // ------------------------------------------------ prefill-regime router --
-// Register-tiled fp32 GEMM in the same order. CTA tile: 32 tokens x 16
-// experts, 8 warps as 4 token groups x 2 expert groups; a warp owns 8 tokens
+// Register-tiled fp32 GEMM in the same order. CTA tile: 48 tokens x 16
+// experts, 12 warps as 6 token groups x 2 expert groups; a warp owns 8 tokens
 // x 8 experts and its lane j keeps the 64 lane-j partials (chunks j, j+32,
 // ...). Each stage holds 256 consecutive h of the tile's tokens and experts
-// in shared memory (cp.async, two buffers): token rows as stored, each Wr row
+// in shared memory (cp.async, kRgStages buffers, kRgStages - 1 in flight):
+// token rows as stored, each Wr row
 // split into its chunks' first halves then second halves so that the 32
 // lanes' 16-byte reads are consecutive.
-constexpr int kRgT = 32, kRgE = 16;
+constexpr int kRgT = 48, kRgE = 16, kRgStages = 3, kRgThreads = 384;
 constexpr size_t kRgStageBytes = (size_t)kRgT * 256 * 2 + (size_t)kRgE * 256 * 4;
 
-__global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(kRgThreads, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
                                                              const float* __restrict__ wr,
                                                              const float* __restrict__ bias, int T, int H, int E,
                                                              float* __restrict__ logits) {
@@ -359,17 +360,16 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
     const int h0 = st * 256;
     uint16_t* xd = xs(buf);
     float* wd = ws(buf);
-    for (int c = tid; c < kRgT * 32; c += 256) {  // token row: 32 x 16 B
+    for (int c = tid; c < kRgT * 32; c += kRgThreads) {  // token row: 32 x 16 B
       const int t = c >> 5, part = c & 31;
       const int row = min(tb + t, T - 1);  // rows past T re-read row T-1 (results discarded)
       cp_async16(xd + (size_t)t * 256 + part * 8, x + (size_t)row * H + h0 + part * 8);
     }
-    for (int c = tid; c < kRgE * 64; c += 256) {  // expert row: 64 x 16 B (32 chunks x 2 halves)
+    for (int c = tid; c < kRgE * 64; c += kRgThreads) {  // expert row: 64 x 16 B (32 chunks x 2 halves)
       const int e = c >> 6, q = c & 63, chunk = q >> 1, half = q & 1;
       const int row = min(eb + e, E - 1);
       cp_async16(wd + (size_t)e * 256 + half * 128 + chunk * 4, wr + (size_t)row * H + h0 + q * 4);
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
   float acc[8][8];
@@ -378,15 +378,19 @@ __global__ void __launch_bounds__(256, 1) route_gemm_kernel(const uint16_t* __re
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
 
-  load_stage(0, 0);
+#pragma unroll
+  for (int st = 0; st < kRgStages - 1; ++st) {
+    if (st < nsteps) load_stage(st, st);
+    asm volatile("cp.async.commit_group;" ::: "memory");  // empty groups keep the count uniform
+  }
   for (int st = 0; st < nsteps; ++st) {
-    const int buf = st & 1;
-    if (st + 1 < nsteps) {
-      load_stage(st + 1, buf ^ 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    const int buf = st % kRgStages;
+    {
+      const int nx = st + kRgStages - 1;  // its buffer was last read in iteration st - 1
+      if (nx < nsteps) load_stage(nx, nx % kRgStages);
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
+    asm volatile("cp.async.wait_group %0;" ::"n"(kRgStages - 1) : "memory");
     __syncthreads();
     const uint16_t* xb = xs(buf);
     const float* wb = ws(buf);
@@ -448,11 +452,11 @@ cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias,
                               float* logits, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
   if (H % 256 != 0) return launch_router_logits(x, wr, bias, T, H, E, logits, s);
-  const size_t smem = 2 * kRgStageBytes;
+  const size_t smem = kRgStages * kRgStageBytes;
   cudaError_t err = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((E + kRgE - 1) / kRgE, (T + kRgT - 1) / kRgT);
-  return launch_ex(route_gemm_kernel, grid, dim3(256), smem, s, false, static_cast<const uint16_t*>(x), wr, bias, T,
+  return launch_ex(route_gemm_kernel, grid, dim3(kRgThreads), smem, s, false, static_cast<const uint16_t*>(x), wr, bias, T,
                    H, E, logits);
 }
 
