@@ -445,13 +445,20 @@ def run_profile_case(kind):
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048)}[kind]
-    layer = M.MoeLayer(H, E_s, K, I, device=device)
+    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64)}[kind]
+    fp8 = kind == "f64"
+    layer = M.MoeLayer(H, E_s, K, I, wdtype=M.MOE_FP8_E4M3_B128 if fp8 else M.MOE_BF16, device=device)
     keep = []
     for e in range(E_s):
         g, d = synth.expert_weights(e, H, I, seed=SEED, device=device)
-        layer.register(e, g, d)
-        keep.append((g, d))
+        if fp8:
+            w = quantize_expert(M, g, d, device)
+            del g, d
+            layer.register(e, *w)
+            keep.append(w)
+        else:
+            layer.register(e, g, d)
+            keep.append((g, d))
     wr = synth.router_weight(E_s, H, seed=SEED, device=device)
     bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind == "p2048" else None
     x = synth.tokens(T_s, H, seed=SEED, device=device)
@@ -464,6 +471,18 @@ def run_profile_case(kind):
     return 1 if st else 0
 
 
+def quantize_expert(M, g, d, device):
+    """(codes_gu, codes_dn, scales_gu, scales_dn): e4m3 with 128x128 block
+    scales, quantised on the GPU by the library's quantiser."""
+    qg = torch.empty((2 * I, H), dtype=torch.uint8, device=device)
+    sg = torch.empty((2 * I // 128, H // 128), dtype=torch.float32, device=device)
+    qd = torch.empty((H, I), dtype=torch.uint8, device=device)
+    sd = torch.empty((H // 128, I // 128), dtype=torch.float32, device=device)
+    M.moe_quantize_e4m3(g, 2 * I, H, 128, qg, sg)
+    M.moe_quantize_e4m3(d, H, I, 128, qd, sd)
+    return qg, qd, sg, sd
+
+
 def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
     """The same layer with e4m3 experts (128x128 block scales, quantised on the
     GPU from the bf16 weights): decode B=1, 8, 64 and a 4096-token chunk."""
@@ -471,15 +490,9 @@ def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
     layer = M.MoeLayer(H, E, K, I, wdtype=M.MOE_FP8_E4M3_B128, device=device)
     qkeep = []
     for e in range(E):
-        g, d = keep[e]
-        qg = torch.empty((2 * I, H), dtype=torch.uint8, device=device)
-        sg = torch.empty((2 * I // 128, H // 128), dtype=torch.float32, device=device)
-        qd = torch.empty((H, I), dtype=torch.uint8, device=device)
-        sd = torch.empty((H // 128, I // 128), dtype=torch.float32, device=device)
-        M.moe_quantize_e4m3(g, 2 * I, H, 128, qg, sg)
-        M.moe_quantize_e4m3(d, H, I, 128, qd, sd)
-        layer.register(e, qg, qd, sg, sd)
-        qkeep.append((qg, sg, qd, sd))
+        w = quantize_expert(M, keep[e][0], keep[e][1], device)
+        layer.register(e, *w)
+        qkeep.append(w)
     torch.cuda.synchronize()
     layer.workspace(4096)
     fp8_bytes = 3 * I * H + 2 * (2 * I // 128) * (H // 128) * 4 + 2 * (H // 128) * (I // 128) * 4
@@ -569,7 +582,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:

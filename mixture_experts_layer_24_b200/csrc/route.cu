@@ -412,18 +412,13 @@ __global__ void __launch_bounds__(kRgThreads, 1) route_gemm_kernel(const uint16_
       const float* wrow = wb + (size_t)(ee0 + j) * 256;
       const float4 wa = *reinterpret_cast<const float4*>(wrow + lane * 4);
       const float4 wc = *reinterpret_cast<const float4*>(wrow + 128 + lane * 4);
+      const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wc.x, wc.y, wc.z, wc.w};
+      // h-element outer, token inner: eight independent chains between two
+      // dependent FMAs (each acc still takes its eight FMAs in h order)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float a = acc[i][j];
-        a = fmaf(xf[i][0], wa.x, a);
-        a = fmaf(xf[i][1], wa.y, a);
-        a = fmaf(xf[i][2], wa.z, a);
-        a = fmaf(xf[i][3], wa.w, a);
-        a = fmaf(xf[i][4], wc.x, a);
-        a = fmaf(xf[i][5], wc.y, a);
-        a = fmaf(xf[i][6], wc.z, a);
-        a = fmaf(xf[i][7], wc.w, a);
-        acc[i][j] = a;
+      for (int q = 0; q < 8; ++q) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i][j] = fmaf(xf[i][q], wv[q], acc[i][j]);
       }
     }
     __syncthreads();
