@@ -112,12 +112,11 @@ size_t moe_workspace_size(const moe_ctx_t* ctx, int T);
 /* Router: logits in the fixed order below, top-k, renormalised weights.
  *   x [T, H] bf16, w_router [E, H] fp32, logit_bias [E] fp32 or NULL.
  *   topk_idx [T, K] int32 out (by logit desc, expert asc), topk_w [T, K] fp32 out.
- * Logit order: H is cut into chunks of 8 (chunk c = h 8c..8c+7); partial j
- * (j = 0..31) accumulates fmaf(x[h], Wr[e][h], acc) from +0 over chunks
- * c = j, j+32, j+64, ... in increasing c (increasing h inside a chunk); the
- * 32 partials are summed pairwise (p[j] += p[j+o], o = 16, 8, 4, 2, 1); then
- * + bias[e] (one fp32 add). H must be a multiple of 8. Ties between equal
- * logits (+0 == -0) go to the lower expert index.
+ * Logit order: partial j (j = 0..31) accumulates fmaf(x[h], Wr[e][h], acc)
+ * from +0 over h = j, j+32, j+64, ... in increasing h; the 32 partials are
+ * summed pairwise (p[j] += p[j+o], o = 16, 8, 4, 2, 1: an xor butterfly's
+ * lane 0); then + bias[e] (one fp32 add). Ties between equal logits
+ * (+0 == -0) go to the lower expert index.
  * Weights: fp32 expf(l_k - l_0), summed k ascending, then one IEEE divide. */
 moe_status_t moe_route(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, moe_stream_t stream);

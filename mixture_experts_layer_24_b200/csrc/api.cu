@@ -272,15 +272,20 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
   CUtensorMap xmap, hmap;
-  ActMaps xmaps, hmaps;  // bf16: one map per tile box height 16 .. bn
+  ActMaps xmaps, hmaps;  // one activation map per tile box height 16 .. bn
+  std::memset(&xmaps, 0, sizeof(xmaps));
+  std::memset(&hmaps, 0, sizeof(hmaps));
   moe_status_t st = MOE_OK;
   if (fp8) {
-    st = encode_2d(ctx, &xmap, at<void>(ws, W.x_perm), true, c.hidden, P, bn);
-    if (st != MOE_OK) return st;
-    st = encode_2d(ctx, &hmap, at<void>(ws, W.hq), true, c.intermediate, P, bn);
+    for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
+      st = encode_2d(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), true, c.hidden, P, rows);
+      if (st != MOE_OK) return st;
+      st = encode_2d(ctx, &hmaps.m[i], at<void>(ws, W.hq), true, c.intermediate, P, rows);
+      if (st != MOE_OK) return st;
+    }
+    xmap = xmaps.m[0];
+    hmap = hmaps.m[0];
   } else {
-    std::memset(&xmaps, 0, sizeof(xmaps));
-    std::memset(&hmaps, 0, sizeof(hmaps));
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
       st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, ffn_k_chunks(kGateUp, bn));
       if (st != MOE_OK) return st;

@@ -20,19 +20,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   const int32_t* iv = inv + (size_t)t * K;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   bool have = false;
-#pragma unroll 4
-  for (int k = 0; k < K; ++k) {
-    const int p = __ldg(iv + k);
-    if (p < 0) continue;  // a pair dropped for an invalid expert id contributes nothing
-    const float4 a = __ldg(y + (size_t)p * H4 + v);
-    if (!have) {
-      acc = a;
-      have = true;
-    } else {
-      acc.x = acc.x + a.x;
-      acc.y = acc.y + a.y;
-      acc.z = acc.z + a.z;
-      acc.w = acc.w + a.w;
+  // eight pairs at a time: their inv entries, then their rows, are loaded
+  // before any is added; the adds run k ascending as before
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    int pk[8];
+    float4 a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) pk[u] = k0 + u < K ? __ldg(iv + k0 + u) : -1;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (pk[u] >= 0) a[u] = __ldg(y + (size_t)pk[u] * H4 + v);  // p < 0: a dropped pair contributes nothing
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (pk[u] < 0) continue;
+      if (!have) {
+        acc = a[u];
+        have = true;
+      } else {
+        acc.x = acc.x + a[u].x;
+        acc.y = acc.y + a[u].y;
+        acc.z = acc.z + a[u].z;
+        acc.w = acc.w + a[u].w;
+      }
     }
   }
   const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);

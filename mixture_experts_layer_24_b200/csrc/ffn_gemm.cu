@@ -48,7 +48,9 @@ struct Bf16Cfg {
   static constexpr uint32_t kChunkA = kABytes;     // 128 rows x 128 B
   static constexpr uint32_t kChunkB = BN * 128;    // BN rows x 128 B
   static constexpr uint32_t kStageBytes = KC * (NA * kChunkA + kChunkB);
-  static constexpr int kStagesFit = (200 * 1024) / kStageBytes;
+  // up to 220 KB of stages (227 KB per CTA at most; one CTA per SM): three
+  // two-chunk stages at BN <= 32
+  static constexpr int kStagesFit = (220 * 1024) / kStageBytes;
   static constexpr int kStagesMax = kStagesFit > 8 ? 8 : kStagesFit;
   // two accumulator buffers whenever both fit in TMEM's 512 columns
   static constexpr int NBUF = 2 * NA * BN <= 512 ? 2 : 1;
@@ -60,45 +62,25 @@ struct Bf16Cfg {
 template <int MODE, int BN>
 struct Fp8Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;
-  static constexpr int kMaxKB = 64;  // K / 128 <= 64 (K <= 8192)
-  static constexpr uint32_t kScaleBytes = BN * kMaxKB * 4;
-  static constexpr int kStagesRaw = (200 * 1024 - (int)kScaleBytes) / (int)kStageBytes;
+  static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;  // one 128-wide K block
+  static constexpr int kMaxKB = 64;                                   // K / 128 <= 64 (K <= 8192)
+  // activation scales [BN][KB], weight scales [2][KB], routing weights [BN]
+  static constexpr uint32_t kScaleBytes = BN * kMaxKB * 4 + 2 * kMaxKB * 4 + BN * 4;
+  static constexpr int kStagesRaw = (220 * 1024 - (int)kScaleBytes) / (int)kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr uint32_t kTmemCols = tmem_cols_for(2 * NA * BN);
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kScaleBytes + 256;
+  // TMEM buffers of per-K-block partial sums (the MMA runs up to NP blocks ahead of the promotion)
+  static constexpr int kNpRaw = 512 / (NA * BN);
+  static constexpr int NP = kNpRaw > 8 ? 8 : kNpRaw;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(NP * NA * BN);
+  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kScaleBytes + 8 * (2 * kStages + 2 * NP) + 64;
+  static_assert(kStages >= 2 && NP >= 2, "FP8 pipeline needs two stages and two partial buffers");
 };
 
 struct TileInfo {
   int e, mapi, mt, row0, nvalid, nti;  // nti: N tiles of this expert (readers of each weight tile)
 };
 
-// Finds this CTA's (expert, M tile, N tile); false if the CTA has no tile.
-__device__ __forceinline__ bool decode_tile(const GemmArgs& a, int m_tiles, int bn, TileInfo& ti) {
-  const int total = a.nt_prefix[a.L] * m_tiles;
-  const int tile = blockIdx.x;
-  if (tile >= total) return false;
-  // once any CTA has given up on a wait, the rest of the grid stands down
-  if (a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT)) return false;
-  int lo = 0, hi = a.L;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (a.nt_prefix[mid] * m_tiles <= tile) lo = mid;
-    else hi = mid;
-  }
-  const int nti = a.nt_prefix[lo + 1] - a.nt_prefix[lo];
-  const int local = tile - a.nt_prefix[lo] * m_tiles;
-  const int mt = local / nti, nt = local - mt * nti;
-  ti.e = a.list_expert[lo];
-  ti.mapi = a.list_map[lo];
-  ti.mt = mt;
-  ti.row0 = a.offsets[ti.e] + nt * bn;
-  ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
-  ti.nti = nti;
-  return true;
-}
-
-// Same as decode_tile for an explicit tile index (no range or status checks).
+// The (expert, 128-row tile, N tile) of tile index `tile` (no range or status checks).
 __device__ __forceinline__ void decode_tile_at(const GemmArgs& a, int m_tiles, int bn, int tile, TileInfo& ti) {
   int lo = 0, hi = a.L;
   while (hi - lo > 1) {
@@ -403,66 +385,67 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
 }
 
 // ======================================================================= fp8
+// Persistent, like the bf16 kernel: one CTA per SM walks tiles blockIdx.x,
+// +gridDim.x, ...; the shared-memory pipeline and a ring of NP TMEM buffers
+// for the per-K-block partial sums run on across tile boundaries. Per tile the
+// epilogue warps stage the tile's activation and weight scales (and, for down,
+// the routing weights) in shared memory, then promote every K block's partial
+// sum in registers, K blocks in increasing order. The MMA width adapts per
+// tile (16 .. BN). After a failed (timed-out) wait a warp stops working but
+// keeps its control flow, so the epilogue warps always meet at the same named
+// barriers.
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__ CUtensorMap act_map,
-                                                         const GemmArgs a) {
+__global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
   using C = Fp8Cfg<MODE, BN>;
-  constexpr int NA = C::NA, S = C::kStages;
+  constexpr int NA = C::NA, S = C::kStages, NP = C::NP;
   constexpr uint32_t STAGE = C::kStageBytes;
-  constexpr uint32_t IDESC = instr_desc(128, BN, 0u);
   constexpr int HALF = BN / 2;  // columns per epilogue warp
   constexpr int NCH = HALF >= 16 ? HALF / 16 : 1;
-  constexpr int CW = HALF >= 16 ? 16 : HALF;  // columns per TMEM load
+  constexpr int CW = HALF >= 16 ? 16 : HALF;  // columns used per TMEM load
 
-  TileInfo ti;
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
+  const int KD = MODE == kGateUp ? a.H : a.I;  // reduction length
+  const int KB = KD / 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
   if (!a.plan_ready) {
     pdl_wait();
     pdl_trigger();
   }
-  if (!decode_tile(a, m_tiles, BN, ti)) {
+  const int total = a.nt_prefix[a.L] * m_tiles;
+  const bool stand_down = a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT);
+  if ((int)blockIdx.x >= total || stand_down) {
     pdl_wait();
     return;
   }
-  const int KD = MODE == kGateUp ? a.H : a.I;  // reduction length
-  const int KB = KD / 128;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  float* s_act = reinterpret_cast<float*>(gbase + S * STAGE);  // [BN][KB]
-  const uint32_t bars = base + S * STAGE + C::kScaleBytes;
+  float* s_act = reinterpret_cast<float*>(gbase + S * STAGE);  // [BN][KB] activation scales of the tile's pairs
+  float* s_w = s_act + BN * C::kMaxKB;                         // [NA][KB] weight scales of the tile's row blocks
+  float* wcol = s_w + 2 * C::kMaxKB;                           // [BN] routing weights (down)
+  const uint32_t bars = base + S * STAGE + C::kScaleBytes;     // full[S], empty[S], pfull[NP], pempty[NP]
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
   auto pfull = [&](int b) { return bars + 8u * (2 * S + b); };
-  auto pempty = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + C::kScaleBytes + 8 * (2 * S + 4));
+  auto pempty = [&](int b) { return bars + 8u * (2 * S + NP + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + C::kScaleBytes + 8 * (2 * S + 2 * NP));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NP; ++b) {
       mbar_init(pfull(b), 1);
       mbar_init(pempty(b), 8);
     }
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  // activation scales of this tile's pairs -> shared memory (they come from the
-  // immediately preceding kernel)
-  if (a.plan_ready) {
-    pdl_wait();
-    pdl_trigger();
-  }
-  for (int i = threadIdx.x; i < BN * KB; i += blockDim.x) {
-    const int n = i / KB, kb = i - n * KB;
-    s_act[i] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -473,130 +456,210 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  const MapEntry* me = a.maps + ti.mapi;
-  const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
-
   if (warp == 8) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tensormap_acquire(wmap);
-      tma_prefetch_map(wmap);
-      tma_prefetch_map(&act_map);
-      // evict-first only when this tile is the weight rows' sole reader
-      const uint64_t pol_w = ti.nti > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
-      int kb = 0;
-      for (; kb < KB; ++kb) {
-        const int s = kb % S;
-        if (kb >= S && !mbar_wait(empty(s), ((kb / S) - 1) & 1)) {
-          *abort_flag = 1;
-          flag_status(a.status, MOE_DEV_TIMEOUT);
-          break;
+      const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
+      int issued = 0;
+      bool first = true;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile_at(a, m_tiles, BN, tile, ti);
+        const int wi = tile_width_index(ti.nvalid, BN);
+        const void* amap = &act.m[wi];
+        const uint32_t stage_tx = NA * kABytes + (16u << wi) * 128u;
+        const uint64_t pol_w = ti.nti > 1 ? pol_shared : pol_once;  // evict-first only for a sole reader
+        const MapEntry* me = a.maps + ti.mapi;
+        const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
+        tensormap_acquire(wmap);
+        int kb = 0;
+        if (first) {
+          first = false;
+          const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
+          for (int j = 0; j < npre; ++j) {
+            const uint32_t st = base + j * STAGE;
+            mbar_arrive_expect_tx(full(j), stage_tx);
+            tma_load_2d_hint(st, wmap, full(j), j * 128, ti.mt * 128, pol_w);
+            if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(j), j * 128, a.I + ti.mt * 128, pol_w);
+          }
+          if (a.plan_ready) {
+            pdl_wait();
+            pdl_trigger();
+          }
+          for (int j = 0; j < npre; ++j) tma_load_2d(base + j * STAGE + NA * kABytes, amap, full(j), j * 128, ti.row0);
+          kb = npre;
+          issued = npre;
         }
-        if (*abort_flag) break;
-        const uint32_t st = base + s * STAGE;
-        mbar_arrive_expect_tx(full(s), STAGE);
-        tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
-        if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
-        tma_load_2d(st + NA * kABytes, &act_map, full(s), kb * 128, ti.row0);
+        for (; kb < KB; ++kb, ++issued) {
+          const int s = issued % S;
+          if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
+            *abort_flag = 1;
+            flag_status(a.status, MOE_DEV_TIMEOUT);
+            break;
+          }
+          const uint32_t st = base + s * STAGE;
+          mbar_arrive_expect_tx(full(s), stage_tx);
+          tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+          if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
+          tma_load_2d(st + NA * kABytes, amap, full(s), kb * 128, ti.row0);
+        }
       }
-      for (int j = kb - S < 0 ? 0 : kb - S; j < kb; ++j) mbar_wait(full(j % S), (j / S) & 1);
+      // every copy this thread issued has landed before the CTA may exit
+      for (int g = issued - S < 0 ? 0 : issued - S; g < issued; ++g) mbar_wait(full(g % S), (g / S) & 1);
+    } else if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
     }
   } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     if (lane == 0) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % S, b = kb & 1;
-        bool ok = mbar_wait(full(s), (kb / S) & 1);
-        if (ok && kb >= 2) ok = mbar_wait(pempty(b), ((kb >> 1) - 1) & 1);
-        if (!ok) {
-          *abort_flag = 1;
-          flag_status(a.status, MOE_DEV_TIMEOUT);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t st = base + s * STAGE;
-        const uint32_t d = tmem + static_cast<uint32_t>(b * NA * BN);
+      int consumed = 0, kp = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile_at(a, m_tiles, BN, tile, ti);
+        const int width = 16 << tile_width_index(ti.nvalid, BN);
+        const uint32_t idesc = instr_desc(128, width, 0u);
+        for (int kb = 0; kb < KB; ++kb, ++consumed, ++kp) {
+          const int s = consumed % S, pb = kp % NP;
+          ok = mbar_wait(full(s), (consumed / S) & 1);
+          if (ok && kp >= NP) ok = mbar_wait(pempty(pb), ((kp / NP) - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = base + s * STAGE;
+          const uint32_t d = tmem + static_cast<uint32_t>(pb * NA * BN);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
-          const uint32_t acc = k != 0 ? 1u : 0u;
-          tc_mma_e4m3(d, sw128_kmajor_desc(st + k * 32), bdesc, IDESC, acc);
-          if (MODE == kGateUp) tc_mma_e4m3(d + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, IDESC, acc);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
+            const uint32_t acc = k != 0 ? 1u : 0u;
+            tc_mma_e4m3(d, sw128_kmajor_desc(st + k * 32), bdesc, idesc, acc);
+            if (MODE == kGateUp) tc_mma_e4m3(d + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, idesc, acc);
+          }
+          tc_commit(empty(s));
+          tc_commit(pfull(pb));
         }
-        tc_commit(empty(s));
-        tc_commit(pfull(b));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_status(a.status, MOE_DEV_TIMEOUT);
       }
     }
   } else {
-    // epilogue: warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
+    // ------------------------------------------------------------ epilogue (warps 0..7)
+    // warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     const int q4 = warp & 3, hf = warp >> 2;
     const int r = q4 * 32 + lane;
+    const int et = threadIdx.x;  // 0..255
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int c0 = hf * HALF;
-    const int wrow_g = ti.mt;                // weight row block of this lane's gate (or down) row
-    const int wrow_u = a.I / 128 + ti.mt;    // weight row block of the up row
-    const float* sw = MODE == kGateUp ? me->s_gu : me->s_dn;
-    float accg[HALF], accu[MODE == kGateUp ? HALF : 1];
-#pragma unroll
-    for (int i = 0; i < HALF; ++i) accg[i] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < (MODE == kGateUp ? HALF : 1); ++i) accu[i] = 0.0f;
-    bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      const int b = kb & 1;
-      ok = mbar_wait(pfull(b), (kb >> 1) & 1);
-      if (!ok || *abort_flag) break;
-      tc_fence_after();
-      const float swg = __ldg(sw + (size_t)wrow_g * KB + kb);
-      const float swu = MODE == kGateUp ? __ldg(sw + (size_t)wrow_u * KB + kb) : 0.0f;
-      const uint32_t pb = tl + static_cast<uint32_t>(b * NA * BN + c0);
-#pragma unroll
-      for (int ch = 0; ch < NCH; ++ch) {
-        uint32_t pg[16], pu[16];
-        if (CW == 16) {
-          tmem_ld16(pb + ch * 16, pg);
-          if (MODE == kGateUp) tmem_ld16(pb + BN + ch * 16, pu);
-        } else {
-          // HALF == 8: load 16 columns starting at c0 (the other half is ignored)
-          tmem_ld16(tl + static_cast<uint32_t>(b * NA * BN), pg);
-          if (MODE == kGateUp) tmem_ld16(tl + static_cast<uint32_t>(b * NA * BN + BN), pu);
-        }
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < CW; ++q) {
-          const int col = ch * 16 + q;             // index within this warp's half
-          const int n = c0 + col;                  // tile column
-          const int src = CW == 16 ? q : c0 + q;   // register holding column n
-          const float sa = s_act[n * KB + kb];
-          accg[col] = fmaf(__uint_as_float(pg[src]), sa * swg, accg[col]);
-          if (MODE == kGateUp) accu[col] = fmaf(__uint_as_float(pu[src]), sa * swu, accu[col]);
-        }
+    bool aborted = false;  // warp-uniform
+    int kp = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      TileInfo ti;
+      decode_tile_at(a, m_tiles, BN, tile, ti);
+      const int width = 16 << tile_width_index(ti.nvalid, BN);
+      const MapEntry* me = a.maps + ti.mapi;
+      const float* sw = MODE == kGateUp ? me->s_gu : me->s_dn;
+      named_bar_sync(1, 256);  // the previous tile's readers are done with the scale tables
+      for (int i = et; i < BN * KB; i += 256) {
+        const int n = i / KB, kb = i - n * KB;
+        s_act[n * KB + kb] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pempty(b));
-    }
-    if (!ok) flag_status(a.status, MOE_DEV_TIMEOUT);
-    if (ok && !*abort_flag) {
-      if (MODE == kGateUp) {
-        const int j = ti.mt * 128 + r;
-        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
-#pragma unroll
-        for (int col = 0; col < HALF; ++col) {
-          const int n = c0 + col;
-          if (n < ti.nvalid) {
-            const float gv = accg[col], uv = accu[col];
-            const float hv = gv / (1.0f + expf(-gv)) * uv;
-            hout[(size_t)(ti.row0 + n) * a.I + j] = __float2bfloat16_rn(hv);
-          }
-        }
-      } else {
-        const int o = ti.mt * 128 + r;
-#pragma unroll
-        for (int col = 0; col < HALF; ++col) {
-          const int n = c0 + col;
+      for (int i = et; i < NA * KB; i += 256) {
+        const int which = i / KB, kb = i - which * KB;
+        const int rb = which == 0 ? ti.mt : a.I / 128 + ti.mt;  // gate (or down) row block, then up
+        s_w[which * KB + kb] = sw[(size_t)rb * KB + kb];
+      }
+      if (MODE == kDown) {
+        for (int n = et; n < BN; n += 256) {
+          float wv = 0.0f;
           if (n < ti.nvalid) {
             const int p = ti.row0 + n;
-            const float wgt = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
-            a.y_out[(size_t)p * a.H + o] = wgt * accg[col];
+            wv = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
+          }
+          wcol[n] = wv;
+        }
+      }
+      named_bar_sync(1, 256);
+
+      float accg[HALF], accu[MODE == kGateUp ? HALF : 1];
+#pragma unroll
+      for (int i = 0; i < HALF; ++i) accg[i] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < (MODE == kGateUp ? HALF : 1); ++i) accu[i] = 0.0f;
+      for (int kb = 0; kb < KB; ++kb, ++kp) {
+        const int pb = kp % NP;
+        if (!aborted) {
+          bool ok = !*abort_flag && mbar_wait(pfull(pb), (kp / NP) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
+            aborted = true;
+            if (lane == 0) {
+              *abort_flag = 1;
+              flag_status(a.status, MOE_DEV_TIMEOUT);
+            }
+          }
+        }
+        if (!aborted) {
+          tc_fence_after();
+          const float swg = s_w[kb];
+          const float swu = MODE == kGateUp ? s_w[KB + kb] : 0.0f;
+          const uint32_t pbase = tl + static_cast<uint32_t>(pb * NA * BN);
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
+            const int cstart = CW == 16 ? c0 + ch * 16 : 0;  // first TMEM column of this load
+            if (cstart < width) {                             // warp-uniform
+              uint32_t pg[16], pu[16];
+              tmem_ld16(pbase + cstart, pg);
+              if (MODE == kGateUp) tmem_ld16(pbase + BN + cstart, pu);
+              tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < CW; ++q) {
+                const int col = ch * CW + q;  // index within this warp's half
+                const int n = c0 + col;       // tile column
+                // register holding column n (HALF < 16: the load holds both halves)
+                const uint32_t gb = CW == 16 ? pg[q] : (hf ? pg[(CW + q) & 15] : pg[q]);
+                const float sa = s_act[n * KB + kb];
+                accg[col] = fmaf(__uint_as_float(gb), sa * swg, accg[col]);
+                if (MODE == kGateUp) {
+                  const uint32_t ub = CW == 16 ? pu[q] : (hf ? pu[(CW + q) & 15] : pu[q]);
+                  accu[col] = fmaf(__uint_as_float(ub), sa * swu, accu[col]);
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pempty(pb));
+      }
+      if (!aborted) {
+        if (MODE == kGateUp) {
+          const int j = ti.mt * 128 + r;
+          __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
+#pragma unroll
+          for (int col = 0; col < HALF; ++col) {
+            const int n = c0 + col;
+            if (n < ti.nvalid) {
+              const float gv = accg[col], uv = accu[col];
+              const float hv = gv / (1.0f + expf(-gv)) * uv;
+              hout[(size_t)(ti.row0 + n) * a.I + j] = __float2bfloat16_rn(hv);
+            }
+          }
+        } else {
+          const int o = ti.mt * 128 + r;
+#pragma unroll
+          for (int col = 0; col < HALF; ++col) {
+            const int n = c0 + col;
+            if (n < ti.nvalid) a.y_out[(size_t)(ti.row0 + n) * a.H + o] = wcol[n] * accg[col];
           }
         }
       }
@@ -629,6 +692,12 @@ static cudaError_t launch_bf16(const ActMaps& maps, GemmArgs a, int grid, cudaSt
   return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 192, persistent, maps, a, s, pdl);
 }
 
+template <int MODE, int BN>
+static cudaError_t launch_fp8(const ActMaps& maps, const GemmArgs& a, int grid, cudaStream_t s, bool pdl) {
+  const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
+  return launch_kernel(ffn_fp8_kernel<MODE, BN>, Fp8Cfg<MODE, BN>::kSmem, 320, persistent, maps, a, s, pdl);
+}
+
 template <int MODE>
 static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const ActMaps* maps, const GemmArgs& a,
                                int grid, cudaStream_t s, bool pdl) {
@@ -642,9 +711,9 @@ static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const
     }
   } else {
     switch (bn) {
-      case 16: return launch_kernel(ffn_fp8_kernel<MODE, 16>, Fp8Cfg<MODE, 16>::kSmem, 320, grid, map, a, s, pdl);
-      case 32: return launch_kernel(ffn_fp8_kernel<MODE, 32>, Fp8Cfg<MODE, 32>::kSmem, 320, grid, map, a, s, pdl);
-      case 64: return launch_kernel(ffn_fp8_kernel<MODE, 64>, Fp8Cfg<MODE, 64>::kSmem, 320, grid, map, a, s, pdl);
+      case 16: return launch_fp8<MODE, 16>(*maps, a, grid, s, pdl);
+      case 32: return launch_fp8<MODE, 32>(*maps, a, grid, s, pdl);
+      case 64: return launch_fp8<MODE, 64>(*maps, a, grid, s, pdl);
     }
   }
   return cudaErrorInvalidValue;

@@ -213,6 +213,21 @@ cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E
 // ----------------------------------------------------------------- gather --
 // x_perm[p, :] = x[perm_src[p], :] for the offsets[E] valid pairs; one warp per
 // row, 16-byte vectors.
+// Copies one row of n 16-byte vectors with a warp, eight loads in flight per
+// lane before the stores.
+__device__ __forceinline__ void copy_row_warp(const uint4* __restrict__ src, uint4* __restrict__ dst, int n,
+                                              int lane) {
+  for (int v0 = lane; v0 < n; v0 += 32 * 8) {
+    uint4 tmp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (v0 + 32 * u < n) tmp[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (v0 + 32 * u < n) dst[v0 + 32 * u] = tmp[u];
+  }
+}
+
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
                                                            const int32_t* __restrict__ perm_src,
                                                            const int32_t* __restrict__ offsets, int E, int P,
@@ -223,9 +238,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
   const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (p >= P || p >= offsets[E]) return;
   const int t = perm_src[p];
-  const uint4* src = x + (size_t)t * vec_per_row;
-  uint4* dst = xp + (size_t)p * vec_per_row;
-  for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+  copy_row_warp(x + (size_t)t * vec_per_row, xp + (size_t)p * vec_per_row, vec_per_row, lane);
 }
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
@@ -323,9 +336,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
     const int warp = i >> 5, lane = i & 31, nw = blockDim.x >> 5;
     for (int row = blockIdx.x * nw + warp; row < total; row += gridDim.x * nw) {
       const int t = s_src[row] / K;
-      const uint4* src = x + (size_t)t * vec_per_row;
-      uint4* dst = x_perm + (size_t)row * vec_per_row;
-      for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+      copy_row_warp(x + (size_t)t * vec_per_row, x_perm + (size_t)row * vec_per_row, vec_per_row, lane);
     }
   }
 }

@@ -5,77 +5,64 @@
 // identical logits at any batch size" is the results-table "quality" row).
 //
 // Logit order (the contract both these kernels and the CPU oracle follow):
-// h is cut into chunks of 8 (chunk c = h 8c..8c+7); lane j of a warp owns the
-// chunks c = j, j+32, j+64, ... and runs fmaf(x[h], Wr[e][h], acc) from +0
-// over them in increasing c (h increasing inside a chunk); the 32 lane
-// partials are then summed by the xor butterfly (offsets 16, 8, 4, 2, 1),
-// which leaves p[j] += p[j+o] (o = 16 .. 1) in every lane; then one fp32 add
-// of bias[e]. Every warp load of Wr or x is 32 consecutive 16-byte pieces,
-// and a token's logits depend on that token alone, whatever the batch.
+// lane j of a warp runs fmaf(x[h], Wr[e][h], acc) from +0 over h = j, j+32,
+// j+64, ... in increasing h; the 32 lane partials are then summed by the xor
+// butterfly (offsets 16, 8, 4, 2, 1), which leaves p[j] += p[j+o]
+// (o = 16 .. 1) in lane 0; then one fp32 add of bias[e]. A warp's loads of
+// one h step are 32 consecutive elements, and a token's logits depend on that
+// token alone, whatever the batch.
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
-// One warp per expert, TG tokens per warp; lane j owns chunks j, j+32, ...
-// U chunks per lane are loaded before any is used, so a warp keeps
-// U x (32 + 16 TG) bytes per lane in flight. Wr streams once per token
-// group with coalesced 512-byte warp loads; x comes through L1 (shared by
-// the CTA's warps, which all read the same tokens).
+__device__ __forceinline__ float bf16_lo(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+__device__ __forceinline__ void butterfly_sum(float& v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
+}
+
+// ------------------------------------------------ direct (global) router --
+// One warp per expert, TG tokens per warp, operands straight from global
+// memory: per h step a warp reads 128 contiguous bytes of Wr and 64 of each x
+// row. U steps are loaded before any is used.
 template <int TG, int U>
-__device__ __forceinline__ void logits_warp(const uint16_t* __restrict__ x, const float* __restrict__ wrow, int T,
-                                            int H, int t0, float (&acc)[TG]) {
+__device__ __forceinline__ void logits_warp_direct(const uint16_t* __restrict__ x, const float* __restrict__ wrow,
+                                                   int T, int H, int t0, float (&acc)[TG]) {
   const int lane = threadIdx.x & 31;
   const int ntok = min(TG, T - t0);
 #pragma unroll
   for (int i = 0; i < TG; ++i) acc[i] = 0.0f;
-  for (int hb = lane * 8; hb < H; hb += 256 * U) {
-    float4 wa[U], wb[U];
-    uint4 xv[U][TG];
+  for (int hb = lane; hb < H; hb += 32 * U) {
+    float w[U];
+    uint32_t xv[U][TG];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int h = hb + 256 * u;
+      const int h = hb + 32 * u;
       if (h < H) {
-        wa[u] = __ldg(reinterpret_cast<const float4*>(wrow + h));
-        wb[u] = __ldg(reinterpret_cast<const float4*>(wrow + h + 4));
+        w[u] = __ldg(wrow + h);
 #pragma unroll
         for (int i = 0; i < TG; ++i)
-          if (i < ntok) xv[u][i] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + i) * H + h));
+          if (i < ntok) xv[u][i] = __ldg(x + (size_t)(t0 + i) * H + h);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      if (hb + 256 * u < H) {
+      if (hb + 32 * u < H) {
 #pragma unroll
-        for (int i = 0; i < TG; ++i) {
-          if (i < ntok) {
-            const uint4 v = xv[u][i];
-            float a = acc[i];
-            a = fmaf(__uint_as_float(v.x << 16), wa[u].x, a);
-            a = fmaf(__uint_as_float(v.x & 0xffff0000u), wa[u].y, a);
-            a = fmaf(__uint_as_float(v.y << 16), wa[u].z, a);
-            a = fmaf(__uint_as_float(v.y & 0xffff0000u), wa[u].w, a);
-            a = fmaf(__uint_as_float(v.z << 16), wb[u].x, a);
-            a = fmaf(__uint_as_float(v.z & 0xffff0000u), wb[u].y, a);
-            a = fmaf(__uint_as_float(v.w << 16), wb[u].z, a);
-            a = fmaf(__uint_as_float(v.w & 0xffff0000u), wb[u].w, a);
-            acc[i] = a;
-          }
-        }
+        for (int i = 0; i < TG; ++i)
+          if (i < ntok) acc[i] = fmaf(bf16_lo(xv[u][i]), w[u], acc[i]);
       }
     }
   }
 #pragma unroll
-  for (int i = 0; i < TG; ++i) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) acc[i] = acc[i] + __shfl_xor_sync(0xffffffffu, acc[i], o);
-  }
+  for (int i = 0; i < TG; ++i) butterfly_sum(acc[i]);
 }
 
-// Loads in flight per lane for a token group of TG (registers: U (8 + 4 TG)).
 template <int TG>
-struct LogitsUnroll {
-  static constexpr int value = TG <= 2 ? 8 : (TG <= 4 ? 4 : 2);
+struct DirectUnroll {
+  static constexpr int value = TG == 1 ? 32 : (TG <= 2 ? 16 : (TG <= 4 ? 8 : 4));
 };
 
 template <int TG>
@@ -87,7 +74,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
   const int t0 = blockIdx.y * TG;
   if (e >= E) return;  // warp-uniform
   float acc[TG];
-  logits_warp<TG, LogitsUnroll<TG>::value>(x, wr + (size_t)e * H, T, H, t0, acc);
+  logits_warp_direct<TG, DirectUnroll<TG>::value>(x, wr + (size_t)e * H, T, H, t0, acc);
   if ((threadIdx.x & 31) == 0) {
     const float b = bias ? bias[e] : 0.0f;
 #pragma unroll
@@ -263,120 +250,62 @@ cudaError_t launch_topk_warp(const float* logits, int T, int E, int K, int32_t* 
   return launch_ex(topk_warp_kernel, dim3((T + 7) / 8), dim3(256), 0, s, pdl, logits, T, E, K, idx, w);
 }
 
-// ------------------------------------------------- decode-regime router --
-// Same warp-per-expert logits (WPC experts per CTA, TG tokens per group); with
-// fuse_topk, the last CTA of each token group (an arrival counter) selects the
-// group's top-k, one warp per token, and returns the counter to zero;
-// otherwise a top-k kernel follows.
-template <int TG, int WPC>
-__global__ void __launch_bounds__(WPC * 32) route_small_kernel(const uint16_t* __restrict__ x,
-                                                           const float* __restrict__ wr,
-                                                           const float* __restrict__ bias, int T, int H, int E, int K,
-                                                           float* __restrict__ logits, int32_t* __restrict__ idx,
-                                                           float* __restrict__ w, unsigned int* __restrict__ counters,
-                                                           int fuse_topk) {
-  __shared__ int s_last;
-  pdl_trigger();  // first kernel of a forward: the next one may launch (it waits for us)
-  const int warp = threadIdx.x >> 5;
-  const int e = blockIdx.x * WPC + warp;
-  const int t0 = blockIdx.y * TG;
-  const int ntok = min(TG, T - t0);
-  if (e < E) {
-    float acc[TG];
-    logits_warp<TG, LogitsUnroll<TG>::value>(x, wr + (size_t)e * H, T, H, t0, acc);
-    if ((threadIdx.x & 31) == 0) {
-      const float b = bias ? bias[e] : 0.0f;
-#pragma unroll
-      for (int i = 0; i < TG; ++i)
-        if (i < ntok) logits[(size_t)(t0 + i) * E + e] = bias ? acc[i] + b : acc[i];
-    }
-  }
-  if (!fuse_topk) return;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(counters + blockIdx.y, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int i = warp; i < ntok; i += WPC) {
-    const int t = t0 + i;
-    topk_warp_any(logits + (size_t)t * E, E, K, idx + (size_t)t * K, w + (size_t)t * K);
-  }
-  if (threadIdx.x == 0) counters[blockIdx.y] = 0u;
-}
+// --------------------------------------------- register-tiled router GEMM --
+// fp32 GEMM in the same order. A warp owns WT tokens x WE experts and its lane
+// j keeps the WT*WE lane-j partials; NWT x NWE warps make the CTA tile
+// (TT = WT*NWT tokens, TE = WE*NWE experts). Each stage holds 256 consecutive
+// h of the tile's tokens and experts in shared memory as stored (cp.async,
+// kRgStages buffers, kRgStages - 1 in flight); lane j reads h = h0 + j + 32q,
+// q = 0..7: consecutive lanes, consecutive elements.
+//   prefill:          WT = 8, WE = 8, 6 x 2 warps (48 tokens x 16 experts)
+//   16 < T <= 64:     WT = 4, WE = 8, 2 x 2 warps (8 x 16)
+//   8 < T <= 16:      WT = 4, WE = 4, 2 x 2 warps (8 x 8)
+constexpr int kRgStages = 3;
 
-// Four warps per CTA: a 384-expert router spreads over 96 SMs.
-constexpr int kRsWarps = 4;
+template <int WT, int WE, int NWT, int NWE>
+struct RgCfg {
+  static constexpr int TT = WT * NWT, TE = WE * NWE, kThreads = 32 * NWT * NWE;
+  static constexpr size_t kStageBytes = (size_t)TT * 256 * 2 + (size_t)TE * 256 * 4;
+  static constexpr size_t kSmem = kRgStages * kStageBytes;
+};
 
-template <int TG>
-static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
-                             float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, cudaStream_t s) {
-  dim3 grid((E + kRsWarps - 1) / kRsWarps, (T + TG - 1) / TG);
-  return launch_ex(route_small_kernel<TG, kRsWarps>, grid, dim3(kRsWarps * 32), 0, s, false, static_cast<const uint16_t*>(x), wr, bias,
-                   T, H, E, K, logits, idx, w, counters, fuse);
-}
-
-// T <= 8: logits + fused top-k in one launch; up to 64 tokens: logits in
-// 8-token groups, then the warp top-k kernel (programmatic launch).
-cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
-                               float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl) {
-  (void)status;
-  if (T <= 0) return cudaSuccess;
-  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
-  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
-  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
-  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, s);
-  cudaError_t err = launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, s);
-  if (err != cudaSuccess) return err;
-  return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
-}
-
-// ------------------------------------------------ prefill-regime router --
-// Register-tiled fp32 GEMM in the same order. CTA tile: 48 tokens x 16
-// experts, 12 warps as 6 token groups x 2 expert groups; a warp owns 8 tokens
-// x 8 experts and its lane j keeps the 64 lane-j partials (chunks j, j+32,
-// ...). Each stage holds 256 consecutive h of the tile's tokens and experts
-// in shared memory (cp.async, kRgStages buffers, kRgStages - 1 in flight):
-// token rows as stored, each Wr row
-// split into its chunks' first halves then second halves so that the 32
-// lanes' 16-byte reads are consecutive.
-constexpr int kRgT = 48, kRgE = 16, kRgStages = 3, kRgThreads = 384;
-constexpr size_t kRgStageBytes = (size_t)kRgT * 256 * 2 + (size_t)kRgE * 256 * 4;
-
-__global__ void __launch_bounds__(kRgThreads, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
-                                                             const float* __restrict__ wr,
-                                                             const float* __restrict__ bias, int T, int H, int E,
-                                                             float* __restrict__ logits) {
+template <int WT, int WE, int NWT, int NWE>
+__global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
+                                                                        const float* __restrict__ wr,
+                                                                        const float* __restrict__ bias, int T, int H,
+                                                                        int E, float* __restrict__ logits) {
+  using C = RgCfg<WT, WE, NWT, NWE>;
+  constexpr int TT = C::TT, TE = C::TE, NT = C::kThreads;
   extern __shared__ __align__(16) uint8_t sm[];
+  pdl_wait();  // x may come from the previous kernel
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tt0 = (warp >> 1) * 8, ee0 = (warp & 1) * 8;
-  const int tb = blockIdx.y * kRgT, eb = blockIdx.x * kRgE;
+  const int tt0 = (warp / NWE) * WT, ee0 = (warp % NWE) * WE;
+  const int tb = blockIdx.y * TT, eb = blockIdx.x * TE;
   const int nsteps = H / 256;
-  auto xs = [&](int buf) { return reinterpret_cast<uint16_t*>(sm + buf * kRgStageBytes); };
-  auto ws = [&](int buf) { return reinterpret_cast<float*>(sm + buf * kRgStageBytes + (size_t)kRgT * 256 * 2); };
+  auto xs = [&](int buf) { return reinterpret_cast<uint16_t*>(sm + buf * C::kStageBytes); };
+  auto ws = [&](int buf) { return reinterpret_cast<float*>(sm + buf * C::kStageBytes + (size_t)TT * 256 * 2); };
   auto load_stage = [&](int st, int buf) {
     const int h0 = st * 256;
     uint16_t* xd = xs(buf);
     float* wd = ws(buf);
-    for (int c = tid; c < kRgT * 32; c += kRgThreads) {  // token row: 32 x 16 B
+    for (int c = tid; c < TT * 32; c += NT) {  // token row: 32 x 16 B
       const int t = c >> 5, part = c & 31;
       const int row = min(tb + t, T - 1);  // rows past T re-read row T-1 (results discarded)
       cp_async16(xd + (size_t)t * 256 + part * 8, x + (size_t)row * H + h0 + part * 8);
     }
-    for (int c = tid; c < kRgE * 64; c += kRgThreads) {  // expert row: 64 x 16 B (32 chunks x 2 halves)
-      const int e = c >> 6, q = c & 63, chunk = q >> 1, half = q & 1;
+    for (int c = tid; c < TE * 64; c += NT) {  // expert row: 64 x 16 B
+      const int e = c >> 6, part = c & 63;
       const int row = min(eb + e, E - 1);
-      cp_async16(wd + (size_t)e * 256 + half * 128 + chunk * 4, wr + (size_t)row * H + h0 + q * 4);
+      cp_async16(wd + (size_t)e * 256 + part * 4, wr + (size_t)row * H + h0 + part * 4);
     }
   };
 
-  float acc[8][8];
+  float acc[WT][WE];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < WT; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < WE; ++j) acc[i][j] = 0.0f;
 
 #pragma unroll
   for (int st = 0; st < kRgStages - 1; ++st) {
@@ -392,50 +321,33 @@ __global__ void __launch_bounds__(kRgThreads, 1) route_gemm_kernel(const uint16_
     }
     asm volatile("cp.async.wait_group %0;" ::"n"(kRgStages - 1) : "memory");
     __syncthreads();
-    const uint16_t* xb = xs(buf);
-    const float* wb = ws(buf);
-    float xf[8][8];
+    const uint16_t* xb = xs(buf) + (size_t)tt0 * 256 + lane;
+    const float* wb = ws(buf) + (size_t)ee0 * 256 + lane;
+#pragma unroll 2
+    for (int q = 0; q < 8; ++q) {
+      float xf[WT];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 v = *reinterpret_cast<const uint4*>(xb + (size_t)(tt0 + i) * 256 + lane * 8);
-      xf[i][0] = __uint_as_float(v.x << 16);
-      xf[i][1] = __uint_as_float(v.x & 0xffff0000u);
-      xf[i][2] = __uint_as_float(v.y << 16);
-      xf[i][3] = __uint_as_float(v.y & 0xffff0000u);
-      xf[i][4] = __uint_as_float(v.z << 16);
-      xf[i][5] = __uint_as_float(v.z & 0xffff0000u);
-      xf[i][6] = __uint_as_float(v.w << 16);
-      xf[i][7] = __uint_as_float(v.w & 0xffff0000u);
-    }
+      for (int i = 0; i < WT; ++i) xf[i] = bf16_lo(xb[(size_t)i * 256 + 32 * q]);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float* wrow = wb + (size_t)(ee0 + j) * 256;
-      const float4 wa = *reinterpret_cast<const float4*>(wrow + lane * 4);
-      const float4 wc = *reinterpret_cast<const float4*>(wrow + 128 + lane * 4);
-      const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wc.x, wc.y, wc.z, wc.w};
-      // h-element outer, token inner: eight independent chains between two
-      // dependent FMAs (each acc still takes its eight FMAs in h order)
+      for (int j = 0; j < WE; ++j) {
+        const float wv = wb[(size_t)j * 256 + 32 * q];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i][j] = fmaf(xf[i][q], wv[q], acc[i][j]);
+        for (int i = 0; i < WT; ++i) acc[i][j] = fmaf(xf[i], wv, acc[i][j]);
       }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < WT; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) acc[i][j] = acc[i][j] + __shfl_xor_sync(0xffffffffu, acc[i][j], o);
+    for (int j = 0; j < WE; ++j) butterfly_sum(acc[i][j]);
   if (lane == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < WT; ++i) {
       const int t = tb + tt0 + i;
       if (t >= T) continue;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < WE; ++j) {
         const int e = eb + ee0 + j;
         if (e < E) logits[(size_t)t * E + e] = bias ? acc[i][j] + bias[e] : acc[i][j];
       }
@@ -443,16 +355,156 @@ __global__ void __launch_bounds__(kRgThreads, 1) route_gemm_kernel(const uint16_
   }
 }
 
+template <int WT, int WE, int NWT, int NWE>
+static cudaError_t launch_rg(const void* x, const float* wr, const float* bias, int T, int H, int E, float* logits,
+                             cudaStream_t s, bool pdl) {
+  using C = RgCfg<WT, WE, NWT, NWE>;
+  auto kern = route_gemm_kernel<WT, WE, NWT, NWE>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((E + C::TE - 1) / C::TE, (T + C::TT - 1) / C::TT);
+  return launch_ex(kern, grid, dim3(C::kThreads), C::kSmem, s, pdl, static_cast<const uint16_t*>(x), wr, bias, T, H,
+                   E, logits);
+}
+
+static bool rg_tile_ok(const void* x, const float* wr, int H) {
+  return ((uintptr_t)x % 16 == 0) && ((uintptr_t)wr % 16 == 0) && (H % 256 == 0);
+}
+
 cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias, int T, int H, int E,
                               float* logits, cudaStream_t s) {
   if (T <= 0) return cudaSuccess;
-  if (H % 256 != 0) return launch_router_logits(x, wr, bias, T, H, E, logits, s);
-  const size_t smem = kRgStages * kRgStageBytes;
-  cudaError_t err = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (!rg_tile_ok(x, wr, H)) return launch_router_logits(x, wr, bias, T, H, E, logits, s);
+  return launch_rg<8, 8, 6, 2>(x, wr, bias, T, H, E, logits, s, false);
+}
+
+// ------------------------------------------------- decode-regime router --
+// WPC warps per CTA, one expert each, TG tokens per CTA. The CTA's x rows and
+// its warps' Wr rows arrive in shared memory by bulk copies (one per row, all
+// in flight together: a single DRAM round trip), then each lane reads its h
+// steps from there (consecutive lanes, consecutive words: no bank conflict).
+// With fuse_topk, the last CTA of each token group (an arrival counter) picks
+// the group's top-k, one warp per token, and returns the counter to zero;
+// otherwise a top-k kernel follows.
+constexpr int kRsWarps = 4;
+
+__host__ __device__ constexpr size_t route_small_smem(int tg, int H) {
+  return 16 + (size_t)kRsWarps * H * 4 + (size_t)tg * H * 2;
+}
+
+template <int TG>
+__global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16_t* __restrict__ x,
+                                                                     const float* __restrict__ wr,
+                                                                     const float* __restrict__ bias, int T, int H,
+                                                                     int E, int K, float* __restrict__ logits,
+                                                                     int32_t* __restrict__ idx, float* __restrict__ w,
+                                                                     unsigned int* __restrict__ counters,
+                                                                     int fuse_topk, int* status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int s_last;
+  pdl_trigger();  // first kernel of a forward: the next one may launch (it waits for us)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.x * kRsWarps, e = e0 + warp;
+  const int t0 = blockIdx.y * TG;
+  const int ntok = min(TG, T - t0), nexp = min(kRsWarps, E - e0);
+  const uint32_t bar = smem_u32(sm);
+  float* ws = reinterpret_cast<float*>(sm + 16);                              // [kRsWarps][H]
+  const uint16_t* xs = reinterpret_cast<const uint16_t*>(sm + 16 + (size_t)kRsWarps * H * 4);  // [TG][H]
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(bar, (uint32_t)(nexp * H * 4 + ntok * H * 2));
+    for (int i = 0; i < nexp; ++i)
+      bulk_load(smem_u32(ws + (size_t)i * H), wr + (size_t)(e0 + i) * H, (uint32_t)H * 4, bar);
+    for (int i = 0; i < ntok; ++i)
+      bulk_load(smem_u32(xs + (size_t)i * H), x + (size_t)(t0 + i) * H, (uint32_t)H * 2, bar);
+  }
+  __syncthreads();
+  bool ok = mbar_wait(bar, 0);
+  ok = __syncthreads_and(ok);
+  if (!ok && threadIdx.x == 0) {
+    // the copies did not land in time: flag it and give them one more bounded
+    // wait (they write this CTA's shared memory); the CTA then skips its
+    // logits but still takes part in the top-k arrival count, which must
+    // return to zero
+    flag_status(status, MOE_DEV_TIMEOUT);
+    mbar_wait(bar, 0);
+  }
+  if (ok && e < E) {
+    const float* wrow = ws + (size_t)warp * H;
+    float acc[TG];
+#pragma unroll
+    for (int i = 0; i < TG; ++i) acc[i] = 0.0f;
+#pragma unroll 4
+    for (int h = lane; h < H; h += 32) {
+      const float wv = wrow[h];
+#pragma unroll
+      for (int i = 0; i < TG; ++i)
+        if (i < ntok) acc[i] = fmaf(bf16_lo(xs[(size_t)i * H + h]), wv, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < TG; ++i) butterfly_sum(acc[i]);
+    if (lane == 0) {
+      const float b = bias ? bias[e] : 0.0f;
+#pragma unroll
+      for (int i = 0; i < TG; ++i)
+        if (i < ntok) logits[(size_t)(t0 + i) * E + e] = bias ? acc[i] + b : acc[i];
+    }
+  }
+  if (!fuse_topk) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(counters + blockIdx.y, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = warp; i < ntok; i += kRsWarps) {
+    const int t = t0 + i;
+    topk_warp_any(logits + (size_t)t * E, E, K, idx + (size_t)t * K, w + (size_t)t * K);
+  }
+  if (threadIdx.x == 0) counters[blockIdx.y] = 0u;
+}
+
+template <int TG>
+static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
+                             float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, int* status,
+                             cudaStream_t s) {
+  const size_t smem = route_small_smem(TG, H);
+  cudaError_t err = cudaFuncSetAttribute(route_small_kernel<TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
   if (err != cudaSuccess) return err;
-  dim3 grid((E + kRgE - 1) / kRgE, (T + kRgT - 1) / kRgT);
-  return launch_ex(route_gemm_kernel, grid, dim3(kRgThreads), smem, s, false, static_cast<const uint16_t*>(x), wr, bias, T,
-                   H, E, logits);
+  dim3 grid((E + kRsWarps - 1) / kRsWarps, (T + TG - 1) / TG);
+  return launch_ex(route_small_kernel<TG>, grid, dim3(kRsWarps * 32), smem, s, false,
+                   static_cast<const uint16_t*>(x), wr, bias, T, H, E, K, logits, idx, w, counters, fuse, status);
+}
+
+// T <= 8: logits + fused top-k in one launch; up to 64 tokens: logits in
+// 8-token groups, then the warp top-k kernel (programmatic launch). Rows that
+// a bulk copy cannot take (not 16-byte aligned, or too large for shared
+// memory) go through the direct kernel.
+cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
+                               float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
+                               cudaStream_t s, bool pdl) {
+  if (T <= 0) return cudaSuccess;
+  const bool bulk_ok = ((uintptr_t)x % 16 == 0) && ((uintptr_t)wr % 16 == 0) && (H % 8 == 0) &&
+                       route_small_smem(8, H) <= 200 * 1024;
+  if (!bulk_ok) {
+    cudaError_t err = launch_router_logits(x, wr, bias, T, H, E, logits, s);
+    if (err != cudaSuccess) return err;
+    return launch_topk_warp(logits, T, E, K, idx, w, s, false);
+  }
+  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
+  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
+  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
+  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
+  // more tokens: W rows would be staged once per 8-token group; register
+  // tiles reuse each loaded element across 4 tokens and 4 or 8 experts
+  cudaError_t err;
+  if (!rg_tile_ok(x, wr, H)) err = launch_router_logits(x, wr, bias, T, H, E, logits, s);
+  else if (T <= 16) err = launch_rg<4, 4, 2, 2>(x, wr, bias, T, H, E, logits, s, false);
+  else err = launch_rg<4, 8, 2, 2>(x, wr, bias, T, H, E, logits, s, false);
+  if (err != cudaSuccess) return err;
+  return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
 }
 
 }  // namespace moe

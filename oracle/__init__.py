@@ -82,7 +82,6 @@ def router_logits(x_u16: np.ndarray, wr: np.ndarray, bias=None, threads: int = 0
     lib = _load()
     T, H = x_u16.shape
     E = wr.shape[0]
-    assert H % 8 == 0
     wr = np.ascontiguousarray(wr, dtype=np.float32)
     out = np.empty((T, E), dtype=np.float32)
     b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)

@@ -27,12 +27,12 @@
  * Reading of the layer where the definition leaves a step open (each one is
  * listed with its reason in the design notes):
  *   - Logit reduction order (needed for bit-exact top-k across two
- *     implementations): h is cut into chunks of 8 (chunk c = h 8c..8c+7);
- *     lane j of 32 owns the chunks c = j, j+32, j+64, ... and accumulates
- *     fmaf(f32(x[h]), Wr[e][h], acc) from +0 over its chunks in increasing c,
- *     h increasing inside a chunk; the 32 partials are then summed pairwise,
- *     p[j] += p[j+o] for o = 16, 8, 4, 2, 1 (j < o); the logit is p[0], then
- *     + bias[e] (one fp32 add) when a bias is given.
+ *     implementations): lane j of 32 accumulates
+ *     fmaf(f32(x[h]), Wr[e][h], acc) from +0 over h = j, j+32, j+64, ... in
+ *     increasing h; the 32 partials are then summed pairwise,
+ *     p[j] += p[j+o] for o = 16, 8, 4, 2, 1 (j < o) -- what an xor butterfly
+ *     over a warp leaves in lane 0; the logit is p[0], then + bias[e] (one
+ *     fp32 add) when a bias is given.
  *   - Top-k runs on the logits (softmax is monotone, so the set is the same
  *     in exact arithmetic, and no exp() rounding can flip an index).
  *   - Within one expert, pairs are ordered by token; no padding.
@@ -148,15 +148,13 @@ void oracle_quant_e4m3(const uint16_t* src, int rows, int cols, int br, uint8_t*
 /* ------------------------------------------------------------- router -- */
 
 #define LANES 32
-#define CHUNK 8
 
 /* One logit in the specified order (see the header comment). */
 static float logit_one(const uint16_t* xrow, const float* wrow, int H) {
   float p[LANES];
   for (int j = 0; j < LANES; ++j) {
     float acc = 0.0f;
-    for (int c = j; c * CHUNK < H; c += LANES)
-      for (int h = c * CHUNK; h < (c + 1) * CHUNK; ++h) acc = fmaf(bf16_to_f32(xrow[h]), wrow[h], acc);
+    for (int h = j; h < H; h += LANES) acc = fmaf(bf16_to_f32(xrow[h]), wrow[h], acc);
     p[j] = acc;
   }
   for (int o = LANES / 2; o >= 1; o /= 2)
@@ -164,7 +162,7 @@ static float logit_one(const uint16_t* xrow, const float* wrow, int H) {
   return p[0];
 }
 
-/* logits [T, E] fp32. H must be a multiple of 8. bias may be NULL. */
+/* logits [T, E] fp32. bias may be NULL. */
 void oracle_router_logits(const uint16_t* x, const float* wr, const float* bias, int T, int H, int E,
                           float* logits, int threads) {
 #ifdef _OPENMP
