@@ -62,6 +62,43 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# --------------------------------------------------------------- traffic --
+# DRAM bytes per launch of the dominant kernel come from an ncu capture whose
+# summary sits under profiles/ with a hash of the kernel's sources at capture
+# time; they are reported only while the sources still hash the same.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_decode_sweep.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "mixture_experts_layer_24_b200", "csrc", f)
+                  for f in ("ffn_gemm.cu", "common.cuh", "internal.h")]
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """(bytes per launch, source note) from the committed capture, or (None, why)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no capture"
+    kv = {}
+    for line in open(TRAFFIC_FILE):
+        if ":" in line and not line.lstrip().startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("workload") != workload:
+        return None, "capture is of another workload"
+    if kv.get("sources_sha256") != kernel_sources_sha256():
+        return None, "kernel changed since the capture"
+    try:
+        return float(kv["dram_bytes_per_launch"]), TRAFFIC_FILE[len(ROOT) + 1:]
+    except (KeyError, ValueError):
+        return None, "capture file incomplete"
+
+
 # ------------------------------------------------------------------ dist --
 
 def dist_env():
@@ -324,6 +361,7 @@ def run_ours(args):
             "gpu_launches": launches, "gpu_launches_per_step": launches / max(args.steps, 1), "clocks": clk}
 
     if world == 1 and not args.no_extras:
+        args.workload_name = workload
         line.update(extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep))
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -349,17 +387,28 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep):
     dn_bytes = sum(t * H * I * 2 + b * K * I * 2 + b * K * H * 4 for t, b in zip(touched, batches))
     gu_ms, gu_n = prof["gate_up"]
     dn_ms, dn_n = prof["down"]
-    per_launch_bytes = gu_bytes / len(batches)
-    achieved = (gu_bytes * steps) / (gu_ms / 1000.0) / 1e9
-    out["roofline"] = {"bound": "hbm", "kernel": "ffn gate/up GEMM + SwiGLU (tcgen05)", "achieved": achieved,
-                       "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+    fu_ms, fu_n = prof["ffn_fused"]
+    if fu_n:
+        # decode batches run both GEMMs in one launch: its bytes are gate/up + down
+        dom_bytes, dom_ms, dom_n = gu_bytes + dn_bytes, fu_ms, fu_n
+        dom_name = "ffn fused gate/up + SwiGLU + down x weight (tcgen05, one launch)"
+    else:
+        dom_bytes, dom_ms, dom_n = gu_bytes, gu_ms, gu_n
+        dom_name = "ffn gate/up GEMM + SwiGLU (tcgen05)"
+    per_launch_bytes = dom_bytes / len(batches)
+    achieved = (dom_bytes * steps) / (dom_ms / 1000.0) / 1e9
+    traffic, traffic_src = measured_traffic(args.workload_name)
+    out["roofline"] = {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
+                       "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                       "traffic_source": traffic_src,
                        "peak_source": f"{peak_kind} hbm_gbs",
                        "algorithmic_bytes_per_launch": per_launch_bytes,
-                       "avg_launch_us": 1000.0 * gu_ms / max(gu_n, 1)}
+                       "avg_launch_us": 1000.0 * dom_ms / max(dom_n, 1)}
     total_ms = sum(v[0] for v in prof.values())
     out["kernels"] = {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1] / steps,
                           "share": v[0] / total_ms if total_ms else 0.0} for k, v in prof.items() if v[1]}
-    out["kernels"]["down"]["achieved_GBps"] = (dn_bytes * steps) / (dn_ms / 1000.0) / 1e9 if dn_ms else None
+    if "down" in out["kernels"]:
+        out["kernels"]["down"]["achieved_GBps"] = (dn_bytes * steps) / (dn_ms / 1000.0) / 1e9 if dn_ms else None
 
     # --- per-batch / prefill breakdown ---
     def kernel_profile(x, reps):

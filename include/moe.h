@@ -250,7 +250,8 @@ typedef enum {
   MOE_PROF_DOWN = 5,    /* down GEMM * routing weight */
   MOE_PROF_QUANT = 6,   /* FP8 quantiser of h */
   MOE_PROF_COMBINE = 7, /* weighted combine */
-  MOE_PROF_KINDS = 8
+  MOE_PROF_FFN_FUSED = 8, /* decode: gate/up + SwiGLU and down * weight in one launch */
+  MOE_PROF_KINDS = 9
 } moe_prof_kind_t;
 
 moe_status_t moe_profile_enable(moe_ctx_t* ctx, int enable);

@@ -33,7 +33,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"]
 
-PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine"]
+PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
 
 class MoeError(RuntimeError):

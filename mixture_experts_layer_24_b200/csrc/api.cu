@@ -141,7 +141,7 @@ namespace {
 
 struct WsLayout {
   size_t logits, rank, chunk_counts, topk_idx, topk_w, counts, offsets, perm_src, perm_k, inv;
-  size_t list_expert, list_map, nt_prefix, x_perm, x_scale, h, hq, h_scale, y_pair, total;
+  size_t list_expert, list_map, nt_prefix, sched, x_perm, x_scale, h, hq, h_scale, y_pair, total;
 };
 
 WsLayout ws_layout(const moe_config_t& c, int T) {
@@ -167,6 +167,7 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
   L.list_expert = take((2 * E + 64) * 4);
   L.list_map = take((2 * E + 64) * 4);
   L.nt_prefix = take((2 * E + 64) * 4);
+  L.sched = take((size_t)fused_sched_entries((int)E) * 4);
   L.x_perm = take(P * H * (fp8 ? 1 : 2));
   L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
   L.h = take(P * I * 2);
@@ -267,7 +268,8 @@ moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void
 moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void* ws, int T, int bn,
                        const int32_t* perm_src, const int32_t* perm_k, const int32_t* offsets, const float* topk_w,
                        float* y_pair, const int32_t* list_expert, const int32_t* list_map, const int32_t* nt_prefix,
-                       int L, int max_ntiles, cudaStream_t s, bool pdl, bool plan_ready_gu) {
+                       int L, int max_ntiles, cudaStream_t s, bool pdl, bool plan_ready_gu,
+                       int* sched = nullptr) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
@@ -296,6 +298,36 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     hmap = hmaps.m[0];
   }
   if (st != MOE_OK) return st;
+  if (sched && !fp8 && bn <= kFusedMaxBn) {
+    // decode: both GEMMs in one launch (x with one K chunk per box, h with two)
+    ActMaps x1;
+    std::memset(&x1, 0, sizeof(x1));
+    for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
+      st = encode_3d_bf16(ctx, &x1.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, 1);
+      if (st != MOE_OK) return st;
+    }
+    GemmArgs a{};
+    a.maps = sl->d_maps;
+    a.list_expert = list_expert;
+    a.list_map = list_map;
+    a.nt_prefix = nt_prefix;
+    a.offsets = offsets;
+    a.L = L;
+    a.H = c.hidden;
+    a.I = c.intermediate;
+    a.K = c.top_k;
+    a.h_out = at<void>(ws, W.h);
+    a.y_out = y_pair;
+    a.topk_w = topk_w;
+    a.perm_src = perm_src;
+    a.perm_k = perm_k;
+    a.status = ctx->d_status;
+    a.sched = sched;
+    a.num_sms = ctx->num_sms;
+    Prof p(ctx, MOE_PROF_FFN_FUSED, s);
+    MOE_CUDA(launch_ffn_fused(bn, x1, hmaps, a, (c.intermediate / 128 + c.hidden / 128) * max_ntiles, s, pdl));
+    return MOE_OK;
+  }
   GemmArgs a{};
   a.maps = sl->d_maps;
   a.list_expert = list_expert;
@@ -485,7 +517,8 @@ moe_status_t permute_impl(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_
     Prof p(ctx, MOE_PROF_PERMUTE, s);
     MOE_CUDA(launch_permute_small(topk_idx, T, c.top_k, c.n_experts, counts, offsets, perm_src, perm_k, inv, map_of,
                                   bn, at<int32_t>(ws, W.list_expert), at<int32_t>(ws, W.list_map),
-                                  at<int32_t>(ws, W.nt_prefix), x, c.hidden, x_perm, ctx->d_status, s, pdl));
+                                  at<int32_t>(ws, W.nt_prefix), x, c.hidden, x_perm, ctx->d_status, s, pdl,
+                                  map_of ? at<int>(ws, W.sched) : nullptr, fused_sched_entries(c.n_experts)));
     if (planned) *planned = map_of != nullptr;
     return MOE_OK;
   }
@@ -536,7 +569,8 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     if (!planned) {
       {
         Prof p(ctx, MOE_PROF_PERMUTE, s);
-        MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl));
+        MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl,
+                                 at<int>(ws, W.sched), fused_sched_entries(E)));
       }
       Prof pg(ctx, MOE_PROF_GATHER, s);
       if (fp8) {
@@ -553,7 +587,7 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
       plan_ready_gu = pdl;  // permutation+plan -> quantiser -> gate/up
     }
     return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
-                     s, ctx->chain, plan_ready_gu);
+                     s, ctx->chain, plan_ready_gu, at<int>(ws, W.sched));
   }
 
   // activation rows in sorted-pair order (quantised for FP8); no PDL on the host-synchronised path

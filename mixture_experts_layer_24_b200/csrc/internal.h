@@ -78,6 +78,8 @@ struct GemmArgs {
   int* status;
   int plan_ready;             // 1: the tile plan was written two or more launches back
                               // (read it, and start streaming weights, before pdl_wait)
+  int* sched;                 // fused decode FFN: [0] tile counter, [1 + n] finished gate/up
+                              // tiles of global N tile n (zeroed by the plan kernel)
   int stages;                 // pipeline depth (set by the launcher)
   int est_tiles;              // host-side bound on the tiles of this launch
   int num_sms;
@@ -95,6 +97,15 @@ struct alignas(64) ActMaps {
 cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const ActMaps* act_maps,
                             const GemmArgs& a, int max_tiles, cudaStream_t s, bool pdl);
 size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn);
+
+// Fused decode FFN (bf16, bn <= 64): gate/up and down tiles of one forward in
+// one persistent launch with a dynamic tile queue. xmaps: x_perm with one K
+// chunk per box; hmaps: h with two. a.sched must be zeroed by the plan kernel.
+cudaError_t launch_ffn_fused(int bn, const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a, int max_tiles,
+                             cudaStream_t s, bool pdl);
+constexpr int kFusedMaxBn = 64;
+// entries of the fused kernel's counter array for a plan of up to n_list experts
+inline int fused_sched_entries(int n_list) { return 1 + 2 * n_list + 64; }
 
 cudaError_t launch_router_logits(const void* x, const float* wr, const float* bias, int T, int H, int E,
                                  float* logits, cudaStream_t s);
@@ -122,7 +133,8 @@ constexpr int kPermuteSmallMaxPairs = 1024;
 cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_t* counts, int32_t* offsets,
                                  int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
                                  int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
-                                 void* x_perm, int* status, cudaStream_t s, bool pdl);
+                                 void* x_perm, int* status, cudaStream_t s, bool pdl, int* sched = nullptr,
+                                 int sched_n = 0);
 
 // Permutation: rank -> scan -> scatter. chunk = tokens per warp-chunk.
 int permute_chunk_tokens(int T, int K);
@@ -136,7 +148,7 @@ cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, cons
 
 // FFN tile plan for the all-resident case: every expert with pairs, in order.
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
-                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl);
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0);
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
                                int H, void* x_perm, cudaStream_t s, bool pdl);

@@ -181,11 +181,13 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
                                                          const int32_t* __restrict__ map_of, int E, int bn,
                                                          int32_t* __restrict__ list_expert,
                                                          int32_t* __restrict__ list_map,
-                                                         int32_t* __restrict__ nt_prefix, int* status) {
+                                                         int32_t* __restrict__ nt_prefix, int* status,
+                                                         int* __restrict__ sched, int sched_n) {
   __shared__ int sh[33];
   pdl_wait();
   pdl_trigger();
   const int e = threadIdx.x;
+  for (int i = e; i < sched_n; i += blockDim.x) sched[i] = 0;  // counters of the fused decode FFN
   int nt = 0;
   if (e < E) {
     const int cnt = offsets[e + 1] - offsets[e];
@@ -205,9 +207,10 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
 }
 
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
-                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl) {
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched,
+                            int sched_n) {
   return launch_ex(ffn_plan_kernel, dim3(1), dim3(1024), 0, s, pdl, offsets, map_of, E, bn, list_expert, list_map,
-                   nt_prefix, status);
+                   nt_prefix, status, sched, sched ? sched_n : 0);
 }
 
 // ----------------------------------------------------------------- gather --
@@ -259,7 +262,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_k,
     int32_t* __restrict__ inv, const int32_t* __restrict__ map_of, int bn, int32_t* __restrict__ list_expert,
     int32_t* __restrict__ list_map, int32_t* __restrict__ nt_prefix, const uint4* __restrict__ x, int vec_per_row,
-    uint4* __restrict__ x_perm, int* status) {
+    uint4* __restrict__ x_perm, int* status, int* __restrict__ sched, int sched_n) {
   __shared__ __align__(16) int s_e[kPermuteSmallMaxPairs];
   __shared__ int s_cnt[1024];
   __shared__ int s_off[1024];
@@ -314,6 +317,7 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
         perm_k[p] = i - (i / K) * K;
       }
     }
+    for (int j = i; j < sched_n; j += blockDim.x) sched[j] = 0;  // counters of the fused decode FFN
     if (map_of) {
       int nt = 0;
       if (i < E) {
@@ -344,13 +348,14 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
 cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_t* counts, int32_t* offsets,
                                  int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
                                  int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
-                                 void* x_perm, int* status, cudaStream_t s, bool pdl) {
+                                 void* x_perm, int* status, cudaStream_t s, bool pdl, int* sched,
+                                 int sched_n) {
   const int P = T * K;
   int ctas = 1;
   if (x_perm) ctas = std::max(1, std::min(64, (P + 31) / 32));
   return launch_ex(permute_small_kernel, dim3(ctas), dim3(1024), 0, s, pdl, idx, T, K, E, counts, offsets, perm_src,
                    perm_k, inv, map_of, bn, list_expert, list_map, nt_prefix, static_cast<const uint4*>(x), H / 8,
-                   static_cast<uint4*>(x_perm), status);
+                   static_cast<uint4*>(x_perm), status, sched, sched ? sched_n : 0);
 }
 
 }  // namespace moe
