@@ -483,14 +483,15 @@ namespace {
 // kernel of the same forward).
 
 moe_status_t route_impl(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
-                        int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s) {
+                        int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, int* sched = nullptr,
+                        int sched_n = 0) {
   const moe_config_t& c = ctx->cfg;
   const WsLayout W = ws_layout(c, T);
   float* logits = at<float>(ws, W.logits);
   if (T <= kRouteSmallMaxT) {
     Prof p(ctx, MOE_PROF_ROUTER, s);
     MOE_CUDA(launch_route_small(x, w_router, logit_bias, T, c.hidden, c.n_experts, c.top_k, logits, topk_idx,
-                                topk_w, ctx->d_counters, ctx->d_status, s, ctx->chain));
+                                topk_w, ctx->d_counters, ctx->d_status, s, ctx->chain, sched, sched_n));
     return MOE_OK;
   }
   {
@@ -541,6 +542,61 @@ moe_status_t permute_impl(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_
                                     perm_src, perm_k, inv, s, ctx->chain));
   }
   return MOE_OK;
+}
+
+// Decode FFN planned inside the kernel from the router's top-k (no permutation
+// kernel, no gathered x). The caller checked decode_path_ok().
+moe_status_t ffn_decode_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* idx, const float* topk_w,
+                             int T, float* y_pair, void* ws, cudaStream_t s, int* sched) {
+  const moe_config_t& c = ctx->cfg;
+  const WsLayout W = ws_layout(c, T);
+  const int E = c.n_experts, P = T * c.top_k;
+  const int tp = std::min(64, (T + 15) / 16 * 16 == 48 ? 64 : (T + 15) / 16 * 16);
+  std::lock_guard<std::mutex> lock(sl->mu);
+  sl->stats.calls++;
+  sl->stats.last_cold = 0;
+  sl->stats.last_touched = -1;
+  CUtensorMap xmap;
+  moe_status_t st = encode_3d_bf16(ctx, &xmap, x, c.hidden, T, tp, 1);
+  if (st != MOE_OK) return st;
+  ActMaps hmaps;
+  std::memset(&hmaps, 0, sizeof(hmaps));
+  for (int i = 0, rows = 16; rows <= tp; ++i, rows <<= 1) {
+    st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, 2);
+    if (st != MOE_OK) return st;
+  }
+  GemmArgs a{};
+  a.maps = sl->d_maps;
+  a.H = c.hidden;
+  a.I = c.intermediate;
+  a.K = c.top_k;
+  a.h_out = at<void>(ws, W.h);
+  a.y_out = y_pair;
+  a.topk_w = topk_w;
+  a.status = ctx->d_status;
+  a.sched = sched;
+  a.num_sms = ctx->num_sms;
+  DecodeArgs d{};
+  d.topk_idx = idx;
+  d.map_of = sl->d_map_of;
+  d.T = T;
+  d.E = E;
+  d.counts = at<int32_t>(ws, W.counts);
+  d.offsets = at<int32_t>(ws, W.offsets);
+  d.perm_src = at<int32_t>(ws, W.perm_src);
+  d.perm_k = at<int32_t>(ws, W.perm_k);
+  d.inv = at<int32_t>(ws, W.inv);
+  Prof p(ctx, MOE_PROF_FFN_FUSED, s);
+  MOE_CUDA(launch_ffn_decode(xmap, hmaps, a, d, (c.intermediate / 128 + c.hidden / 128) * std::min(E, P), s,
+                             ctx->chain));
+  return MOE_OK;
+}
+
+bool decode_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, int T) {
+  const moe_config_t& c = ctx->cfg;
+  return c.wdtype == MOE_BF16 && sl->n_host == 0 && T >= 1 && T <= kDecodeMaxT &&
+         (long long)T * c.top_k <= kDecodeMaxPairs && ((uintptr_t)x % 16) == 0 &&
+         ffn_decode_smem_bytes(T, c.n_experts) <= 232448;
 }
 
 // Expert FFN. `planned`: the permutation step already wrote the tile plan and
@@ -771,6 +827,16 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
   float* y = at<float>(ws, W.y_pair);
   const bool resident = sl->n_host == 0;
   const bool chain = ctx->chain;
+  if (decode_path_ok(ctx, sl, x, T)) {
+    // decode: router (which also zeroes the FFN's counters) -> FFN planned from the top-k -> combine
+    int* sched = at<int>(ws, W.sched);
+    const int sched_n = 1 + std::min(c.n_experts, T * c.top_k);
+    if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n)) != MOE_OK) return st;
+    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched)) != MOE_OK) return st;
+    Prof p(ctx, MOE_PROF_COMBINE, s);
+    MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, chain));
+    return MOE_OK;
+  }
   // route (first kernel: ordinary stream order with whatever came before)
   if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s)) != MOE_OK) return st;
   // permutation (+ tile plan + sorted bf16 rows when the batch is small)

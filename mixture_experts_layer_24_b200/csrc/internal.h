@@ -104,6 +104,26 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn);
 cudaError_t launch_ffn_fused(int bn, const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a, int max_tiles,
                              cudaStream_t s, bool pdl);
 constexpr int kFusedMaxBn = 64;
+
+// The decode forward's FFN planned from the router's top-k inside the kernel
+// (no permutation kernel, no gathered x): T <= 64 tokens, T*K <= 512 pairs,
+// bf16, every expert resident, x 16-byte aligned. xmap: x [T, H] with box
+// {64, TP, 1}, TP = T rounded up to 16 (48 -> 64); hmaps: h, two K chunks.
+// a.sched: [0] tile counter, [1 + l] per touched expert, zeroed by the router.
+struct DecodeArgs {
+  const int32_t* topk_idx;  // [T*K] from the router
+  const int32_t* map_of;    // [E] expert -> slot (map entry), -1 if not registered
+  int T, E;
+  int32_t* counts;          // [E]    written by CTA 0
+  int32_t* offsets;         // [E+1]
+  int32_t* perm_src;        // [P]
+  int32_t* perm_k;          // [P]
+  int32_t* inv;             // [P]
+};
+cudaError_t launch_ffn_decode(const CUtensorMap& xmap, const ActMaps& hmaps, const GemmArgs& a, const DecodeArgs& d,
+                              int max_tiles, cudaStream_t s, bool pdl);
+size_t ffn_decode_smem_bytes(int T, int E);
+constexpr int kDecodeMaxT = 64, kDecodeMaxPairs = 512;
 // entries of the fused kernel's counter array for a plan of up to n_list experts
 inline int fused_sched_entries(int n_list) { return 1 + 2 * n_list + 64; }
 
@@ -118,7 +138,7 @@ cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, 
 constexpr int kRouteSmallMaxT = 64;
 cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                                float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl);
+                               cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0);
 // Prefill-regime router logits (register-tiled fp32 GEMM in the same order).
 cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias, int T, int H, int E,
                               float* logits, cudaStream_t s);

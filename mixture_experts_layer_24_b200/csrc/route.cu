@@ -273,13 +273,16 @@ template <int WT, int WE, int NWT, int NWE>
 __global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
                                                                         const float* __restrict__ wr,
                                                                         const float* __restrict__ bias, int T, int H,
-                                                                        int E, float* __restrict__ logits) {
+                                                                        int E, float* __restrict__ logits,
+                                                                        int* __restrict__ sched, int sched_n) {
   using C = RgCfg<WT, WE, NWT, NWE>;
   constexpr int TT = C::TT, TE = C::TE, NT = C::kThreads;
   extern __shared__ __align__(16) uint8_t sm[];
   pdl_wait();  // x may come from the previous kernel
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0 && blockIdx.y == 0)  // counters of the decode FFN that follows (first kernel of the forward)
+    for (int i = tid; i < sched_n; i += NT) sched[i] = 0;
   const int tt0 = (warp / NWE) * WT, ee0 = (warp % NWE) * WE;
   const int tb = blockIdx.y * TT, eb = blockIdx.x * TE;
   const int nsteps = H / 256;
@@ -357,14 +360,14 @@ __global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uin
 
 template <int WT, int WE, int NWT, int NWE>
 static cudaError_t launch_rg(const void* x, const float* wr, const float* bias, int T, int H, int E, float* logits,
-                             cudaStream_t s, bool pdl) {
+                             cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0) {
   using C = RgCfg<WT, WE, NWT, NWE>;
   auto kern = route_gemm_kernel<WT, WE, NWT, NWE>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (err != cudaSuccess) return err;
   dim3 grid((E + C::TE - 1) / C::TE, (T + C::TT - 1) / C::TT);
   return launch_ex(kern, grid, dim3(C::kThreads), C::kSmem, s, pdl, static_cast<const uint16_t*>(x), wr, bias, T, H,
-                   E, logits);
+                   E, logits, sched, sched ? sched_n : 0);
 }
 
 static bool rg_tile_ok(const void* x, const float* wr, int H) {
@@ -399,11 +402,14 @@ __global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16
                                                                      int E, int K, float* __restrict__ logits,
                                                                      int32_t* __restrict__ idx, float* __restrict__ w,
                                                                      unsigned int* __restrict__ counters,
-                                                                     int fuse_topk, int* status) {
+                                                                     int fuse_topk, int* status,
+                                                                     int* __restrict__ sched, int sched_n) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
   pdl_trigger();  // first kernel of a forward: the next one may launch (it waits for us)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && blockIdx.y == 0)  // counters of the decode FFN that follows
+    for (int i = threadIdx.x; i < sched_n; i += blockDim.x) sched[i] = 0;
   const int e0 = blockIdx.x * kRsWarps, e = e0 + warp;
   const int t0 = blockIdx.y * TG;
   const int ntok = min(TG, T - t0), nexp = min(kRsWarps, E - e0);
@@ -468,14 +474,15 @@ __global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16
 template <int TG>
 static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                              float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, int* status,
-                             cudaStream_t s) {
+                             cudaStream_t s, int* sched, int sched_n) {
   const size_t smem = route_small_smem(TG, H);
   cudaError_t err = cudaFuncSetAttribute(route_small_kernel<TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((E + kRsWarps - 1) / kRsWarps, (T + TG - 1) / TG);
   return launch_ex(route_small_kernel<TG>, grid, dim3(kRsWarps * 32), smem, s, false,
-                   static_cast<const uint16_t*>(x), wr, bias, T, H, E, K, logits, idx, w, counters, fuse, status);
+                   static_cast<const uint16_t*>(x), wr, bias, T, H, E, K, logits, idx, w, counters, fuse, status,
+                   sched, sched ? sched_n : 0);
 }
 
 // T <= 8: logits + fused top-k in one launch; up to 64 tokens: logits in
@@ -484,25 +491,31 @@ static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, 
 // memory) go through the direct kernel.
 cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                                float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl) {
+                               cudaStream_t s, bool pdl, int* sched, int sched_n) {
   if (T <= 0) return cudaSuccess;
   const bool bulk_ok = ((uintptr_t)x % 16 == 0) && ((uintptr_t)wr % 16 == 0) && (H % 8 == 0) &&
                        route_small_smem(8, H) <= 200 * 1024;
   if (!bulk_ok) {
+    if (sched) cudaMemsetAsync(sched, 0, sizeof(int) * sched_n, s);
     cudaError_t err = launch_router_logits(x, wr, bias, T, H, E, logits, s);
     if (err != cudaSuccess) return err;
     return launch_topk_warp(logits, T, E, K, idx, w, s, false);
   }
-  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
-  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
-  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
-  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s);
+  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
+  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
+  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
+  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
   // more tokens: W rows would be staged once per 8-token group; register
   // tiles reuse each loaded element across 4 tokens and 4 or 8 experts
   cudaError_t err;
-  if (!rg_tile_ok(x, wr, H)) err = launch_router_logits(x, wr, bias, T, H, E, logits, s);
-  else if (T <= 16) err = launch_rg<4, 4, 2, 2>(x, wr, bias, T, H, E, logits, s, false);
-  else err = launch_rg<4, 8, 2, 2>(x, wr, bias, T, H, E, logits, s, false);
+  if (!rg_tile_ok(x, wr, H)) {
+    if (sched) cudaMemsetAsync(sched, 0, sizeof(int) * sched_n, s);
+    err = launch_router_logits(x, wr, bias, T, H, E, logits, s);
+  } else if (T <= 16) {
+    err = launch_rg<4, 4, 2, 2>(x, wr, bias, T, H, E, logits, s, false, sched, sched_n);
+  } else {
+    err = launch_rg<4, 8, 2, 2>(x, wr, bias, T, H, E, logits, s, false, sched, sched_n);
+  }
   if (err != cudaSuccess) return err;
   return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
 }
