@@ -1553,6 +1553,448 @@ cudaError_t launch_ffn_decode(const CUtensorMap& xmap, const ActMaps& hmaps, con
   return cudaErrorInvalidValue;
 }
 
+// ============================================================== fused fp8 decode
+// FP8 counterpart of ffn_bf16_fused_kernel: gate/up and down tiles of one
+// forward in one persistent launch with the same dynamic queue and per-N-tile
+// dependency counters. The gate/up epilogue also does the activation
+// quantisation of h: for each pair its 128 h values of the tile are one
+// 128-column scale block, so amax (a max over the 4 row-quarter warps), the
+// scale s = amax / 448 (1 for an all-zero block) and the e4m3 codes of the
+// bf16-rounded h are formed right there, with the arithmetic of
+// quant_rows_kernel, and written to hq and h_scale; the bf16 h is not stored.
+// Per-K-block promotion as in ffn_fp8_kernel.
+
+template <int BN>
+struct Fp8FusedCfg {
+  static constexpr uint32_t kStageBytes = 2 * kABytes + BN * 128;  // gate/up; down uses kABytes + BN * 128
+  static constexpr int kMaxKB = 64;
+  // activation scales [BN][64], weight scales [2][64], routing weights [BN], amax partials [4][BN]
+  static constexpr uint32_t kScaleBytes = BN * kMaxKB * 4 + 2 * kMaxKB * 4 + BN * 4 + 4 * BN * 4;
+  static constexpr int kStagesRaw = (212 * 1024 - (int)kScaleBytes) / (int)kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kRing = 8;
+  static constexpr int kNpRaw = 512 / (2 * BN);
+  static constexpr int NP = kNpRaw > 8 ? 8 : kNpRaw;
+  static constexpr uint32_t kTmemCols = tmem_cols_for(NP * 2 * BN);
+  static constexpr size_t kSmem =
+      1024 + (size_t)kStages * kStageBytes + kScaleBytes + 8 * (2 * kStages + 2 * NP + 2 * kRing) + 4 * kRing + 64;
+  static_assert(kStages >= 2 && NP >= 2, "FP8 pipeline needs two stages and two partial buffers");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_constant__ ActMaps xact,
+                                                               const __grid_constant__ ActMaps hact,
+                                                               const GemmArgs a) {
+  using C = Fp8FusedCfg<BN>;
+  constexpr int S = C::kStages, NP = C::NP, R = C::kRing;
+  constexpr uint32_t STAGE = C::kStageBytes;
+  constexpr int HALF = BN / 2;
+  constexpr int NCH = HALF >= 16 ? HALF / 16 : 1;
+  constexpr int CW = HALF >= 16 ? 16 : HALF;
+  const int mg = a.I / 128, md = a.H / 128;
+  const int KBg = a.H / 128, KBd = a.I / 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  pdl_wait();  // the plan, the quantised x and the counters come from earlier kernels of the forward
+  pdl_trigger();
+  const int NT = a.nt_prefix[a.L];
+  const int Gt = NT * mg, total = Gt + NT * md;
+  const bool stand_down = a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT);
+  if ((int)blockIdx.x >= total || stand_down) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  float* s_act = reinterpret_cast<float*>(gbase + S * STAGE);  // [BN][KB]
+  float* s_w = s_act + BN * C::kMaxKB;                         // [2][KB]
+  float* wcol = s_w + 2 * C::kMaxKB;                           // [BN]
+  float* s_amax = wcol + BN;                                   // [4][BN]
+  const uint32_t bars = base + S * STAGE + C::kScaleBytes;
+  auto full = [&](int s) { return bars + 8u * s; };
+  auto empty = [&](int s) { return bars + 8u * (S + s); };
+  auto pfull = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto pempty = [&](int b) { return bars + 8u * (2 * S + NP + b); };
+  auto rfull = [&](int r) { return bars + 8u * (2 * S + 2 * NP + r); };
+  auto rempty = [&](int r) { return bars + 8u * (2 * S + 2 * NP + R + r); };
+  uint8_t* after = gbase + S * STAGE + C::kScaleBytes + 8 * (2 * S + 2 * NP + 2 * R);
+  volatile int* ring = reinterpret_cast<volatile int*>(after);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(after + 4 * R);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ep_abort = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < NP; ++b) {
+      mbar_init(pfull(b), 1);
+      mbar_init(pempty(b), 8);
+    }
+    for (int r = 0; r < R; ++r) {
+      mbar_init(rfull(r), 1);
+      mbar_init(rempty(r), 9);  // the MMA issuer and the eight epilogue warps
+    }
+    *abort_flag = 0;
+    *ep_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
+      int issued = 0;
+      int tile = blockIdx.x;
+      auto fail = [&]() {
+        *abort_flag = 1;
+        flag_status(a.status, MOE_DEV_TIMEOUT);
+      };
+      for (int j = 0;; ++j) {
+        const int slot = j % R;
+        if (j >= R && !mbar_wait(rempty(slot), ((j / R) - 1) & 1)) {
+          fail();
+          break;
+        }
+        const int pub = (tile < total && !*abort_flag) ? tile : -1;
+        ring[slot] = pub;
+        mbar_arrive(rfull(slot));
+        if (pub < 0) break;
+        const bool gu = tile < Gt;
+        TileInfo ti;
+        decode_tile_at(a, gu ? mg : md, BN, gu ? tile : tile - Gt, ti);
+        const int wi = tile_width_index(ti.nvalid, BN);
+        const uint64_t pol_w = ti.nti > 1 ? pol_shared : pol_once;
+        const MapEntry* me = a.maps + ti.mapi;
+        bool ok = true;
+        if (gu) {
+          const void* wmap = &me->gu;
+          const void* amap = &xact.m[wi];
+          const uint32_t tx = 2 * kABytes + (16u << wi) * 128u;
+          tensormap_acquire(wmap);
+          for (int kb = 0; kb < KBg; ++kb, ++issued) {
+            const int s = issued % S;
+            if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            const uint32_t st = base + s * STAGE;
+            mbar_arrive_expect_tx(full(s), tx);
+            tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+            tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
+            tma_load_2d(st + 2 * kABytes, amap, full(s), kb * 128, ti.row0);
+          }
+        } else {
+          const void* wmap = &me->dn;
+          const void* amap = &hact.m[wi];
+          const uint32_t tx = kABytes + (16u << wi) * 128u;
+          tensormap_acquire(wmap);
+          const int npre = KBd < S ? KBd : S;
+          int kb = 0;
+          for (; kb < npre; ++kb) {
+            const int n = issued + kb, s = n % S;
+            if (n >= S && !mbar_wait(empty(s), ((n / S) - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full(s), tx);
+            tma_load_2d_hint(base + s * STAGE, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+          }
+          if (ok) {
+            const int* dep = a.sched + 1 + ti.ng;
+            const uint64_t t0 = global_timer_ns();
+            while (ld_acquire_gpu(dep) < mg) {
+              if (global_timer_ns() - t0 > kWaitLimitNs) {
+                ok = false;
+                break;
+              }
+              __nanosleep(64);
+            }
+          }
+          if (ok) {
+            fence_proxy_async_global();
+            for (int j2 = 0; j2 < npre; ++j2) {
+              const int s = (issued + j2) % S;
+              tma_load_2d(base + s * STAGE + kABytes, amap, full(s), j2 * 128, ti.row0);
+            }
+            issued += npre;
+            for (; kb < KBd; ++kb, ++issued) {
+              const int s = issued % S;
+              if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
+                ok = false;
+                break;
+              }
+              const uint32_t st = base + s * STAGE;
+              mbar_arrive_expect_tx(full(s), tx);
+              tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+              tma_load_2d(st + kABytes, amap, full(s), kb * 128, ti.row0);
+            }
+          } else {
+            issued += kb;
+          }
+        }
+        if (!ok) {
+          fail();
+          tile = total;
+          continue;
+        }
+        tile = (int)gridDim.x + atomicAdd(a.sched, 1);
+      }
+      for (int g = issued - S < 0 ? 0 : issued - S; g < issued; ++g) mbar_wait(full(g % S), (g / S) & 1);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int consumed = 0, kp = 0;
+      bool ok = true;
+      for (int j = 0; ok; ++j) {
+        const int slot = j % R;
+        if (!mbar_wait(rfull(slot), (j / R) & 1)) {
+          ok = false;
+          break;
+        }
+        const int tile = ring[slot];
+        mbar_arrive(rempty(slot));
+        if (tile < 0) break;
+        const bool gu = tile < Gt;
+        TileInfo ti;
+        decode_tile_at(a, gu ? mg : md, BN, gu ? tile : tile - Gt, ti);
+        const int width = 16 << tile_width_index(ti.nvalid, BN);
+        const uint32_t idesc = instr_desc(128, width, 0u);
+        const uint32_t b_off = gu ? 2 * kABytes : kABytes;
+        const int KB = gu ? KBg : KBd;
+        for (int kb = 0; kb < KB; ++kb, ++consumed, ++kp) {
+          const int s = consumed % S, pb = kp % NP;
+          ok = mbar_wait(full(s), (consumed / S) & 1);
+          if (ok && kp >= NP) ok = mbar_wait(pempty(pb), ((kp / NP) - 1) & 1);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t st = base + s * STAGE;
+          const uint32_t dd = tmem + static_cast<uint32_t>(pb * 2 * BN);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t bdesc = sw128_kmajor_desc(st + b_off + k * 32);
+            const uint32_t acc = k != 0 ? 1u : 0u;
+            tc_mma_e4m3(dd, sw128_kmajor_desc(st + k * 32), bdesc, idesc, acc);
+            if (gu) tc_mma_e4m3(dd + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, idesc, acc);
+          }
+          tc_commit(empty(s));
+          tc_commit(pfull(pb));
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_status(a.status, MOE_DEV_TIMEOUT);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0..7)
+    // warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const int et = threadIdx.x;  // 0..255
+    const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int c0 = hf * HALF;
+    bool aborted = false;  // warp-uniform
+    int kp = 0;
+    for (int j = 0;; ++j) {
+      const int slot = j % R;
+      int tile = -1;
+      if (lane == 0) {
+        if (!*abort_flag && mbar_wait(rfull(slot), (j / R) & 1)) {
+          tile = ring[slot];
+          mbar_arrive(rempty(slot));
+        } else {
+          *ep_abort = 1;
+        }
+      }
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      named_bar_sync(2, 256);  // the eight warps leave together or not at all
+      if (*ep_abort) {
+        flag_status(a.status, MOE_DEV_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      if (tile < 0) break;
+      const bool gu = tile < Gt;
+      TileInfo ti;
+      decode_tile_at(a, gu ? mg : md, BN, gu ? tile : tile - Gt, ti);
+      const int width = 16 << tile_width_index(ti.nvalid, BN);
+      const int KB = gu ? KBg : KBd;
+      const MapEntry* me = a.maps + ti.mapi;
+      const float* sw = gu ? me->s_gu : me->s_dn;
+      named_bar_sync(1, 256);  // the previous tile's readers are done with the tables
+      if (!gu && et == 0) {
+        // h scales of this N tile come from its gate/up tiles (the producer waited for their h codes)
+        const int* dep = a.sched + 1 + ti.ng;
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire_gpu(dep) < mg) {
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            flag_status(a.status, MOE_DEV_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      named_bar_sync(1, 256);
+      const float* act_scale = gu ? a.act_scale : a.h_scale;
+      for (int i = et; i < BN * KB; i += 256) {  // through L2: h scales are written during this launch
+        const int n = i / KB, kb = i - n * KB;
+        s_act[n * KB + kb] = n < ti.nvalid ? __ldcg(act_scale + (size_t)(ti.row0 + n) * KB + kb) : 0.0f;
+      }
+      for (int i = et; i < (gu ? 2 : 1) * KB; i += 256) {
+        const int which = i / KB, kb = i - which * KB;
+        const int rb = which == 0 ? ti.mt : a.I / 128 + ti.mt;
+        s_w[which * KB + kb] = sw[(size_t)rb * KB + kb];
+      }
+      if (!gu) {
+        for (int n = et; n < BN; n += 256) {
+          float wv = 0.0f;
+          if (n < ti.nvalid) {
+            const int p = ti.row0 + n;
+            wv = __ldg(a.topk_w + (size_t)__ldg(a.perm_src + p) * a.K + __ldg(a.perm_k + p));
+          }
+          wcol[n] = wv;
+        }
+      }
+      named_bar_sync(1, 256);
+
+      float accg[HALF], accu[HALF];
+#pragma unroll
+      for (int i = 0; i < HALF; ++i) {
+        accg[i] = 0.0f;
+        accu[i] = 0.0f;
+      }
+      for (int kb = 0; kb < KB; ++kb, ++kp) {
+        const int pb = kp % NP;
+        if (!aborted) {
+          bool ok = !*abort_flag && mbar_wait(pfull(pb), (kp / NP) & 1);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
+            aborted = true;
+            if (lane == 0) {
+              *abort_flag = 1;
+              flag_status(a.status, MOE_DEV_TIMEOUT);
+            }
+          }
+        }
+        if (!aborted) {
+          tc_fence_after();
+          const float swg = s_w[kb];
+          const float swu = gu ? s_w[KB + kb] : 0.0f;
+          const uint32_t pbase = tl + static_cast<uint32_t>(pb * 2 * BN);
+#pragma unroll
+          for (int ch = 0; ch < NCH; ++ch) {
+            const int cstart = CW == 16 ? c0 + ch * 16 : 0;
+            if (cstart < width) {
+              uint32_t pg[16], pu[16];
+              tmem_ld16(pbase + cstart, pg);
+              if (gu) tmem_ld16(pbase + BN + cstart, pu);
+              tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < CW; ++q) {
+                const int col = ch * CW + q;
+                const int n = c0 + col;
+                const uint32_t gb = CW == 16 ? pg[q] : (hf ? pg[(CW + q) & 15] : pg[q]);
+                const float sa = s_act[n * KB + kb];
+                accg[col] = fmaf(__uint_as_float(gb), sa * swg, accg[col]);
+                if (gu) {
+                  const uint32_t ub = CW == 16 ? pu[q] : (hf ? pu[(CW + q) & 15] : pu[q]);
+                  accu[col] = fmaf(__uint_as_float(ub), sa * swu, accu[col]);
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pempty(pb));
+      }
+      if (gu) {
+        // h = bf16(silu(g) * u), then its e4m3 block code: amax over the tile's 128 rows per pair
+        const int jj = ti.mt * 128 + r;
+        float hv[HALF];
+#pragma unroll
+        for (int col = 0; col < HALF; ++col) {
+          const int n = c0 + col;
+          float h = 0.0f;
+          if (n < ti.nvalid) {
+            const float gv = accg[col], uv = accu[col];
+            h = __bfloat162float(__float2bfloat16_rn(gv / (1.0f + expf(-gv)) * uv));
+          }
+          hv[col] = h;
+          float m = fabsf(h);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) s_amax[q4 * BN + n] = m;
+        }
+        named_bar_sync(1, 256);
+        uint8_t* hq = static_cast<uint8_t*>(a.h_out);
+#pragma unroll
+        for (int col = 0; col < HALF; ++col) {
+          const int n = c0 + col;
+          if (n < ti.nvalid && !aborted) {
+            const float amax = fmaxf(fmaxf(s_amax[n], s_amax[BN + n]), fmaxf(s_amax[2 * BN + n], s_amax[3 * BN + n]));
+            const float sc = (amax == 0.0f) ? 1.0f : amax / 448.0f;
+            const int p = ti.row0 + n;
+            hq[(size_t)p * a.I + jj] =
+                static_cast<uint8_t>(__nv_cvt_float_to_fp8(hv[col] / sc, __NV_SATFINITE, __NV_E4M3));
+            if (r == 0) a.h_scale[(size_t)p * KBd + ti.mt] = sc;
+          }
+        }
+        __threadfence();
+        named_bar_sync(1, 256);
+        if (et == 0 && !*abort_flag) atomicAdd(a.sched + 1 + ti.ng, 1);
+      } else if (!aborted) {
+        const int o = ti.mt * 128 + r;
+#pragma unroll
+        for (int col = 0; col < HALF; ++col) {
+          const int n = c0 + col;
+          if (n < ti.nvalid) a.y_out[(size_t)(ti.row0 + n) * a.H + o] = wcol[n] * accg[col];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN>
+static cudaError_t launch_fp8_fused(const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a, int grid,
+                                    cudaStream_t s, bool pdl) {
+  using C = Fp8FusedCfg<BN>;
+  cudaError_t err = cudaFuncSetAttribute(ffn_fp8_fused_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmem);
+  if (err != cudaSuccess) return err;
+  const int persistent = grid < a.num_sms ? grid : a.num_sms;
+  if (persistent <= 0) return cudaSuccess;
+  return launch_ex(ffn_fp8_fused_kernel<BN>, dim3(persistent), dim3(320), C::kSmem, s, pdl, xmaps, hmaps, a);
+}
+
+cudaError_t launch_ffn_fp8_fused(int bn, const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a,
+                                 int max_tiles, cudaStream_t s, bool pdl) {
+  switch (bn) {
+    case 16: return launch_fp8_fused<16>(xmaps, hmaps, a, max_tiles, s, pdl);
+    case 32: return launch_fp8_fused<32>(xmaps, hmaps, a, max_tiles, s, pdl);
+    case 64: return launch_fp8_fused<64>(xmaps, hmaps, a, max_tiles, s, pdl);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <int BN>
 static cudaError_t launch_fused(const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a, int grid,
                                 cudaStream_t s, bool pdl) {

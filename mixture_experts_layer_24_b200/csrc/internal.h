@@ -104,6 +104,10 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn);
 cudaError_t launch_ffn_fused(int bn, const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a, int max_tiles,
                              cudaStream_t s, bool pdl);
 constexpr int kFusedMaxBn = 64;
+// FP8 counterpart (the gate/up epilogue also quantises h into a.h_out (e4m3
+// codes [P, I]) and a.h_scale): xmaps over the e4m3 x rows, hmaps over hq.
+cudaError_t launch_ffn_fp8_fused(int bn, const ActMaps& xmaps, const ActMaps& hmaps, const GemmArgs& a,
+                                 int max_tiles, cudaStream_t s, bool pdl);
 
 // The decode forward's FFN planned from the router's top-k inside the kernel
 // (no permutation kernel, no gathered x): T <= 64 tokens, T*K <= 512 pairs,
