@@ -18,6 +18,20 @@ namespace moe {
 
 __device__ __forceinline__ float bf16_lo(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
+// Two fp32 values in one 64-bit register, and the paired fused multiply-add
+// (two independent IEEE fmaf with round-to-nearest, one instruction).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void fma2(uint64_t& c, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(c) : "l"(a), "l"(b));
+}
+
 __device__ __forceinline__ void butterfly_sum(float& v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
@@ -304,11 +318,12 @@ __global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uin
     }
   };
 
-  float acc[WT][WE];
+  static_assert(WT % 2 == 0, "tokens go in pairs");
+  uint64_t acc2[WT / 2][WE];  // (token 2m, token 2m+1) partials of expert j
 #pragma unroll
-  for (int i = 0; i < WT; ++i)
+  for (int m = 0; m < WT / 2; ++m)
 #pragma unroll
-    for (int j = 0; j < WE; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < WE; ++j) acc2[m][j] = 0ull;
 
 #pragma unroll
   for (int st = 0; st < kRgStages - 1; ++st) {
@@ -328,18 +343,25 @@ __global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uin
     const float* wb = ws(buf) + (size_t)ee0 * 256 + lane;
 #pragma unroll 2
     for (int q = 0; q < 8; ++q) {
-      float xf[WT];
+      uint64_t xp[WT / 2];
 #pragma unroll
-      for (int i = 0; i < WT; ++i) xf[i] = bf16_lo(xb[(size_t)i * 256 + 32 * q]);
+      for (int m = 0; m < WT / 2; ++m)
+        xp[m] = pack2(bf16_lo(xb[(size_t)(2 * m) * 256 + 32 * q]), bf16_lo(xb[(size_t)(2 * m + 1) * 256 + 32 * q]));
 #pragma unroll
       for (int j = 0; j < WE; ++j) {
         const float wv = wb[(size_t)j * 256 + 32 * q];
+        const uint64_t wp = pack2(wv, wv);
 #pragma unroll
-        for (int i = 0; i < WT; ++i) acc[i][j] = fmaf(xf[i], wv, acc[i][j]);
+        for (int m = 0; m < WT / 2; ++m) fma2(acc2[m][j], xp[m], wp);
       }
     }
     __syncthreads();
   }
+  float acc[WT][WE];
+#pragma unroll
+  for (int m = 0; m < WT / 2; ++m)
+#pragma unroll
+    for (int j = 0; j < WE; ++j) unpack2(acc2[m][j], acc[2 * m][j], acc[2 * m + 1][j]);
 #pragma unroll
   for (int i = 0; i < WT; ++i)
 #pragma unroll
