@@ -564,11 +564,16 @@ def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
     return out
 
 
-def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_spare=32):
-    """120 of the 384 experts resident (greedy hot set from a seeded 2048-token
-    routing histogram), the other 264 in pinned host memory staged through 32
-    spare HBM slots on demand: decode B=1, B=4 and a 4096-token chunk. Bound:
-    max(resident bytes / HBM, staged bytes / measured pinned H2D rate)."""
+def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_spare=32, n_cache_all=128):
+    """Expert residency with the spare slots as an LRU cache of host-resident experts.
+
+    "hot set": 120 of the 384 experts resident (greedy hot set from a seeded
+    2048-token routing histogram), the other 264 in pinned host memory behind 32
+    spare HBM slots. "all through the cache": every expert in pinned host
+    memory behind 128 slots. Decode runs a stream of forwards over new tokens
+    (so hits come from routing locality, not from repeating a batch): 4
+    forwards fill the cache, the next 20 are timed. Bound per forward:
+    max(HBM-read bytes / HBM, copied bytes / measured pinned H2D rate)."""
     import mixture_experts_layer_24_b200 as M
     probe = M.MoeLayer(H, E, K, I, device=device)
     for e in range(E):
@@ -578,16 +583,7 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
     hist = torch.bincount(idx.reshape(-1).long(), minlength=E).cpu()
     hot = set(M.moe_plan_hot_set(hist, n_hot).tolist())
     probe.close()
-    layer = M.MoeLayer(H, E, K, I, n_spare_slots=n_spare, device=device)
-    host = {}
-    for e in range(E):
-        g, d = keep[e]
-        if e in hot:
-            layer.register(e, g, d)
-        else:
-            hg, hd = g.cpu().pin_memory(), d.cpu().pin_memory()
-            host[e] = (hg, hd)
-            layer.register(e, hg, hd, None, None, M.MOE_LOC_HOST_PINNED)
+    host = {e: tuple(t.cpu().pin_memory() for t in keep[e]) for e in range(E)}
     # pinned host -> HBM rate on this machine: 400 MB copies after one warm-up copy, best of three
     src = torch.empty(200 << 20, dtype=torch.bfloat16).pin_memory()
     dst = torch.empty_like(src, device=device)
@@ -604,23 +600,60 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
     h2d_gbs = src.numel() * 2 / (best_ms / 1000) / 1e9
     del src, dst
     out = {"hotcold_h2d_GBps": h2d_gbs}
-    for T in (1, 4, 4096):
-        x = synth.tokens(T, H, seed=SEED, device=device, first_token=610000)
-        time_forwards(layer, [x], wr, bias, flush, stream, 1)
-        reps = 3
-        ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
-        st = layer.stats()
-        cold = st["last_cold"]
-        touched = st["last_touched"]
-        hot_bytes = (touched - cold) * EXPERT_BYTES
-        cold_bytes = cold * EXPERT_BYTES
-        bound_s = max(hot_bytes / (hbm * 1e9), cold_bytes / (h2d_gbs * 1e9))
-        out[f"hotcold_B{T}" if T < 4096 else "hotcold_prefill4096"] = {
-            "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": touched,
-            "cold_experts_staged": cold, "cold_bytes": cold_bytes,
-            "roofline_frac": bound_s / (ms / 1000) if ms > 0 else None}
+
+    def stream_of(layer, T, n_fill=4, n_time=20, base=610000):
+        ms_tot, bound_tot, hits, routed, copied, touched_tot = 0.0, 0.0, 0, 0, 0, 0
+        for i in range(n_fill + n_time):
+            x = synth.tokens(T, H, seed=SEED, device=device, first_token=base + 1000 * i)
+            ms = time_forwards(layer, [x], wr, bias, flush, stream, 1)
+            if i < n_fill:
+                continue
+            st = layer.stats()
+            ms_tot += ms
+            hits += st["last_hits"]
+            routed += st["last_routed_cold"]
+            copied += st["last_cold"]
+            touched_tot += st["last_touched"]
+            hbm_bytes = st["last_touched"] * EXPERT_BYTES
+            bound_tot += max(hbm_bytes / (hbm * 1e9), st["last_cold"] * EXPERT_BYTES / (h2d_gbs * 1e9))
+        return {"us_per_layer": 1000 * ms_tot / n_time, "tokens_per_s": T * n_time / (ms_tot / 1000),
+                "touched_experts_mean": touched_tot / n_time, "host_experts_routed_mean": routed / n_time,
+                "copied_experts_mean": copied / n_time, "hit_rate": hits / routed if routed else None,
+                "roofline_frac": bound_tot / (ms_tot / 1000) if ms_tot > 0 else None,
+                "sample": f"{n_time} forwards over new tokens after {n_fill} that fill the cache"}
+
+    # ---- hot set + LRU cache of the rest
+    layer = M.MoeLayer(H, E, K, I, n_spare_slots=n_spare, device=device)
+    for e in range(E):
+        if e in hot:
+            layer.register(e, *keep[e])
+        else:
+            layer.register(e, *host[e], None, None, M.MOE_LOC_HOST_PINNED)
+    for T in (1, 4):
+        out[f"hotcold_B{T}"] = stream_of(layer, T)
+    x = synth.tokens(4096, H, seed=SEED, device=device, first_token=610000)
+    time_forwards(layer, [x], wr, bias, flush, stream, 1)
+    reps = 3
+    ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
+    st = layer.stats()
+    cold, touched = st["last_cold"], st["last_touched"]
+    bound_s = max((touched - cold) * EXPERT_BYTES / (hbm * 1e9), cold * EXPERT_BYTES / (h2d_gbs * 1e9))
+    out["hotcold_prefill4096"] = {"us_per_layer": 1000 * ms, "tokens_per_s": 4096 / (ms / 1000),
+                                  "touched_experts": touched, "cold_experts_staged": cold,
+                                  "cold_bytes": cold * EXPERT_BYTES,
+                                  "roofline_frac": bound_s / (ms / 1000) if ms > 0 else None}
     if layer.status():
         out["hotcold_device_status"] = layer.status()
+    layer.close()
+
+    # ---- every expert through a 128-slot cache
+    layer = M.MoeLayer(H, E, K, I, n_spare_slots=n_cache_all, device=device)
+    for e in range(E):
+        layer.register(e, *host[e], None, None, M.MOE_LOC_HOST_PINNED)
+    out["lru_all_B4"] = stream_of(layer, 4, n_fill=8)
+    out["lru_all_B4"]["cache_slots"] = n_cache_all
+    if layer.status():
+        out["lru_all_device_status"] = layer.status()
     layer.close()
     del host
     return out

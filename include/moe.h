@@ -209,13 +209,31 @@ moe_status_t moe_slots_query(const moe_slots_t* slots, int expert, int* location
 
 typedef struct {
   int64_t calls;          /* moe_expert_ffn calls that used this table */
-  int64_t cold_staged;    /* cold experts copied host -> HBM, cumulative */
+  int64_t cold_staged;    /* cold experts copied host -> HBM (cache misses), cumulative */
   int64_t bytes_staged;   /* bytes copied host -> HBM, cumulative */
-  int32_t last_cold;      /* cold experts staged by the most recent call */
+  int32_t last_cold;      /* cold experts staged (copied) by the most recent call */
   int32_t last_touched;   /* experts with at least one pair in the most recent call */
+  int64_t cache_hits;     /* routed host-resident experts found in a spare slot, cumulative */
+  int32_t last_hits;      /* ... in the most recent call */
+  int32_t last_routed_cold; /* routed host-resident experts in the most recent call */
 } moe_slots_stats_t;
 
 moe_status_t moe_slots_stats(const moe_slots_t* slots, moe_slots_stats_t* stats);
+
+/* What the spare slots hold between calls (the pages' hybrid keeps a subset of
+ * the experts on the cards and serves the rest from host memory; the recipes
+ * wiki's cache variant keeps recently used experts resident).
+ *   MOE_SLOTS_LRU (default): the spare slots are an LRU cache of host-resident
+ *     experts. A routed host expert already in a slot is a hit (no copy); a
+ *     miss takes the least recently used slot that the call does not need.
+ *     Registering every expert as MOE_LOC_HOST_PINNED sends every expert
+ *     through the cache. A call that routes more host experts than there are
+ *     spare slots falls back to per-call staging and empties the cache.
+ *   MOE_SLOTS_PER_CALL: every call copies its routed host experts again.
+ * Results are bit-identical under either policy (the same kernels read the
+ * same bytes). Synchronous with respect to the host; call between forwards. */
+enum { MOE_SLOTS_LRU = 0, MOE_SLOTS_PER_CALL = 1 };
+moe_status_t moe_slots_set_policy(moe_slots_t* slots, int policy);
 
 /* Greedy hot set (the "hotsplit" recipes wiki, Home page: the planner picks
  * the experts with the largest routing share per byte from routing

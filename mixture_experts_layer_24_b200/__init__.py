@@ -17,6 +17,8 @@ from .binding import (  # noqa: F401
     MOE_FP8_E4M3_B128,
     MOE_LOC_HBM,
     MOE_LOC_HOST_PINNED,
+    MOE_SLOTS_LRU,
+    MOE_SLOTS_PER_CALL,
     MoeError,
     MoeLayer,
     lib,
@@ -38,6 +40,7 @@ from .binding import (  # noqa: F401
     moe_slots_destroy,
     moe_slots_query,
     moe_slots_register,
+    moe_slots_set_policy,
     moe_slots_stats,
     moe_workspace_size,
 )

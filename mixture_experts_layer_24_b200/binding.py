@@ -20,6 +20,8 @@ MOE_BF16 = 0
 MOE_FP8_E4M3_B128 = 1
 MOE_LOC_HBM = 0
 MOE_LOC_HOST_PINNED = 1
+MOE_SLOTS_LRU = 0
+MOE_SLOTS_PER_CALL = 1
 MOE_DEV_BAD_EXPERT = 1
 MOE_DEV_NO_SLOT = 2
 MOE_DEV_TIMEOUT = 4
@@ -31,7 +33,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_e4m3", "moe_slots_create",
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_read", "moe_route_noalloc"]
+           "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
@@ -49,7 +51,8 @@ class MoeConfig(ctypes.Structure):
 
 class MoeSlotsStats(ctypes.Structure):
     _fields_ = [("calls", ctypes.c_int64), ("cold_staged", ctypes.c_int64), ("bytes_staged", ctypes.c_int64),
-                ("last_cold", ctypes.c_int32), ("last_touched", ctypes.c_int32)]
+                ("last_cold", ctypes.c_int32), ("last_touched", ctypes.c_int32), ("cache_hits", ctypes.c_int64),
+                ("last_hits", ctypes.c_int32), ("last_routed_cold", ctypes.c_int32)]
 
 
 _lib = None
@@ -79,6 +82,7 @@ def lib():
         "moe_slots_register": ([P, I, P, P, P, P, I], S),
         "moe_slots_query": ([P, I, ctypes.POINTER(I), ctypes.POINTER(I)], S),
         "moe_slots_stats": ([P, ctypes.POINTER(MoeSlotsStats)], S),
+        "moe_slots_set_policy": ([P, I], S),
         "moe_plan_hot_set": ([P, I, I, P], S),
         "moe_get_device_status": ([P, ctypes.POINTER(ctypes.c_int32), I], S),
         "moe_last_error": ([], ctypes.c_char_p),
@@ -202,6 +206,10 @@ def moe_slots_stats(slots) -> dict:
     st = MoeSlotsStats()
     _check(lib().moe_slots_stats(slots, ctypes.byref(st)), "moe_slots_stats")
     return {k: getattr(st, k) for k, _ in MoeSlotsStats._fields_}
+
+
+def moe_slots_set_policy(slots, policy: int) -> None:
+    _check(lib().moe_slots_set_policy(slots, int(policy)), "moe_slots_set_policy")
 
 
 def moe_plan_hot_set(hist, n_hot: int):

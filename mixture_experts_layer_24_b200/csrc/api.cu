@@ -132,6 +132,14 @@ struct moe_slots {
   size_t h_pinned_ints = 0;
   int n_host = 0;
   moe_slots_stats_t stats{};
+  // spare slots as an LRU cache of host-resident experts (MOE_SLOTS_LRU)
+  int policy = MOE_SLOTS_LRU;
+  std::vector<int> slot_expert;     // [n_spare] expert held, -1 empty
+  std::vector<int> expert_slot;     // [E] its spare slot, -1 not cached
+  std::vector<int64_t> slot_tick;   // [n_spare] call that last used the slot
+  int64_t tick = 0;
+  cudaEvent_t ev_done = nullptr;    // after the most recent call's GEMMs (they may read the slots)
+  bool ev_done_valid = false;
   std::mutex mu;
 };
 
@@ -702,7 +710,98 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   }
   sl->stats.last_touched = touched;
   sl->stats.last_cold = (int32_t)cold.size();
+  sl->stats.last_hits = 0;
+  sl->stats.last_routed_cold = (int32_t)cold.size();
   if (!cold.empty() && sl->n_spare <= 0) return fail(MOE_ERR_SLOT, "cold experts routed but no spare slots");
+
+  if (sl->policy == MOE_SLOTS_LRU && (int)cold.size() <= sl->n_spare) {
+    // ---- LRU: hits keep their slot; each miss takes the least recently used slot this call does not need
+    const int64_t tick = ++sl->tick;
+    std::vector<int> miss;
+    int hits = 0;
+    for (int e : cold) {
+      const int sidx = sl->expert_slot[e];
+      if (sidx >= 0) {
+        sl->slot_tick[sidx] = tick;
+        ++hits;
+      } else {
+        miss.push_back(e);
+      }
+    }
+    bool waited = false;
+    for (int e : miss) {
+      int victim = -1;
+      for (int i = 0; i < sl->n_spare; ++i) {
+        if (sl->slot_tick[i] == tick) continue;  // holds an expert of this call
+        if (victim < 0 || sl->slot_tick[i] < sl->slot_tick[victim]) victim = i;
+      }
+      if (victim < 0) return fail(MOE_ERR_SLOT, "no free spare slot");  // cannot happen: cold.size() <= n_spare
+      if (sl->slot_expert[victim] >= 0) sl->expert_slot[sl->slot_expert[victim]] = -1;
+      sl->slot_expert[victim] = e;
+      sl->expert_slot[e] = victim;
+      sl->slot_tick[victim] = tick;
+      if (!waited && sl->ev_done_valid) {
+        // the previous call's GEMMs may still read the slot being overwritten
+        MOE_CUDA(cudaStreamWaitEvent(sl->copy_stream, sl->ev_done, 0));
+        waited = true;
+      }
+      uint8_t* slot = sl->spare + (size_t)victim * sl->slot_bytes;
+      MOE_CUDA(cudaMemcpyAsync(slot, sl->gu[e], sl->bytes_gu, cudaMemcpyHostToDevice, sl->copy_stream));
+      MOE_CUDA(cudaMemcpyAsync(slot + sl->off_dn, sl->dn[e], sl->bytes_dn, cudaMemcpyHostToDevice, sl->copy_stream));
+      if (fp8) {
+        MOE_CUDA(cudaMemcpyAsync(slot + sl->off_sgu, sl->sgu[e], sl->bytes_sgu, cudaMemcpyHostToDevice,
+                                 sl->copy_stream));
+        MOE_CUDA(cudaMemcpyAsync(slot + sl->off_sdn, sl->sdn[e], sl->bytes_sdn, cudaMemcpyHostToDevice,
+                                 sl->copy_stream));
+      }
+      sl->stats.cold_staged++;
+      sl->stats.bytes_staged += (int64_t)(sl->bytes_gu + sl->bytes_dn + (fp8 ? sl->bytes_sgu + sl->bytes_sdn : 0));
+    }
+    sl->stats.last_cold = (int32_t)miss.size();
+    sl->stats.last_hits = hits;
+    sl->stats.cache_hits += hits;
+    // one list over every touched expert, ascending: resident ones by their own map, cached ones by their slot's
+    std::vector<int32_t> he, hm, hp;
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      const int cnt = hoff[e + 1] - hoff[e];
+      if (cnt <= 0) continue;
+      int m;
+      if (sl->loc[e] == MOE_LOC_HBM) m = e;
+      else if (sl->loc[e] == MOE_LOC_HOST_PINNED) m = E + sl->expert_slot[e];
+      else continue;
+      he.push_back(e);
+      hm.push_back(m);
+      hp.push_back(acc);
+      acc += (cnt + bn - 1) / bn;
+    }
+    hp.push_back(acc);
+    int32_t* stage = sl->h_pinned + (E + 1);
+    const size_t n_e = he.size(), n_p = hp.size();
+    std::memcpy(stage, he.data(), n_e * 4);
+    std::memcpy(stage + n_e, hm.data(), n_e * 4);
+    std::memcpy(stage + 2 * n_e, hp.data(), n_p * 4);
+    MOE_CUDA(cudaMemcpyAsync(le, stage, n_e * 4, cudaMemcpyHostToDevice, s));
+    MOE_CUDA(cudaMemcpyAsync(lm, stage + n_e, n_e * 4, cudaMemcpyHostToDevice, s));
+    MOE_CUDA(cudaMemcpyAsync(np, stage + 2 * n_e, n_p * 4, cudaMemcpyHostToDevice, s));
+    if (!miss.empty()) {
+      MOE_CUDA(cudaEventRecord(sl->ev_ready[0], sl->copy_stream));
+      MOE_CUDA(cudaStreamWaitEvent(s, sl->ev_ready[0], 0));
+    }
+    if (n_e > 0) {
+      st = run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, (int)n_e,
+                     ntile_bound, s, false, false);
+      if (st != MOE_OK) return st;
+    }
+    MOE_CUDA(cudaEventRecord(sl->ev_done, s));
+    sl->ev_done_valid = true;
+    return MOE_OK;
+  }
+  // per-call staging (or more routed host experts than slots): every slot is overwritten, the cache empties
+  std::fill(sl->slot_expert.begin(), sl->slot_expert.end(), -1);
+  std::fill(sl->expert_slot.begin(), sl->expert_slot.end(), -1);
+  std::fill(sl->slot_tick.begin(), sl->slot_tick.end(), -1);
+  if (sl->ev_done_valid) MOE_CUDA(cudaStreamWaitEvent(sl->copy_stream, sl->ev_done, 0));
   const bool two_buf = (int)cold.size() > sl->n_spare && sl->n_spare >= 2;
   const int bsz = two_buf ? sl->n_spare / 2 : sl->n_spare;
 
@@ -774,7 +873,8 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     if (st != MOE_OK) return st;
     MOE_CUDA(cudaEventRecord(sl->ev_free[buf], s));
   }
-  return MOE_OK;
+  MOE_CUDA(cudaEventRecord(sl->ev_done, s));
+  sl->ev_done_valid = true;
   return MOE_OK;
 }
 
@@ -938,6 +1038,11 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
         cudaEventCreateWithFlags(&sl->ev_free[i], cudaEventDisableTiming) != cudaSuccess)
       return cleanup(MOE_ERR_CUDA, "cudaEventCreate failed");
   }
+  if (cudaEventCreateWithFlags(&sl->ev_done, cudaEventDisableTiming) != cudaSuccess)
+    return cleanup(MOE_ERR_CUDA, "cudaEventCreate failed");
+  sl->slot_expert.assign(n_spare, -1);
+  sl->expert_slot.assign(sl->E, -1);
+  sl->slot_tick.assign(n_spare, -1);
   for (int i = 0; i < n_spare; ++i) {
     uint8_t* slot = sl->spare + (size_t)i * sl->slot_bytes;
     moe_status_t st = make_entry(ctx, &sl->h_maps[sl->E + i], slot, slot + sl->off_dn,
@@ -963,6 +1068,7 @@ moe_status_t moe_slots_destroy(moe_slots_t* sl) {
     if (sl->ev_ready[i]) cudaEventDestroy(sl->ev_ready[i]);
     if (sl->ev_free[i]) cudaEventDestroy(sl->ev_free[i]);
   }
+  if (sl->ev_done) cudaEventDestroy(sl->ev_done);
   if (sl->copy_stream) cudaStreamDestroy(sl->copy_stream);
   if (sl->h_pinned) cudaFreeHost(sl->h_pinned);
   if (sl->spare) cudaFree(sl->spare);
@@ -994,6 +1100,11 @@ moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, c
   } else {
     sl->h_map_of[expert] = -1;
   }
+  if (sl->expert_slot[expert] >= 0) {  // its cached copy no longer matches
+    sl->slot_expert[sl->expert_slot[expert]] = -1;
+    sl->slot_tick[sl->expert_slot[expert]] = -1;
+    sl->expert_slot[expert] = -1;
+  }
   const int prev = sl->loc[expert];
   if (prev == MOE_LOC_HOST_PINNED) sl->n_host--;
   if (location == MOE_LOC_HOST_PINNED) sl->n_host++;
@@ -1011,6 +1122,17 @@ moe_status_t moe_slots_query(const moe_slots_t* sl, int expert, int* location, i
   if (expert < 0 || expert >= sl->E) return fail(MOE_ERR_SLOT, "expert index out of range");
   *location = sl->loc[expert];
   *slot = sl->loc[expert] == MOE_LOC_HBM ? sl->h_map_of[expert] : -1;
+  return MOE_OK;
+}
+
+moe_status_t moe_slots_set_policy(moe_slots_t* sl, int policy) {
+  if (!sl) return fail(MOE_ERR_INVALID_ARG, "NULL slot table");
+  if (policy != MOE_SLOTS_LRU && policy != MOE_SLOTS_PER_CALL) return fail(MOE_ERR_INVALID_ARG, "bad policy");
+  std::lock_guard<std::mutex> lock(sl->mu);
+  sl->policy = policy;
+  std::fill(sl->slot_expert.begin(), sl->slot_expert.end(), -1);
+  std::fill(sl->expert_slot.begin(), sl->expert_slot.end(), -1);
+  std::fill(sl->slot_tick.begin(), sl->slot_tick.end(), -1);
   return MOE_OK;
 }
 
