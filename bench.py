@@ -494,8 +494,8 @@ def run_profile_case(kind):
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64)}[kind]
-    fp8 = kind == "f64"
+    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64), "f2048": (48, 2048)}[kind]
+    fp8 = kind in ("f64", "f2048")
     layer = M.MoeLayer(H, E_s, K, I, wdtype=M.MOE_FP8_E4M3_B128 if fp8 else M.MOE_BF16, device=device)
     keep = []
     for e in range(E_s):
@@ -509,7 +509,7 @@ def run_profile_case(kind):
             layer.register(e, g, d)
             keep.append((g, d))
     wr = synth.router_weight(E_s, H, seed=SEED, device=device)
-    bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind == "p2048" else None
+    bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind in ("p2048", "f2048") else None
     x = synth.tokens(T_s, H, seed=SEED, device=device)
     for _ in range(3):
         layer.forward(x, wr, bias)
@@ -669,7 +669,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:
