@@ -640,11 +640,19 @@ bool decode_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, 
 // (bf16) the sorted rows; `pdl`: the previous launch is this forward's own.
 moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
                       const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T, float* y_pair,
-                      void* ws, cudaStream_t s, bool pdl, bool planned) {
+                      void* ws, cudaStream_t s, bool pdl, bool planned, const int32_t* inv = nullptr) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const WsLayout W = ws_layout(c, T);
   const int E = c.n_experts, P = T * c.top_k;
+  // FP8 activation rows in sorted-pair order: with inv each token is quantised once and stored to its K rows
+  auto quant_x = [&](bool chain_pdl) -> cudaError_t {
+    if (inv)
+      return launch_quant_scatter_rows(x, inv, T, c.top_k, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                       at<float>(ws, W.x_scale), s, chain_pdl);
+    return launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                    at<float>(ws, W.x_scale), s, chain_pdl);
+  };
   const int bn = ffn_block_n(T, c.wdtype);
   moe_status_t st = MOE_OK;
   std::lock_guard<std::mutex> lock(sl->mu);
@@ -667,16 +675,14 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
       }
       Prof pg(ctx, MOE_PROF_GATHER, s);
       if (fp8) {
-        MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
-                                          at<float>(ws, W.x_scale), s, ctx->chain));
+        MOE_CUDA(quant_x(ctx->chain));
       } else {
         MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s, ctx->chain));
       }
       plan_ready_gu = true;  // plan -> gather -> gate/up
     } else if (fp8) {
       Prof pg(ctx, MOE_PROF_GATHER, s);
-      MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
-                                        at<float>(ws, W.x_scale), s, pdl));
+      MOE_CUDA(quant_x(pdl));
       plan_ready_gu = pdl;  // permutation+plan -> quantiser -> gate/up
     }
     return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
@@ -687,8 +693,7 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   {
     Prof pg(ctx, MOE_PROF_GATHER, s);
     if (fp8) {
-      MOE_CUDA(launch_gather_quant_rows(x, perm_src, offsets, E, P, c.hidden, at<uint8_t>(ws, W.x_perm),
-                                        at<float>(ws, W.x_scale), s, false));
+      MOE_CUDA(quant_x(false));
     } else {
       MOE_CUDA(launch_gather_rows(x, perm_src, offsets, E, P, c.hidden, at<void>(ws, W.x_perm), s, false));
     }
@@ -975,7 +980,7 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
                          ffn_block_n(T, c.wdtype), x, (resident && !fp8) ? at<void>(ws, W.x_perm) : nullptr,
                          &planned)) != MOE_OK)
     return st;
-  if ((st = ffn_impl(ctx, sl, x, ps, pk, offsets, w, T, y, ws, s, chain, planned)) != MOE_OK) return st;
+  if ((st = ffn_impl(ctx, sl, x, ps, pk, offsets, w, T, y, ws, s, chain, planned, inv)) != MOE_OK) return st;
   Prof p(ctx, MOE_PROF_COMBINE, s);
   MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, resident && chain));
   return MOE_OK;

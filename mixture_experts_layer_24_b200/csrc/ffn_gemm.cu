@@ -73,6 +73,9 @@ struct Fp8Cfg {
   static constexpr int NP = kNpRaw > 8 ? 8 : kNpRaw;
   static constexpr uint32_t kTmemCols = tmem_cols_for(NP * NA * BN);
   static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kScaleBytes + 8 * (2 * kStages + 2 * NP) + 64;
+  // epilogue warps (4 TMEM lane quarters x EW/4 column groups); 16 at BN = 64
+  // measured no faster than 8
+  static constexpr int EW = 8;
   static_assert(kStages >= 2 && NP >= 2, "FP8 pipeline needs two stages and two partial buffers");
 };
 
@@ -398,11 +401,15 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
 // barriers.
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
+__global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
+    ffn_fp8_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
   using C = Fp8Cfg<MODE, BN>;
   constexpr int NA = C::NA, S = C::kStages, NP = C::NP;
   constexpr uint32_t STAGE = C::kStageBytes;
-  constexpr int HALF = BN / 2;  // columns per epilogue warp
+  constexpr int EW = C::EW;            // epilogue warps: 4 TMEM lane quarters x EW/4 column groups
+  constexpr int EPT = 32 * EW;         // epilogue threads
+  constexpr int PW = EW, MW = EW + 1;  // producer warp, MMA warp
+  constexpr int HALF = BN * 4 / EW;    // columns per epilogue warp
   constexpr int NCH = HALF >= 16 ? HALF / 16 : 1;
   constexpr int CW = HALF >= 16 ? 16 : HALF;  // columns used per TMEM load
 
@@ -444,12 +451,12 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
     }
     for (int b = 0; b < NP; ++b) {
       mbar_init(pfull(b), 1);
-      mbar_init(pempty(b), 8);
+      mbar_init(pempty(b), EW);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == MW) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -458,7 +465,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
-  if (warp == 8) {
+  if (warp == PW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
@@ -512,7 +519,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
       pdl_wait();
       pdl_trigger();
     }
-  } else if (warp == 9) {
+  } else if (warp == MW) {
     // ------------------------------------------------------------ MMA issuer
     if (a.plan_ready) {
       pdl_wait();
@@ -551,7 +558,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 0..7)
+    // ------------------------------------------------------------ epilogue (warps 0..EW-1)
     // warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
     if (a.plan_ready) {
       pdl_wait();
@@ -559,7 +566,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
     }
     const int q4 = warp & 3, hf = warp >> 2;
     const int r = q4 * 32 + lane;
-    const int et = threadIdx.x;  // 0..255
+    const int et = threadIdx.x;  // 0..EPT-1
     const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int c0 = hf * HALF;
     bool aborted = false;  // warp-uniform
@@ -570,18 +577,18 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
       const int width = 16 << tile_width_index(ti.nvalid, BN);
       const MapEntry* me = a.maps + ti.mapi;
       const float* sw = MODE == kGateUp ? me->s_gu : me->s_dn;
-      named_bar_sync(1, 256);  // the previous tile's readers are done with the scale tables
-      for (int i = et; i < BN * KB; i += 256) {
+      named_bar_sync(1, EPT);  // the previous tile's readers are done with the scale tables
+      for (int i = et; i < BN * KB; i += EPT) {
         const int n = i / KB, kb = i - n * KB;
         s_act[n * KB + kb] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
       }
-      for (int i = et; i < NA * KB; i += 256) {
+      for (int i = et; i < NA * KB; i += EPT) {
         const int which = i / KB, kb = i - which * KB;
         const int rb = which == 0 ? ti.mt : a.I / 128 + ti.mt;  // gate (or down) row block, then up
         s_w[which * KB + kb] = sw[(size_t)rb * KB + kb];
       }
       if (MODE == kDown) {
-        for (int n = et; n < BN; n += 256) {
+        for (int n = et; n < BN; n += EPT) {
           float wv = 0.0f;
           if (n < ti.nvalid) {
             const int p = ti.row0 + n;
@@ -590,7 +597,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
           wcol[n] = wv;
         }
       }
-      named_bar_sync(1, 256);
+      named_bar_sync(1, EPT);
 
       float accg[HALF], accu[MODE == kGateUp ? HALF : 1];
 #pragma unroll
@@ -669,7 +676,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_kernel(const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == MW) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -2039,7 +2046,8 @@ static cudaError_t launch_bf16(const ActMaps& maps, GemmArgs a, int grid, cudaSt
 template <int MODE, int BN>
 static cudaError_t launch_fp8(const ActMaps& maps, const GemmArgs& a, int grid, cudaStream_t s, bool pdl) {
   const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
-  return launch_kernel(ffn_fp8_kernel<MODE, BN>, Fp8Cfg<MODE, BN>::kSmem, 320, persistent, maps, a, s, pdl);
+  return launch_kernel(ffn_fp8_kernel<MODE, BN>, Fp8Cfg<MODE, BN>::kSmem, 32 * (Fp8Cfg<MODE, BN>::EW + 2), persistent,
+                       maps, a, s, pdl);
 }
 
 template <int MODE>

@@ -176,6 +176,10 @@ cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
                                int H, void* x_perm, cudaStream_t s, bool pdl);
+// FP8 activation rows of the forward: each token's row quantised once (per 128
+// columns) and stored to its K sorted pair rows through inv.
+cudaError_t launch_quant_scatter_rows(const void* x, const int32_t* inv, int T, int K, int H, uint8_t* xq, float* xs,
+                                      cudaStream_t s, bool pdl);
 cudaError_t launch_gather_quant_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E,
                                      int P, int H, uint8_t* xq, float* xs, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int H, void* out, cudaStream_t s,

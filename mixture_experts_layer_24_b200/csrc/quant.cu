@@ -86,6 +86,46 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const uint16_t* __restr
   if (lane == 0) scales[(size_t)row * groups + g] = s;
 }
 
+// One warp per (token, 128-column group), lane l owns columns 4l..4l+3: the
+// same codes and scale as quant_rows_kernel on each gathered row, computed
+// once per token and stored to the token's K pair rows (inv[t*K+k] = its
+// sorted row; -1: a dropped pair, skipped).
+__global__ void __launch_bounds__(256) quant_scatter_rows_kernel(const uint16_t* __restrict__ src,
+                                                                  const int32_t* __restrict__ inv, int T, int K,
+                                                                  int cols, uint8_t* __restrict__ q,
+                                                                  float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int groups = cols / 128;
+  const int t = (int)(wid / groups), g = (int)(wid - (int64_t)t * groups);
+  if (t >= T) return;
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(src + (size_t)t * cols + g * 128 + lane * 4));
+  const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xffff0000u);
+  const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xffff0000u);
+  float amax = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float sc = (amax == 0.0f) ? 1.0f : amax / 448.0f;
+  const uint32_t packed = (uint32_t)to_e4m3(f0 / sc) | ((uint32_t)to_e4m3(f1 / sc) << 8) |
+                          ((uint32_t)to_e4m3(f2 / sc) << 16) | ((uint32_t)to_e4m3(f3 / sc) << 24);
+  for (int k = 0; k < K; ++k) {
+    const int p = __ldg(inv + (size_t)t * K + k);
+    if (p < 0) continue;
+    *reinterpret_cast<uint32_t*>(q + (size_t)p * cols + g * 128 + lane * 4) = packed;
+    if (lane == 0) scales[(size_t)p * groups + g] = sc;
+  }
+}
+
+cudaError_t launch_quant_scatter_rows(const void* x, const int32_t* inv, int T, int K, int H, uint8_t* xq, float* xs,
+                                      cudaStream_t s, bool pdl) {
+  if (T <= 0) return cudaSuccess;
+  const int64_t warps = (int64_t)T * (H / 128);
+  return launch_ex(quant_scatter_rows_kernel, dim3((unsigned)((warps + 7) / 8)), dim3(256), 0, s, pdl,
+                   static_cast<const uint16_t*>(x), inv, T, K, H, xq, xs);
+}
+
 cudaError_t launch_quant_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                               cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
