@@ -490,7 +490,9 @@ def run_profile_case(kind):
     """Small cases for ncu captures of the FFN kernels, three forwards each:
     "t64": the layer shape with 32 experts (1.6 GB of bf16 weights, all
     touched) and 64 tokens; "t1": 8 experts (top-8 of 8, all touched, 400 MB)
-    and one token -- the per-launch shape of batch-1 decode."""
+    and one token -- the per-launch shape of batch-1 decode; "p2048": 48
+    experts and a 2048-token prefill chunk under the Zipf logit prior;
+    "f64" / "f2048": "t64" / "p2048" with e4m3 experts."""
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
@@ -515,7 +517,7 @@ def run_profile_case(kind):
         layer.forward(x, wr, bias)
     torch.cuda.synchronize()
     st = layer.status()
-    print(json.dumps({"profile_case": f"E={E_s} H=4096 I=2048 K=8 T={T_s} bf16", "status": st}))
+    print(json.dumps({"profile_case": f"E={E_s} H={H} I={I} K={K} T={T_s} {'e4m3' if fp8 else 'bf16'}", "status": st}))
     layer.close()
     return 1 if st else 0
 

@@ -44,7 +44,7 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
 template <int MODE, int BN>
 struct Bf16Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr int KC = ffn_k_chunks(MODE, BN);
+  static constexpr int KC = kBf16KChunks;
   static constexpr uint32_t kChunkA = kABytes;     // 128 rows x 128 B
   static constexpr uint32_t kChunkB = BN * 128;    // BN rows x 128 B
   static constexpr uint32_t kStageBytes = KC * (NA * kChunkA + kChunkB);
@@ -118,7 +118,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Per-tile MMA width: the smallest of 16, 32, 64, 128, 256 (<= BN) that holds
+// Per-tile MMA width: the smallest of 16, 32, 64, 128 (<= BN) that holds
 // the tile's pairs; its index selects the activation map of that box height.
 __device__ __forceinline__ int tile_width_index(int nvalid, int bn) {
   int w = 16, i = 0;
@@ -2059,7 +2059,6 @@ static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const
       case 32: return launch_bf16<MODE, 32>(*maps, a, grid, s, pdl);
       case 64: return launch_bf16<MODE, 64>(*maps, a, grid, s, pdl);
       case 128: return launch_bf16<MODE, 128>(*maps, a, grid, s, pdl);
-      case 256: return launch_bf16<MODE, 256>(*maps, a, grid, s, pdl);
     }
   } else {
     switch (bn) {
@@ -2087,7 +2086,6 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
         case 32: return Bf16Cfg<kGateUp, 32>::smem(Bf16Cfg<kGateUp, 32>::kStagesMax);
         case 64: return Bf16Cfg<kGateUp, 64>::smem(Bf16Cfg<kGateUp, 64>::kStagesMax);
         case 128: return Bf16Cfg<kGateUp, 128>::smem(Bf16Cfg<kGateUp, 128>::kStagesMax);
-        case 256: return Bf16Cfg<kGateUp, 256>::smem(Bf16Cfg<kGateUp, 256>::kStagesMax);
       }
     } else {
       switch (bn) {
@@ -2095,7 +2093,6 @@ size_t ffn_gemm_smem_bytes(int mode, int wdtype, int bn) {
         case 32: return Bf16Cfg<kDown, 32>::smem(Bf16Cfg<kDown, 32>::kStagesMax);
         case 64: return Bf16Cfg<kDown, 64>::smem(Bf16Cfg<kDown, 64>::kStagesMax);
         case 128: return Bf16Cfg<kDown, 128>::smem(Bf16Cfg<kDown, 128>::kStagesMax);
-        case 256: return Bf16Cfg<kDown, 256>::smem(Bf16Cfg<kDown, 256>::kStagesMax);
       }
     }
   } else {

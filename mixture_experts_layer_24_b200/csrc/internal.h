@@ -30,11 +30,10 @@ struct alignas(64) MapEntry {
 enum FfnMode { kGateUp = 0, kDown = 1 };
 
 // 64-wide K chunks per pipeline stage (one 3-D TMA copy per operand) of the
-// bf16 GEMM: two, except the 256-wide gate/up tile, whose two-chunk stage
-// would not fit twice in shared memory. Fewer, larger copies stream faster
-// than more, smaller stages: the TMA unit's per-copy cost bounds one SM's
-// rate (measured at BN = 128: one chunk per stage is 5-25% slower).
-constexpr int ffn_k_chunks(int mode, int bn) { return (mode == 0 && bn == 256) ? 1 : 2; }
+// bf16 GEMM. Fewer, larger copies stream faster than more, smaller stages:
+// the TMA unit's per-copy cost bounds one SM's rate (measured at BN = 128:
+// one chunk per stage is 5-25% slower than two).
+constexpr int kBf16KChunks = 2;
 
 // Launches `kern` on `s`, with programmatic stream serialisation when pdl is
 // true (the kernel must then follow the pdl_wait / pdl_trigger rule).
@@ -85,10 +84,10 @@ struct GemmArgs {
   int num_sms;
 };
 
-// Activation-operand TMA descriptors for box heights 16, 32, 64, 128, 256
-// rows (the bf16 GEMMs pick, per tile, the smallest that holds its pairs).
+// Activation-operand TMA descriptors for box heights 16, 32, 64, 128 rows
+// (the GEMMs pick, per tile, the smallest that holds its pairs).
 struct alignas(64) ActMaps {
-  CUtensorMap m[5];
+  CUtensorMap m[4];
 };
 
 // Launches one FFN GEMM (gate/up+SwiGLU or down*weight) over the tile list.
