@@ -492,10 +492,23 @@ def run_profile_case(kind):
     touched) and 64 tokens; "t1": 8 experts (top-8 of 8, all touched, 400 MB)
     and one token -- the per-launch shape of batch-1 decode; "p2048": 48
     experts and a 2048-token prefill chunk under the Zipf logit prior;
-    "f64" / "f2048": "t64" / "p2048" with e4m3 experts."""
+    "f64" / "f2048": "t64" / "p2048" with e4m3 experts; "r4096": the router
+    alone (384 experts, 4096 tokens, Zipf prior), three calls."""
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    if kind == "r4096":
+        layer = M.MoeLayer(H, E, K, I, device=device)
+        wr = synth.router_weight(E, H, seed=SEED, device=device)
+        bias = synth.zipf_logit_bias(E, ZIPF_S, seed=SEED).to(device)
+        x = synth.tokens(4096, H, seed=SEED, device=device)
+        for _ in range(3):
+            layer.route(x, wr, bias)
+        torch.cuda.synchronize()
+        st = layer.status()
+        print(json.dumps({"profile_case": f"router E={E} H={H} K={K} T=4096", "status": st}))
+        layer.close()
+        return 1 if st else 0
     E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64), "f2048": (48, 2048)}[kind]
     fp8 = kind in ("f64", "f2048")
     layer = M.MoeLayer(H, E_s, K, I, wdtype=M.MOE_FP8_E4M3_B128 if fp8 else M.MOE_BF16, device=device)
@@ -671,7 +684,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "r4096"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:

@@ -42,7 +42,8 @@ def M():
 
 @pytest.mark.parametrize("T,H,E,K,zipf", [(16, 256, 8, 2, None), (1, 4096, 384, 8, 1.1), (3, 4096, 384, 8, 1.1),
                                           (64, 4096, 384, 8, 1.1), (300, 1024, 64, 6, None),
-                                          (1000, 512, 100, 4, 1.1)])
+                                          (1000, 512, 100, 4, 1.1), (333, 1024, 40, 8, None),
+                                          (2049, 4096, 384, 8, 1.1)])
 def test_route_matches_oracle(T, H, E, K, zipf):
     dev = torch.device("cuda")
     x = synth.tokens(T, H, seed=1, device=dev)
@@ -84,6 +85,44 @@ def test_route_reduction_order_decides_topk():
         io = oracle.route(oracle.as_u16(x.to(torch.bfloat16)), wr.numpy(), None, 1)[1]
         assert idx.cpu().numpy()[0, 0] == io[0, 0], c["why"]
         layer.close()
+
+
+@pytest.mark.parametrize("T", [1, 5, 13, 40, 64, 65, 200, 333])
+def test_route_reduction_order_every_router_kernel(T):
+    """The golden order cases again, side by side in one batch, so that every
+    router kernel (one-launch small batches, the register-tiled decode tiles,
+    the token-pair prefill tile) meets them, with the cases of neighbouring
+    tokens different and ragged token and expert tiles. Case c lives in h block
+    [256c, 256c + 256) (a multiple of 32, so its lanes and in-lane order are
+    unchanged); expert 2c holds its weights, expert 2c+1 the midpoint between
+    the specified and the sequential sum, read through x[256c + 255] = 1."""
+    cases = json.load(open(os.path.join(GOLD, "order_cases.json")))["logit_cases"]
+    n = len(cases)
+    H, E = 256 * n, 2 * n + 4  # four all-zero experts make the expert tiles ragged
+    x = torch.zeros((T, H), dtype=torch.float32)
+    wr = torch.zeros((E, H), dtype=torch.float32)
+    for c, case in enumerate(cases):
+        base = 256 * c
+        seq = np.float32(0)
+        for h, xv, wv in case["terms"]:
+            assert h < 255
+            wr[2 * c, base + h] = wv
+            seq = np.float32(np.float64(seq) + np.float64(np.float32(xv)) * np.float64(np.float32(wv)))
+        exp = np.float32(case["expected"])
+        wr[2 * c + 1, base + 255] = (float(exp) + float(seq)) / 2 if float(seq) != float(exp) else float(exp) - 1e-3
+    for t in range(T):
+        c = (3 * t + 1) % n
+        for h, xv, wv in cases[c]["terms"]:
+            x[t, 256 * c + h] = xv
+        x[t, 256 * c + 255] = 1.0
+    xb = x.to(torch.bfloat16)
+    layer = M().MoeLayer(H, E, 1, 128)
+    idx, w = layer.route(xb.to(torch.device("cuda")), wr.to(torch.device("cuda")))
+    torch.cuda.synchronize()
+    io = oracle.route(oracle.as_u16(xb), wr.numpy(), None, 1)[1]
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert layer.status() == 0
+    layer.close()
 
 
 def test_route_ties_go_to_lower_index():
