@@ -214,6 +214,34 @@ def test_forward_small_bf16(T, H, E, K, I):
     case.close()
 
 
+@pytest.mark.parametrize("wdtype", [0, 1])
+@pytest.mark.parametrize("T,H,E,K,I,mode", [(33, 256, 4, 4, 256, "k_eq_e"),    # every token on every expert
+                                            (300, 256, 8, 2, 256, "one_pair"),  # all tokens on experts 5 and 2
+                                            (7, 512, 1, 1, 384, "single"),      # one expert, top-1
+                                            (129, 384, 6, 1, 256, "one_pair")])
+def test_forward_routing_edge_cases(T, H, E, K, I, mode, wdtype):
+    """Routing extremes through the whole forward: K = E; every token on the
+    same experts (the others get no rows; 300 rows is not a multiple of any
+    tile width); a single expert with top-1 (the layer is one dense SwiGLU FFN
+    scaled by weight 1)."""
+    case = LayerCase(T, H, E, K, I, seed=T + E, wdtype=wdtype)
+    if mode == "one_pair":  # a logit prior far above the logits' spread
+        bias = torch.zeros(E, dtype=torch.float32)
+        bias[5 % E] = 64.0
+        bias[2 % E] = 32.0
+        case.bias = bias.to(case.dev)
+    out = case.forward()
+    torch.cuda.synchronize()
+    assert case.layer.status() == 0
+    ref = case.oracle_forward()
+    if mode == "one_pair":
+        assert set(np.unique(ref["idx"]).tolist()) <= {5 % E, 2 % E}
+    assert_close_out(oracle.as_u16(out), ref["out"], TOL_FP8 if wdtype else TOL_BF16)
+    idx, _ = case.layer.route(case.x, case.wr, case.bias)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    case.close()
+
+
 def test_expert_ffn_y_pair_bf16():
     T, H, E, K, I = 48, 512, 8, 2, 256
     case = LayerCase(T, H, E, K, I, seed=5)
