@@ -1,10 +1,12 @@
 """The oracle's pins catch plausible mistakes (CPU only).
 
-Each case plants one mistake in a copy of the oracle's C source: a dropped
-term, a wrong sign, index or reduction order, a missed rounding point, a wrong
-constant. The case then runs the pin tests (``test_oracle_pins.py``) against
-the copy, which must fail. An unmodified copy must pass, so that a failure
-means the pins saw the mistake and not that the harness is broken.
+Each case plants one mistake in a copy of the oracle (its C source, or the
+Python layer that composes the steps): a dropped term, a wrong sign, index or
+reduction order, a missed rounding point, a wrong constant. The case then runs
+the pin tests (``test_oracle_pins.py``) against the copy, and at least one of
+them must fail (pytest's exit code 1: a test failed, not a crash or a
+collection error). An unmodified copy must pass, so that a failure means the
+pins saw the mistake and not that the harness is broken.
 """
 
 import os
@@ -21,7 +23,7 @@ TRUNC_H = ("{ float hv_ = silu_f32(g) * u; uint32_t hu_; memcpy(&hu_, &hv_, 4); 
            "hrow[j] = (uint16_t)(hu_ >> 16); }")
 TRUNC_OUT = ("{ uint32_t ou_; memcpy(&ou_, &acc, 4); out[(size_t)t * H + o] = (uint16_t)(ou_ >> 16); }")
 
-# (name, text in moe_oracle.c, replacement)
+# (name, text in moe_oracle.c, replacement); names starting "py_" edit __init__.py instead
 MUTATIONS = [
     # router logits: reduction order and arithmetic
     ("sequential_logit", "for (int o = LANES / 2; o >= 1; o /= 2)",
@@ -61,6 +63,9 @@ MUTATIONS = [
     ("quantiser_zero_block_scale", "float s = (amax == 0.0f) ? 1.0f : amax / 448.0f;", "float s = amax / 448.0f;"),
     ("fp8_activation_scale_dropped", "acc = fmaf(part, sa[kb] * sw[kb], acc);", "acc = fmaf(part, sw[kb], acc);"),
     ("fp8_weight_block_row", "sgu[e] + (size_t)(rg / 128) * (H / 128)", "sgu[e] + (size_t)(rg / 256) * (H / 128)"),
+    # composition of the steps
+    ("py_weights_of_the_wrong_slot", "pw = w64[sel].reshape(-1)", "pw = w64[sel][:, ::-1].reshape(-1)"),
+    ("py_pairs_of_the_wrong_token", "pt = np.repeat(sel, K)", "pt = np.tile(sel, K)"),
 ]
 
 
@@ -68,7 +73,7 @@ def _run_pins(tmp_path, name, old=None, new=None):
     d = tmp_path / name
     shutil.copytree(os.path.join(ROOT, "oracle"), d / "oracle",
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
-    src = d / "oracle" / "moe_oracle.c"
+    src = d / "oracle" / ("__init__.py" if name.startswith("py_") else "moe_oracle.c")
     if old is not None:
         s = src.read_text()
         assert s.count(old) >= 1, f"{name}: text not found in the oracle"
@@ -87,3 +92,4 @@ def test_unmodified_copy_passes_the_pins(tmp_path):
 def test_planted_mistake_fails_a_pin(tmp_path, name, old, new):
     r = _run_pins(tmp_path, name, old, new)
     assert r.returncode != 0, f"{name} survived every pin:\n{r.stdout[-2000:]}"
+    assert r.returncode == 1, f"{name}: the pins did not run to a failure:\n{r.stdout[-2000:]}{r.stderr[-2000:]}"
