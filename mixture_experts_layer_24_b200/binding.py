@@ -246,16 +246,46 @@ def moe_profile_read(ctx, reset: bool = True) -> dict:
 
 # ------------------------------------------------------------- convenience --
 
+def check_tensor(t, name, dtype, shape, device=None, pinned=False):
+    """Raises unless t is a contiguous tensor of this dtype and shape, on this
+    device (a CUDA torch.device with its index, or "cpu"), and in pinned
+    memory when asked. The C ABI takes raw pointers and cannot see any of it."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (row-major)")
+    if device is not None:
+        d = torch.device(device)
+        if t.device.type != d.type or (d.type == "cuda" and t.device.index != d.index):
+            raise ValueError(f"{name}: on {t.device}, expected {d}")
+    if pinned and not t.is_pinned():
+        raise ValueError(f"{name}: host-resident weights must be in pinned memory")
+
+
+def _rows(x, name):
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{name}: expected a 2-D [tokens, hidden] tensor")
+    return x.shape[0]
+
+
 class MoeLayer:
     """One MoE layer: a context, its slot table and a reusable workspace.
 
     Registered weight tensors are kept referenced here because the library
-    borrows them."""
+    borrows them. Every method checks its tensors' dtype, shape, layout and
+    device before the call (``check_tensor``)."""
 
     def __init__(self, hidden, n_experts, top_k, intermediate, wdtype=MOE_BF16, n_spare_slots=0, device=None,
                  flags=0):
         self.H, self.E, self.K, self.I, self.wdtype = hidden, n_experts, top_k, intermediate, wdtype
-        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        d = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        if d.type == "cuda" and d.index is None:
+            d = torch.device("cuda", torch.cuda.current_device())
+        self.device = d
         with torch.cuda.device(self.device):
             self.ctx = moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype, flags)
             self.slots = moe_slots_create(self.ctx, n_spare_slots)
@@ -263,6 +293,25 @@ class MoeLayer:
         self._ws = None
 
     def register(self, e, w_gu, w_dn, s_gu=None, s_dn=None, location=MOE_LOC_HBM):
+        if not 0 <= int(e) < self.E:
+            raise ValueError(f"expert {e} out of range [0, {self.E})")
+        if location == MOE_LOC_HBM:
+            dev, pinned = self.device, False
+        elif location == MOE_LOC_HOST_PINNED:
+            dev, pinned = "cpu", True
+        else:
+            raise ValueError(f"unknown location {location}")
+        H, I = self.H, self.I
+        if self.wdtype == MOE_FP8_E4M3_B128:
+            check_tensor(w_gu, "w_gu", torch.uint8, (2 * I, H), dev, pinned)
+            check_tensor(w_dn, "w_dn", torch.uint8, (H, I), dev, pinned)
+            check_tensor(s_gu, "s_gu", torch.float32, (2 * I // 128, H // 128), dev, pinned)
+            check_tensor(s_dn, "s_dn", torch.float32, (H // 128, I // 128), dev, pinned)
+        else:
+            check_tensor(w_gu, "w_gu", torch.bfloat16, (2 * I, H), dev, pinned)
+            check_tensor(w_dn, "w_dn", torch.bfloat16, (H, I), dev, pinned)
+            if s_gu is not None or s_dn is not None:
+                raise ValueError("bf16 experts take no block scales")
         self._keep[e] = (w_gu, w_dn, s_gu, s_dn)
         moe_slots_register(self.slots, e, w_gu, w_dn, s_gu, s_dn, location)
 
@@ -272,23 +321,38 @@ class MoeLayer:
             self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=self.device)
         return self._ws
 
+    def _check_route_inputs(self, x, w_router, logit_bias):
+        T = _rows(x, "x")
+        check_tensor(x, "x", torch.bfloat16, (T, self.H), self.device)
+        check_tensor(w_router, "w_router", torch.float32, (self.E, self.H), self.device)
+        if logit_bias is not None:
+            check_tensor(logit_bias, "logit_bias", torch.float32, (self.E,), self.device)
+        return T
+
     def forward(self, x, w_router, logit_bias=None, out=None, stream=None, ws=None):
-        T = x.shape[0]
+        T = self._check_route_inputs(x, w_router, logit_bias)
         if out is None:
             out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
+        else:
+            check_tensor(out, "out", torch.bfloat16, (T, self.H), self.device)
+        if ws is not None:
+            check_tensor(ws, "ws", torch.uint8, (ws.numel(),), self.device)
+            if ws.numel() < moe_workspace_size(self.ctx, T):
+                raise ValueError(f"ws: {ws.numel()} bytes, the call needs {moe_workspace_size(self.ctx, T)}")
         moe_forward(self.ctx, self.slots, x, w_router, logit_bias, T, out, self.workspace(T) if ws is None else ws,
                     stream)
         return out
 
     def route(self, x, w_router, logit_bias=None, stream=None):
-        T = x.shape[0]
+        T = self._check_route_inputs(x, w_router, logit_bias)
         idx = torch.empty((T, self.K), dtype=torch.int32, device=self.device)
         w = torch.empty((T, self.K), dtype=torch.float32, device=self.device)
         moe_route(self.ctx, x, w_router, logit_bias, T, idx, w, self.workspace(T), stream)
         return idx, w
 
     def permute(self, topk_idx, stream=None):
-        T = topk_idx.shape[0]
+        T = _rows(topk_idx, "topk_idx")
+        check_tensor(topk_idx, "topk_idx", torch.int32, (T, self.K), self.device)
         P = T * self.K
         d = self.device
         counts = torch.empty(self.E, dtype=torch.int32, device=d)
@@ -300,13 +364,21 @@ class MoeLayer:
         return counts, offsets, perm_src, perm_k, inv
 
     def expert_ffn(self, x, perm_src, perm_k, offsets, topk_w, stream=None):
-        T = x.shape[0]
+        T = _rows(x, "x")
+        P = T * self.K
+        check_tensor(x, "x", torch.bfloat16, (T, self.H), self.device)
+        check_tensor(perm_src, "perm_src", torch.int32, (P,), self.device)
+        check_tensor(perm_k, "perm_k", torch.int32, (P,), self.device)
+        check_tensor(offsets, "offsets", torch.int32, (self.E + 1,), self.device)
+        check_tensor(topk_w, "topk_w", torch.float32, (T, self.K), self.device)
         y = torch.empty((T * self.K, self.H), dtype=torch.float32, device=self.device)
         moe_expert_ffn(self.ctx, self.slots, x, perm_src, perm_k, offsets, topk_w, T, y, self.workspace(T), stream)
         return y
 
     def combine(self, y_pair, inv, stream=None):
-        T = inv.shape[0]
+        T = _rows(inv, "inv")
+        check_tensor(inv, "inv", torch.int32, (T, self.K), self.device)
+        check_tensor(y_pair, "y_pair", torch.float32, (T * self.K, self.H), self.device)
         out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)
         moe_combine(self.ctx, y_pair, inv, T, out, stream)
         return out

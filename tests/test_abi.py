@@ -99,3 +99,96 @@ def test_hot_set_planner():
     ref = np.lexsort((np.arange(384), -hist))[:120]  # count desc, ties -> lower index
     assert hot.tolist() == ref.tolist()
     assert M.moe_plan_hot_set(torch.zeros(10, dtype=torch.int64), 3).tolist() == [0, 1, 2]
+
+
+def test_tensor_checks_of_the_binding():
+    """MoeLayer's methods pass raw pointers to the C ABI, so the binding checks
+    dtype, shape, layout, device and pinning first (CPU-checkable part)."""
+    from mixture_experts_layer_24_b200.binding import check_tensor
+    t = torch.zeros((4, 8), dtype=torch.bfloat16)
+    check_tensor(t, "x", torch.bfloat16, (4, 8), "cpu")
+    with pytest.raises(TypeError):
+        check_tensor(t, "x", torch.float32, (4, 8))
+    with pytest.raises(ValueError):
+        check_tensor(t, "x", torch.bfloat16, (8, 4))
+    with pytest.raises(ValueError):
+        check_tensor(t.t(), "x", torch.bfloat16, (8, 4))  # a transposed view is not row-major
+    with pytest.raises(ValueError):
+        check_tensor(t, "x", torch.bfloat16, (4, 8), torch.device("cuda", 0))  # wrong device
+    with pytest.raises(ValueError):
+        check_tensor(t, "w_gu", torch.bfloat16, (4, 8), "cpu", pinned=True)  # pageable host memory
+    with pytest.raises(TypeError):
+        check_tensor(np.zeros((4, 8)), "x", torch.bfloat16, (4, 8))
+    check_tensor(t[:0], "x", torch.bfloat16, (0, 8), "cpu")  # an empty batch is fine
+
+
+def test_layer_methods_accept_valid_calls_and_reject_bad_ones(monkeypatch):
+    """The checked MoeLayer methods, driven on the CPU: the C calls are replaced
+    by no-ops and the layer's device is the host, so only the argument checks
+    and the output allocation run. Valid calls of every method pass; each kind
+    of bad argument is refused before any C call."""
+    from mixture_experts_layer_24_b200 import binding as B
+    calls = []
+    for name in ("moe_forward", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_slots_register"):
+        monkeypatch.setattr(B, name, lambda *a, _n=name, **k: calls.append(_n))
+    monkeypatch.setattr(B, "moe_workspace_size", lambda ctx, T: 4096)
+
+    def layer(wdtype):
+        L = object.__new__(B.MoeLayer)
+        L.H, L.E, L.K, L.I, L.wdtype = 256, 8, 2, 128, wdtype
+        L.device, L.ctx, L.slots, L._keep, L._ws = torch.device("cpu"), None, None, {}, None
+        return L
+
+    L = layer(B.MOE_BF16)
+    T, H, E, K, I = 5, 256, 8, 2, 128
+    x = torch.zeros((T, H), dtype=torch.bfloat16)
+    wr = torch.zeros((E, H), dtype=torch.float32)
+    bias = torch.zeros(E, dtype=torch.float32)
+    L.register(3, torch.zeros((2 * I, H), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16))
+    assert L.forward(x, wr, bias).shape == (T, H)
+    L.forward(x, wr, None, out=torch.empty((T, H), dtype=torch.bfloat16), ws=torch.empty(4096, dtype=torch.uint8))
+    L.forward(x[:0], wr, None, out=torch.empty((0, H), dtype=torch.bfloat16))
+    idx, w = L.route(x, wr, bias)
+    assert idx.shape == (T, K) and idx.dtype == torch.int32 and w.dtype == torch.float32
+    counts, offsets, ps, pk, inv = L.permute(idx)
+    assert offsets.shape == (E + 1,) and ps.shape == (T * K,) and inv.shape == (T, K)
+    y = L.expert_ffn(x, ps, pk, offsets, w)
+    assert y.shape == (T * K, H) and y.dtype == torch.float32
+    assert L.combine(y, inv).shape == (T, H)
+    n_ok = len(calls)
+
+    bad = [
+        lambda: L.forward(x.float(), wr, bias),                                     # x not bf16
+        lambda: L.forward(x[:, :128], wr, bias),                                    # wrong hidden size
+        lambda: L.forward(x, wr.t().contiguous().t(), bias),                        # w_router not row-major
+        lambda: L.forward(x, wr[:4], bias),                                         # wrong expert count
+        lambda: L.forward(x, wr, bias.double()),                                    # bias not fp32
+        lambda: L.forward(x, wr, bias, out=torch.empty((T, H), dtype=torch.float32)),
+        lambda: L.forward(x, wr, bias, ws=torch.empty(16, dtype=torch.uint8)),      # workspace too small
+        lambda: L.forward(x[0], wr, bias),                                          # 1-D x
+        lambda: L.permute(idx.long()),
+        lambda: L.permute(idx[:, :1].contiguous()),
+        lambda: L.expert_ffn(x, ps[:-1], pk, offsets, w),
+        lambda: L.combine(y[:, :128].contiguous(), inv),
+        lambda: L.register(8, torch.zeros((2 * I, H), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16)),
+        lambda: L.register(0, torch.zeros((H, I), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16)),
+        lambda: L.register(0, torch.zeros((2 * I, H), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16),
+                           torch.zeros((2, 2)), None),                              # scales on bf16 experts
+        lambda: L.register(0, torch.zeros((2 * I, H), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16),
+                           location=B.MOE_LOC_HOST_PINNED),                         # host weights, not pinned
+        lambda: L.register(0, torch.zeros((2 * I, H), dtype=torch.bfloat16), torch.zeros((H, I), dtype=torch.bfloat16),
+                           location=7),
+    ]
+    for i, f in enumerate(bad):
+        with pytest.raises((TypeError, ValueError)):
+            f()
+        assert len(calls) == n_ok, f"bad call {i} reached the C ABI"
+
+    F = layer(B.MOE_FP8_E4M3_B128)
+    qg, qd = torch.zeros((2 * I, H), dtype=torch.uint8), torch.zeros((H, I), dtype=torch.uint8)
+    sg, sd = torch.zeros((2 * I // 128, H // 128)), torch.zeros((H // 128, I // 128))
+    F.register(0, qg, qd, sg, sd)
+    with pytest.raises(TypeError):
+        F.register(0, qg, qd, sg.double(), sd)
+    with pytest.raises(TypeError):
+        F.register(0, qg, qd, None, sd)
