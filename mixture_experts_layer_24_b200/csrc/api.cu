@@ -11,6 +11,7 @@
 // row "identity").
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -86,14 +87,21 @@ struct moe_ctx {
 };
 
 namespace {
-// Counts one kernel launch and, when timing is on, brackets it with events on
-// the launching stream.
+// Step names of the MOE_PROF_* kinds, for the NVTX ranges below.
+static const char* const kStepNames[MOE_PROF_KINDS] = {"moe.router",  "moe.topk", "moe.permute",
+                                                       "moe.gather",  "moe.gate_up", "moe.down",
+                                                       "moe.quant",   "moe.combine", "moe.ffn_fused"};
+
+// Counts one kernel launch, names it with an NVTX range on the host timeline
+// (free unless a profiler is attached), and, when timing is on, brackets it
+// with events on the launching stream.
 struct Prof {
   moe_ctx* c;
   int kind;
   cudaStream_t s;
   cudaEvent_t a = nullptr;
   Prof(moe_ctx* c_, int kind_, cudaStream_t s_) : c(c_), kind(kind_), s(s_) {
+    nvtxRangePushA(kStepNames[kind]);
     if (c->prof_on) {
       std::lock_guard<std::mutex> g(c->prof_mu);
       a = c->take_event();
@@ -101,6 +109,7 @@ struct Prof {
     }
   }
   ~Prof() {
+    nvtxRangePop();
     c->launches.fetch_add(1, std::memory_order_relaxed);
     if (a) {
       std::lock_guard<std::mutex> g(c->prof_mu);
