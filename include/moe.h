@@ -138,7 +138,10 @@ moe_status_t moe_permute(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_t
  * expert lives in pinned host memory, this call reads offsets back to the host
  * (it synchronises `stream` once), stages the routed cold experts into spare
  * HBM slots on an internal copy stream, and computes them with the same
- * kernels as resident experts (bit-identical results). */
+ * kernels as resident experts (bit-identical results). The slot table's
+ * pinned staging buffer, its cache state and its spare slots are shared by
+ * every call that uses the table: such calls must run on one stream, or the
+ * caller must order them (an event), as with the workspace. */
 moe_status_t moe_expert_ffn(moe_ctx_t* ctx, moe_slots_t* slots, const void* x, const int32_t* perm_src,
                             const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T,
                             float* y_pair, void* ws, size_t ws_bytes, moe_stream_t stream);
