@@ -54,6 +54,13 @@ def _load():
         lib.oracle_e4m3_to_f32.restype = ctypes.c_float
         lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
         lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        lib.oracle_f32_to_e2m1.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_e2m1.restype = ctypes.c_uint8
+        lib.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
+        lib.oracle_e2m1_to_f32.restype = ctypes.c_float
+        lib.oracle_quant_mx.argtypes = [P, I, I, I, P, P]
+        lib.oracle_ffn_mxfp4.argtypes = [P, I, I, I, P, P, P, P, P, P, P, P, P, I]
+        lib.oracle_ffn_mxfp4.restype = I
         _lib = lib
     return _lib
 
@@ -176,6 +183,30 @@ def ffn_fp8(x_u16, pair_token, pair_expert, pair_weight, q_gu, s_gu, q_dn, s_dn,
     return (y, h) if want_h else y
 
 
+def ffn_mxfp4(x_u16, pair_token, pair_expert, pair_weight, q_gu, s_gu, q_dn, s_dn, E, threads=0,
+              want_h=False):
+    """y [npairs, H] fp32 for MXFP4 experts (e2m1 codes [2I, H] / [H, I], one
+    E8M0 scale byte per 32 elements along each row); activations MX e4m3."""
+    lib = _load()
+    T, H = x_u16.shape
+    pair_token = np.ascontiguousarray(pair_token, np.int32)
+    pair_expert = np.ascontiguousarray(pair_expert, np.int32)
+    pair_weight = np.ascontiguousarray(pair_weight, np.float32)
+    n = pair_token.shape[0]
+    pqg, k1 = _ptr_array(q_gu, E, np.uint8)
+    psg, k2 = _ptr_array(s_gu, E, np.uint8)
+    pqd, k3 = _ptr_array(q_dn, E, np.uint8)
+    psd, k4 = _ptr_array(s_dn, E, np.uint8)
+    I = k1[0].shape[0] // 2
+    y = np.empty((n, H), np.float32)
+    h = np.empty((n, I), np.uint16) if want_h else None
+    rc = lib.oracle_ffn_mxfp4(_p(x_u16), H, I, n, _p(pair_token), _p(pair_expert), _p(pair_weight), pqg, psg,
+                              pqd, psd, _p(y), None if h is None else _p(h), threads)
+    if rc != 0:
+        raise ValueError("oracle_ffn_mxfp4: weights of a needed expert were not given")
+    return (y, h) if want_h else y
+
+
 def combine(y_pair: np.ndarray, inv: np.ndarray) -> np.ndarray:
     """out [T, H] bf16 bits = bf16(sum_k y_pair[inv[t,k]]) in k order."""
     lib = _load()
@@ -198,6 +229,30 @@ def quant_e4m3(src_u16: np.ndarray, block_rows: int):
     s = np.empty(((rows + block_rows - 1) // block_rows, cols // 128), np.float32)
     lib.oracle_quant_e4m3(_p(src_u16), rows, cols, block_rows, _p(q), _p(s))
     return q, s
+
+
+def quant_mx(src_u16: np.ndarray, elem: str = "e2m1"):
+    """(q uint8 [rows, cols] one code per byte, scales uint8 [rows, cols/32] E8M0)."""
+    lib = _load()
+    src_u16 = np.ascontiguousarray(src_u16, np.uint16)
+    rows, cols = src_u16.shape
+    assert cols % 32 == 0
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows, cols // 32), np.uint8)
+    lib.oracle_quant_mx(_p(src_u16), rows, cols, {"e2m1": 0, "e4m3": 1}[elem], _p(q), _p(s))
+    return q, s
+
+
+def f32_to_e2m1(v: float) -> int:
+    return int(_load().oracle_f32_to_e2m1(float(v)))
+
+
+def e2m1_to_f32(c: int) -> float:
+    return float(_load().oracle_e2m1_to_f32(int(c)))
+
+
+def e2m1_table() -> np.ndarray:
+    return np.array([e2m1_to_f32(c) for c in range(16)], dtype=np.float32)
 
 
 def f32_to_e4m3(v: float) -> int:
@@ -232,7 +287,8 @@ def forward(x_u16, wr, bias, K, E, w_gu, w_dn, dtype="bf16", scales=None, thread
     tokens: optional index array; when given only those tokens' outputs are
     computed (routing of a token depends on that token alone, and its output
     on its own pairs alone), and 'out' has one row per listed token.
-    For dtype 'fp8', w_gu/w_dn hold e4m3 codes and ``scales`` = (s_gu, s_dn)."""
+    For dtype 'fp8', w_gu/w_dn hold e4m3 codes and ``scales`` = (s_gu, s_dn);
+    for 'mxfp4', e2m1 codes and their E8M0 scale bytes."""
     T, H = x_u16.shape
     logits, idx, w64 = route(x_u16, wr, bias, K, threads)
     counts, offsets, perm_src, perm_k, inv = permute(idx, E)
@@ -243,6 +299,9 @@ def forward(x_u16, wr, bias, K, E, w_gu, w_dn, dtype="bf16", scales=None, thread
     pw = w64[sel].reshape(-1).astype(np.float32)
     if dtype == "bf16":
         y = ffn_bf16(x_u16, pt, pe, pw, w_gu, w_dn, E, acc64=acc64, threads=threads)
+    elif dtype == "mxfp4":
+        s_gu, s_dn = scales
+        y = ffn_mxfp4(x_u16, pt, pe, pw, w_gu, s_gu, w_dn, s_dn, E, threads=threads)
     else:
         s_gu, s_dn = scales
         y = ffn_fp8(x_u16, pt, pe, pw, w_gu, s_gu, w_dn, s_dn, E, threads=threads)

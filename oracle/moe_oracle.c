@@ -23,6 +23,10 @@
  *   7. FP8 variant    e4m3 weights with 128x128 block scales, activations
  *                     quantised per token per 128 columns, per-block
  *                     promotion acc = fma(P_kb, sx*sw, acc)
+ *   8. MXFP4 variant  OCP MX block scaling along K: e2m1 weights and e4m3
+ *                     activations, one E8M0 (power-of-two) scale per 32
+ *                     consecutive elements of a row, per-block promotion
+ *                     acc = fma(P_b, 2^(ew + ea), acc)
  *
  * Reading of the layer where the definition leaves a step open (each one is
  * listed with its reason in the design notes):
@@ -362,6 +366,146 @@ int oracle_ffn_fp8(const uint16_t* x, int H, int I, int npairs, const int32_t* p
       oracle_quant_e4m3(hb, 1, I, 1, qh, shh);
       for (int o = 0; o < H; ++o) {
         float acc = dot_fp8(qdn[e] + (size_t)o * I, sdn[e] + (size_t)(o / 128) * (I / 128), qh, shh, I, lut);
+        y[(size_t)p * H + o] = pair_weight[p] * acc;
+      }
+    }
+    free(qx);
+    free(sx);
+    free(hb);
+    free(qh);
+    free(shh);
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------- MX (e2m1) -- */
+/* OCP Microscaling formats: E2M1 elements (sign, 2 exponent bits with bias
+ * 1, 1 mantissa bit; no infinities or NaN; magnitudes 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6) and E4M3 elements (above), with one E8M0 scale -- a power of two,
+ * stored as its exponent + 127 -- per block of 32 consecutive elements. */
+
+float oracle_e2m1_to_f32(uint8_t c) {
+  int sign = (c >> 3) & 1;
+  int ex = (c >> 1) & 3;
+  int man = c & 1;
+  double v = (ex == 0) ? 0.5 * man : ldexp(1.0 + 0.5 * man, ex - 1);
+  return (float)(sign ? -v : v);
+}
+
+/* fp32 -> e2m1, round to nearest even, saturating to +-6 (finite inputs). */
+uint8_t oracle_f32_to_e2m1(float f) {
+  uint8_t sign = signbit(f) ? 0x8 : 0x0;
+  double a = fabs((double)f);
+  if (a >= 6.0) return sign | 0x7;
+  if (a < 1.0) {
+    /* subnormal step 0.5: codes 0 (0), 1 (0.5) and 2 (1.0, the smallest normal) */
+    double q = nearbyint(a * 2.0); /* exact scaling; default mode = RNE */
+    return sign | (uint8_t)q;
+  }
+  int e;
+  double m = frexp(a, &e); /* a = m * 2^e, m in [0.5, 1) */
+  m *= 2.0;
+  e -= 1; /* a = m * 2^e, m in [1, 2), e in {0, 1, 2} */
+  double q = nearbyint((m - 1.0) * 2.0);
+  if (q == 2.0) {
+    q = 0.0;
+    e += 1;
+  }
+  if (e > 2) return sign | 0x7; /* only from rounding just below 6 up: 6 itself */
+  return sign | (uint8_t)(((e + 1) << 1) | (int)q);
+}
+
+/* MX quantiser of a [rows, cols] bf16 matrix along its rows: for each run of
+ * 32 elements, X = 2^(floor(log2 amax) - emax) with emax = 2 for E2M1
+ * (6 = 1.5 * 2^2) and 8 for E4M3 (448 = 1.75 * 2^8), clamped to 2^-127 ..
+ * 2^127 (an all-zero block takes 2^-127); q = encode(v / X), round to
+ * nearest even, saturating (the block's largest element can exceed the
+ * element format's maximum after scaling and is then clamped to it).
+ * q [rows, cols] one code per byte; scales [rows, cols/32] E8M0 bytes.
+ * elem: 0 = E2M1, 1 = E4M3. */
+void oracle_quant_mx(const uint16_t* src, int rows, int cols, int elem, uint8_t* q, uint8_t* scales) {
+  const int emax = elem == 0 ? 2 : 8;
+  const int nb = cols / 32;
+  for (int r = 0; r < rows; ++r)
+    for (int b = 0; b < nb; ++b) {
+      const uint16_t* v = src + (size_t)r * cols + (size_t)b * 32;
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i) {
+        float a = fabsf(bf16_to_f32(v[i]));
+        if (a > amax) amax = a;
+      }
+      int sexp = -127;
+      if (amax > 0.0f) {
+        int e;
+        frexpf(amax, &e); /* amax = m * 2^e, m in [0.5, 1): floor(log2 amax) = e - 1 */
+        sexp = (e - 1) - emax;
+        if (sexp < -127) sexp = -127;
+        if (sexp > 127) sexp = 127;
+      }
+      scales[(size_t)r * nb + b] = (uint8_t)(sexp + 127);
+      for (int i = 0; i < 32; ++i) {
+        float t = (float)ldexp((double)bf16_to_f32(v[i]), -sexp);
+        q[(size_t)r * cols + (size_t)b * 32 + i] = elem == 0 ? oracle_f32_to_e2m1(t) : oracle_f32_to_e4m3(t);
+      }
+    }
+}
+
+/* MX dot product of a weight row (e2m1 codes, E8M0 scales) with an
+ * activation row (e4m3 codes, E8M0 scales): P_b = sum over the 32-element
+ * block of f32(w)*f32(a) (fp32), acc = fmaf(P_b, 2^(ew_b + ea_b), acc) for
+ * blocks in increasing order. */
+static float dot_mx(const uint8_t* qw, const uint8_t* sw, const uint8_t* qa, const uint8_t* sa, int n,
+                    const float* lw, const float* la) {
+  float acc = 0.0f;
+  for (int b = 0; b < n / 32; ++b) {
+    float part = 0.0f;
+    for (int i = b * 32; i < (b + 1) * 32; ++i) part = fmaf(lw[qw[i]], la[qa[i]], part);
+    acc = fmaf(part, (float)ldexp(1.0, (int)sw[b] + (int)sa[b] - 254), acc);
+  }
+  return acc;
+}
+
+/* MXFP4 FFN for a list of pairs.
+ *   x [T, H] bf16 (quantised here to MX e4m3 per token);
+ *   qgu[e] [2I, H] e2m1 codes + sgu[e] [2I, H/32] E8M0; qdn[e] [H, I] + sdn[e] [H, I/32].
+ *   y [npairs, H] fp32; h [npairs, I] bf16 (may be NULL). */
+int oracle_ffn_mxfp4(const uint16_t* x, int H, int I, int npairs, const int32_t* pair_token,
+                     const int32_t* pair_expert, const float* pair_weight, const uint8_t* const* qgu,
+                     const uint8_t* const* sgu, const uint8_t* const* qdn, const uint8_t* const* sdn, float* y,
+                     uint16_t* h, int threads) {
+  for (int p = 0; p < npairs; ++p) {
+    int e = pair_expert[p];
+    if (!qgu[e] || !sgu[e] || !qdn[e] || !sdn[e]) return -1;
+  }
+  float lw[16], la[256];
+  for (int c = 0; c < 16; ++c) lw[c] = oracle_e2m1_to_f32((uint8_t)c);
+  for (int c = 0; c < 256; ++c) la[c] = oracle_e4m3_to_f32((uint8_t)c);
+#ifdef _OPENMP
+  if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel
+#endif
+  {
+    uint8_t* qx = (uint8_t*)malloc((size_t)H);
+    uint8_t* sx = (uint8_t*)malloc((size_t)(H / 32));
+    uint16_t* hb = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)I);
+    uint8_t* qh = (uint8_t*)malloc((size_t)I);
+    uint8_t* shh = (uint8_t*)malloc((size_t)(I / 32));
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+    for (int p = 0; p < npairs; ++p) {
+      int e = pair_expert[p];
+      oracle_quant_mx(x + (size_t)pair_token[p] * H, 1, H, 1, qx, sx);
+      for (int j = 0; j < I; ++j) {
+        int rg = j, ru = I + j;
+        float g = dot_mx(qgu[e] + (size_t)rg * H, sgu[e] + (size_t)rg * (H / 32), qx, sx, H, lw, la);
+        float u = dot_mx(qgu[e] + (size_t)ru * H, sgu[e] + (size_t)ru * (H / 32), qx, sx, H, lw, la);
+        hb[j] = f32_to_bf16(silu_f32(g) * u);
+      }
+      if (h) memcpy(h + (size_t)p * I, hb, sizeof(uint16_t) * (size_t)I);
+      oracle_quant_mx(hb, 1, I, 1, qh, shh);
+      for (int o = 0; o < H; ++o) {
+        float acc = dot_mx(qdn[e] + (size_t)o * I, sdn[e] + (size_t)o * (I / 32), qh, shh, I, lw, la);
         y[(size_t)p * H + o] = pair_weight[p] * acc;
       }
     }

@@ -63,6 +63,12 @@ MUTATIONS = [
     ("quantiser_zero_block_scale", "float s = (amax == 0.0f) ? 1.0f : amax / 448.0f;", "float s = amax / 448.0f;"),
     ("fp8_activation_scale_dropped", "acc = fmaf(part, sa[kb] * sw[kb], acc);", "acc = fmaf(part, sw[kb], acc);"),
     ("fp8_weight_block_row", "sgu[e] + (size_t)(rg / 128) * (H / 128)", "sgu[e] + (size_t)(rg / 256) * (H / 128)"),
+    # MX (MXFP4 weights, MX e4m3 activations)
+    ("e2m1_round_half_up", "double q = nearbyint((m - 1.0) * 2.0);", "double q = floor((m - 1.0) * 2.0 + 0.5);"),
+    ("mx_e2m1_emax_3", "const int emax = elem == 0 ? 2 : 8;", "const int emax = elem == 0 ? 3 : 8;"),
+    ("mx_scale_applied_upside_down", "ldexp((double)bf16_to_f32(v[i]), -sexp)", "ldexp((double)bf16_to_f32(v[i]), sexp)"),
+    ("mx_zero_block_scale", "int sexp = -127;", "int sexp = 0;"),
+    ("mx_activation_scale_dropped", "(int)sw[b] + (int)sa[b] - 254", "(int)sw[b] - 127"),
     # composition of the steps
     ("py_weights_of_the_wrong_slot", "pw = w64[sel].reshape(-1)", "pw = w64[sel][:, ::-1].reshape(-1)"),
     ("py_pairs_of_the_wrong_token", "pt = np.repeat(sel, K)", "pt = np.tile(sel, K)"),

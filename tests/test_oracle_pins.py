@@ -331,3 +331,124 @@ def test_fp8_ffn_against_float64_dequantised_math():
     # and the fp8 layer stays near the bf16 one
     yb = oracle.ffn_bf16(oracle.as_u16(x), pt, pe, pw, gu, dn, 1)
     assert np.max(np.abs(y - yb)) <= 1e-1 * np.max(np.abs(yb))
+
+
+# --------------------------------------------------------------------- MX --
+
+MX = json.load(open(os.path.join(GOLD, "mx_cases.json")))
+
+
+def test_e2m1_decode_table():
+    """The OCP MX E2M1 element: sign, 2 exponent bits (bias 1), 1 mantissa bit."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    t = oracle.e2m1_table()
+    assert t[:8].tolist() == mags
+    assert t[8:].tolist() == [-m for m in mags]
+    assert np.signbit(t[8])
+
+
+def test_e2m1_golden_cases():
+    for c in MX["e2m1_cases"]:
+        assert oracle.f32_to_e2m1(c["x"]) == int(c["code"], 16), c["why"]
+
+
+def test_e2m1_encoder_against_exhaustive_nearest():
+    """Round to nearest even by exhaustive search over the 8 magnitudes (ties
+    go to the code with mantissa bit 0), against the oracle's arithmetic
+    encoder; saturation above 6."""
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    rng = np.random.default_rng(11)
+    mids = (mags[:-1] + mags[1:]) / 2
+    vals = np.concatenate([rng.uniform(-6.5, 6.5, 4000), mids, -mids, mags, rng.uniform(-0.6, 0.6, 500)])
+    vals = vals.astype(np.float32)
+    for v in vals:
+        a = abs(float(v))
+        if a >= 6.0:
+            want = 7
+        else:
+            d = np.abs(mags - a)
+            best = np.flatnonzero(d == d.min())
+            want = int(best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0])
+        want |= 8 if np.signbit(v) else 0
+        assert oracle.f32_to_e2m1(float(v)) == want, float(v)
+
+
+def test_mx_block_golden_cases():
+    for c in MX["block_cases"]:
+        blk = np.zeros((1, 32), np.uint16)
+        if "values_bf16" in c:
+            for i, hx in enumerate(c["values_bf16"]):
+                blk[0, i] = int(hx, 16)
+        else:
+            vals = np.zeros(32, np.float32)
+            vals[:len(c["values"])] = c["values"]
+            blk[0] = bf16_bits_np(vals)
+        q, s = oracle.quant_mx(blk, c["elem"])
+        assert int(s[0, 0]) == c["scale"], c["why"]
+        for i, code in c["codes"].items():
+            assert int(q[0, int(i)]) == int(code, 16), c["why"]
+
+
+def bf16_bits_np(v):
+    return torch.from_numpy(np.asarray(v, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_mx_quantiser_properties():
+    """For every 32-element block of seeded rows: the scale X is the power of
+    two with 2^emax <= amax / X < 2^(emax+1); each element decodes to the
+    nearest representable value of v / X (or the format's largest, when
+    v / X lies beyond it); an all-zero block has X = 2^-127 and zero codes."""
+    src = synth.tokens(6, 256, seed=19)
+    su = oracle.as_u16(src)
+    su[2, 64:96] = 0
+    v = f32(su)
+    for elem, emax, table, top in (("e2m1", 2, oracle.e2m1_table(), 6.0), ("e4m3", 8, oracle.e4m3_table(), 448.0)):
+        q, s = oracle.quant_mx(su, elem)
+        finite = table[~np.isnan(table)].astype(np.float64)
+        for r in range(v.shape[0]):
+            for b in range(v.shape[1] // 32):
+                blk = v[r, b * 32:(b + 1) * 32]
+                X = 2.0 ** (int(s[r, b]) - 127)
+                amax = np.abs(blk).max()
+                if amax == 0:
+                    assert s[r, b] == 0 and np.all(q[r, b * 32:(b + 1) * 32] & 0x7F == 0)
+                    continue
+                assert 2.0 ** emax <= amax / X < 2.0 ** (emax + 1)
+                deq = table[q[r, b * 32:(b + 1) * 32]].astype(np.float64)
+                for vi, di in zip(blk / X, deq):
+                    tgt = np.clip(vi, -top, top)
+                    assert abs(di - tgt) == np.min(np.abs(finite - tgt))  # nearest (ties either way)
+
+
+def test_mxfp4_ffn_against_float64_dequantised_math():
+    T, H, I = 3, 256, 128
+    x = synth.tokens(T, H, seed=23)
+    gu, dn = _experts(1, H, I, seed=23)
+    qgu, sgu = oracle.quant_mx(gu[0], "e2m1")
+    qdn, sdn = oracle.quant_mx(dn[0], "e2m1")
+    l4 = oracle.e2m1_table().astype(np.float64)
+    l8 = oracle.e4m3_table().astype(np.float64)
+    pt = np.arange(T, dtype=np.int32)
+    pe = np.zeros(T, np.int32)
+    pw = np.array([1.0, 0.5, 0.25], np.float32)
+    y, h = oracle.ffn_mxfp4(oracle.as_u16(x), pt, pe, pw, {0: qgu}, {0: sgu}, {0: qdn}, {0: sdn}, 1, want_h=True)
+
+    def deq(q, s, table):
+        return table[q] * np.repeat(2.0 ** (s.astype(np.float64) - 127), 32, axis=1)
+
+    Wgu, Wdn = deq(qgu, sgu, l4), deq(qdn, sdn, l4)
+    for t in range(T):
+        qx, sx = oracle.quant_mx(oracle.as_u16(x)[t:t + 1], "e4m3")
+        xd = deq(qx, sx, l8)[0]
+        g = Wgu[:I] @ xd
+        u = Wgu[I:] @ xd
+        hh = bf16_round_np(silu64(g) * u)
+        assert np.max(np.abs(f32(h[t]) - hh)) <= 2 ** -7 * np.max(np.abs(hh))
+        qh, sh = oracle.quant_mx(h[t:t + 1], "e4m3")
+        hd = deq(qh, sh, l8)[0]
+        ref = pw[t] * (Wdn @ hd)
+        assert np.max(np.abs(y[t] - ref)) <= 1e-4 * np.max(np.abs(ref))
+    # and the MXFP4 layer stays within a few tens of percent of the bf16 one (one mantissa bit per weight)
+    yb = oracle.ffn_bf16(oracle.as_u16(x), pt, pe, pw, gu, dn, 1)
+    rel = np.sqrt(np.mean((y - yb) ** 2)) / np.sqrt(np.mean(yb ** 2))
+    assert rel <= 0.25, rel
