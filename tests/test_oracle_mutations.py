@@ -14,8 +14,6 @@ import shutil
 import subprocess
 import sys
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
 
@@ -94,8 +92,13 @@ def test_unmodified_copy_passes_the_pins(tmp_path):
     assert r.returncode == 0, r.stdout[-3000:]
 
 
-@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
-def test_planted_mistake_fails_a_pin(tmp_path, name, old, new):
-    r = _run_pins(tmp_path, name, old, new)
-    assert r.returncode != 0, f"{name} survived every pin:\n{r.stdout[-2000:]}"
-    assert r.returncode == 1, f"{name}: the pins did not run to a failure:\n{r.stdout[-2000:]}{r.stderr[-2000:]}"
+def test_every_planted_mistake_fails_a_pin(tmp_path):
+    """All mutants at once (one process each, run side by side)."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(2, (os.cpu_count() or 2))) as ex:
+        runs = list(ex.map(lambda m: (m[0], _run_pins(tmp_path, *m)), MUTATIONS))
+    survived = [name for name, r in runs if r.returncode == 0]
+    crashed = [(name, r.returncode, r.stderr[-500:]) for name, r in runs if r.returncode not in (0, 1)]
+    assert not survived, f"mistakes that no pin caught: {survived}"
+    assert not crashed, f"mutants that did not run to a pin failure: {crashed}"
+    assert len(runs) == len({m[0] for m in MUTATIONS}) == len(MUTATIONS)
