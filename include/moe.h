@@ -247,6 +247,14 @@ moe_status_t moe_plan_hot_set(const int64_t* hist, int E, int n_hot, int32_t* ho
 
 /* ---- diagnostics ------------------------------------------------------ */
 
+/* Test hook for failure detection: launches one thread on `stream` that
+ * waits, with the library's bounded acquire-load loop, until *flag (a device
+ * int32) is nonzero or limit_ns nanoseconds pass (%globaltimer). On time-out it
+ * sets MOE_DEV_TIMEOUT in the device status word and returns; nothing traps,
+ * and the context stays usable. limit_ns must be in (0, 2e9]: larger or
+ * non-positive limits return MOE_ERR_INVALID_ARG without launching. */
+moe_status_t moe_debug_wait_flag(moe_ctx_t* ctx, const int32_t* flag, int64_t limit_ns, moe_stream_t stream);
+
 /* Copies the device status word to *status (synchronises the context's
  * device); reset != 0 clears it afterwards. */
 moe_status_t moe_get_device_status(moe_ctx_t* ctx, int32_t* status, int reset);

@@ -25,6 +25,7 @@ from .binding import (  # noqa: F401
     moe_combine,
     moe_ctx_create,
     moe_ctx_destroy,
+    moe_debug_wait_flag,
     moe_expert_ffn,
     moe_forward,
     moe_get_device_status,

@@ -33,7 +33,8 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_expert_ffn", "moe_combine", "moe_forward", "moe_quantize_e4m3", "moe_slots_create",
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
-           "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy"]
+           "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy",
+           "moe_debug_wait_flag"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
@@ -90,6 +91,7 @@ def lib():
         "moe_profile_enable": ([P, I], S),
         "moe_profile_read": ([P, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], S),
         "moe_route_noalloc": ([P, P, P, I, I, I, I, P, P, P], S),
+        "moe_debug_wait_flag": ([P, P, ctypes.c_int64, P], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -224,6 +226,12 @@ def moe_get_device_status(ctx, reset: bool = True) -> int:
     v = ctypes.c_int32()
     _check(lib().moe_get_device_status(ctx, ctypes.byref(v), int(reset)), "moe_get_device_status")
     return v.value
+
+
+def moe_debug_wait_flag(ctx, flag, limit_ns: int, stream=None):
+    """Test hook: one thread waits (bounded by limit_ns) for the device int32
+    ``flag`` to become nonzero; on time-out the status word gets MOE_DEV_TIMEOUT."""
+    _check(lib().moe_debug_wait_flag(ctx, _p(flag), int(limit_ns), _s(stream)), "moe_debug_wait_flag")
 
 
 def moe_launch_count(ctx) -> int:

@@ -26,6 +26,11 @@
 
 using namespace moe;
 
+namespace moe {
+// debug.cu: the bounded-wait test hook behind moe_debug_wait_flag
+cudaError_t launch_debug_wait_flag(const int* flag, uint64_t limit_ns, int* status, cudaStream_t s);
+}  // namespace moe
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -504,6 +509,14 @@ moe_status_t moe_profile_read(moe_ctx_t* ctx, int kind, double* total_ms, int64_
     ctx->prof_ms[kind] = 0.0;
     ctx->prof_n[kind] = 0;
   }
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_wait_flag(moe_ctx_t* ctx, const int32_t* flag, int64_t limit_ns, moe_stream_t stream) {
+  if (!ctx || !flag) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
+  if (limit_ns <= 0 || limit_ns > 2000000000LL) return fail(MOE_ERR_INVALID_ARG, "limit_ns must be in (0, 2 s]");
+  MOE_CUDA(moe::launch_debug_wait_flag(flag, static_cast<uint64_t>(limit_ns), ctx->d_status,
+                                       static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

@@ -65,6 +65,7 @@ def test_host_side_argument_checks(lib):
     assert lib.moe_workspace_size(None, 5) == 0
     assert lib.moe_quantize_e4m3(None, 0, 128, 1, None, None, None) == 0  # empty input is a no-op
     assert lib.moe_slots_set_policy(None, M.MOE_SLOTS_LRU) == 1  # NULL table
+    assert lib.moe_debug_wait_flag(None, None, 1000, None) == 1  # NULL context
     assert M.MOE_SLOTS_LRU != M.MOE_SLOTS_PER_CALL
 
 
