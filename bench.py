@@ -149,7 +149,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -328,7 +328,7 @@ def run_ours(args):
 
     use_graphs = not args.eager
     clocks = ClockSampler(local)
-    clocks.start()  # sampled through warm-up and the timed region (the timed region alone is short)
+    clocks.start()  # every 20 ms by a separate process, through warm-up and the timed region (the latter is short)
     # warm-up (also captures the graphs)
     launches0 = layer.launches()
     time_forwards(layer, xs, wr, bias, flush, stream, 1, graphs=False)
