@@ -38,7 +38,10 @@
  *   - Errors the device detects (an expert id outside [0, E), an expert that
  *     is routed to but not registered, a bounded wait that ran out) set bits
  *     in the context's device status word (moe_get_device_status) and never
- *     trap; the affected outputs are unspecified.
+ *     trap. A pair with a bad expert id or an unregistered expert is dropped:
+ *     moe_forward leaves it out of the token's sum (as if the token had one
+ *     pair fewer), moe_expert_ffn writes its y_pair row as zeros. Outputs after
+ *     a time-out are unspecified.
  *   - There is no CPU fallback: every step runs in this library's kernels.
  *
  * Size limits: H and I multiples of 128; 1 <= K <= 32; K <= E <= 1024;
@@ -79,7 +82,7 @@ enum { MOE_LOC_HBM = 0, MOE_LOC_HOST_PINNED = 1 };
 /* Bits of the device status word. */
 enum {
   MOE_DEV_BAD_EXPERT = 1, /* a top-k index outside [0, E) reached moe_permute */
-  MOE_DEV_NO_SLOT = 2,    /* a pair was routed to an expert with no registered weights */
+  MOE_DEV_NO_SLOT = 2,    /* a pair was routed to an expert with no registered weights (pair dropped) */
   MOE_DEV_TIMEOUT = 4     /* a bounded wait inside a kernel gave up (~2 s) */
 };
 
@@ -180,11 +183,13 @@ moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_ro
  * logits, is a fixed array of MOE_ROUTE_NOALLOC_MAX_LOGITS floats (256 KiB)
  * compiled into the library, present on every GPU that loads it until the
  * process exits. T * E above that limit returns MOE_ERR_UNSUPPORTED. The
- * first call on each device looks up the array's device address (make it
- * before any stream capture). All calls share the array: calls that overlap
- * on the GPU (two streams, two host threads) race and must be serialised by
- * the caller. Size limits otherwise as above; errors do not set a status word
- * (there is no context). */
+ * first call on each device looks up the array's device address and keeps it
+ * for that device's CUDA context; the first call in a new context (after
+ * cudaDeviceReset) looks it up again. Make those calls before any stream
+ * capture: a lookup during capture is refused with MOE_ERR_UNSUPPORTED. All
+ * calls share the array: calls that overlap on the GPU (two streams, two host
+ * threads) race and must be serialised by the caller. Size limits otherwise as
+ * above; errors do not set a status word (there is no context). */
 #define MOE_ROUTE_NOALLOC_MAX_LOGITS 65536
 moe_status_t moe_route_noalloc(const void* x, const float* w_router, const float* logit_bias, int T, int H, int E,
                                int K, int32_t* topk_idx, float* topk_w, moe_stream_t stream);

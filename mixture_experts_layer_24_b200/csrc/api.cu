@@ -684,6 +684,8 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   int32_t* lm = at<int32_t>(ws, W.list_map);
   int32_t* np = at<int32_t>(ws, W.nt_prefix);
   const int ntile_bound = (P + bn - 1) / bn + std::min(E, P);
+  // pairs routed to an expert with no registered weights: zero rows, and inv = -1 in the forward
+  const DropArgs drop{perm_src, perm_k, c.top_k, const_cast<int32_t*>(inv), y_pair, c.hidden};
 
   if (sl->n_host == 0) {
     sl->stats.last_cold = 0;
@@ -693,7 +695,7 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
       {
         Prof p(ctx, MOE_PROF_PERMUTE, s);
         MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl,
-                                 at<int>(ws, W.sched), fused_sched_entries(E)));
+                                 at<int>(ws, W.sched), fused_sched_entries(E), drop));
       }
       Prof pg(ctx, MOE_PROF_GATHER, s);
       if (fp8) {
@@ -733,7 +735,10 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     ++touched;
     if (sl->loc[e] == MOE_LOC_HBM) hot.push_back(e);
     else if (sl->loc[e] == MOE_LOC_HOST_PINNED) cold.push_back(e);
-    else ctx->host_status |= MOE_DEV_NO_SLOT;
+    else {
+      ctx->host_status |= MOE_DEV_NO_SLOT;
+      MOE_CUDA(launch_drop_pairs(hoff[e], hoff[e + 1], drop, s));
+    }
   }
   sl->stats.last_touched = touched;
   sl->stats.last_cold = (int32_t)cold.size();

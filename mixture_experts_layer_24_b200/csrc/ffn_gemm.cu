@@ -1208,8 +1208,8 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
     }
   }
   __syncthreads();
-  if (blockIdx.x == 0)
-    for (int i = tid; i < P; i += 192) d.inv[i] = s_inv[i];
+  if (blockIdx.x == 0)  // a pair of an unregistered expert is dropped: the combine skips inv = -1
+    for (int i = tid; i < P; i += 192) d.inv[i] = (s_e[i] >= 0 && d.map_of[s_e[i]] < 0) ? -1 : s_inv[i];
   if (blockIdx.x == 0) {
     for (int e = tid; e < E; e += 192) {
       d.counts[e] = s_cnt[e];

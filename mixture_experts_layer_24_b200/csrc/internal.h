@@ -168,9 +168,24 @@ cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, cons
                                    const int32_t* offsets, int T, int K, int E, int chunk, int32_t* perm_src,
                                    int32_t* perm_k, int32_t* inv, cudaStream_t s, bool pdl);
 
+// Pairs routed to an expert with no registered weights are dropped: their
+// y_pair rows are zeroed and, with inv (the forward), their inv entries set to
+// -1 so the combine skips them. y_pair == nullptr: nothing is dropped.
+struct DropArgs {
+  const int32_t* perm_src;
+  const int32_t* perm_k;
+  int K;
+  int32_t* inv;     // nullable
+  float* y_pair;    // [P, H]
+  int H;
+};
+
 // FFN tile plan for the all-resident case: every expert with pairs, in order.
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
-                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0);
+                            int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched,
+                            int sched_n, const DropArgs& drop);
+// Drops the sorted pairs [p0, p1) (one unregistered expert) as above.
+cudaError_t launch_drop_pairs(int p0, int p1, const DropArgs& drop, cudaStream_t s);
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_src, const int32_t* offsets, int E, int P,
                                int H, void* x_perm, cudaStream_t s, bool pdl);

@@ -16,12 +16,17 @@
 // library, until the process exits. In host code its name is only a host-side
 // stand-in, never a device address: the first call on each device (with that
 // device current) looks the real address up with cudaGetSymbolAddress and
-// keeps it; later calls reuse it. Make that first call before any stream
-// capture. All calls share the one array, which keeps the last call's
-// contents; nothing in it needs to start at zero (every logit a call reads is
-// written by that call first). Calls that overlap on the GPU -- on two
-// streams, or from two host threads -- race on the array and must be
+// keeps it, together with the id of the device's current CUDA context; later
+// calls reuse it while that context is still the current one. A new context
+// (after cudaDeviceReset, say) gets its address looked up again. Make the
+// first call on a device, and the first after a reset, before any stream
+// capture: a lookup that would happen while the stream is capturing is refused
+// with MOE_ERR_UNSUPPORTED. All calls share the one array, which keeps the
+// last call's contents; nothing in it needs to start at zero (every logit a
+// call reads is written by that call first). Calls that overlap on the GPU --
+// on two streams, or from two host threads -- race on the array and must be
 // serialised by the caller.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -39,6 +44,33 @@ __device__ __align__(256) float g_route_scratch[kMaxLogits];
 
 std::mutex g_mu;
 float* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address belongs to
+
+// The driver's context calls, resolved through the runtime (the library does
+// not link libcuda directly).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Id of the calling thread's current CUDA context (0 if it cannot be read).
+unsigned long long current_ctx_id() {
+  if (!g_ctx_get_current || !g_ctx_get_id) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+      return 0;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_get_current(&c) != CUDA_SUCCESS || !c || g_ctx_get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 moe_status_t bad(moe_status_t st, const std::string& msg) {
   moe::record_error(msg.c_str());
@@ -63,19 +95,29 @@ extern "C" moe_status_t moe_route_noalloc(const void* x, const float* w_router, 
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return bad(MOE_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(err));
   if (dev < 0 || dev >= kMaxDevices) return bad(MOE_ERR_UNSUPPORTED, "device ordinal out of range");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    const unsigned long long ctx_id = current_ctx_id();  // 0: none current yet (the lookup below creates it)
+    if (!g_scratch_ptr[dev] || ctx_id == 0 || ctx_id != g_scratch_ctx[dev]) {
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      err = cudaStreamIsCapturing(s, &cap);
+      if (err != cudaSuccess)
+        return bad(MOE_ERR_CUDA, std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(err));
+      if (cap != cudaStreamCaptureStatusNone)
+        return bad(MOE_ERR_UNSUPPORTED,
+                   "moe_route_noalloc: the first call on a device (or after a device reset) looks up the static "
+                   "scratch's address and cannot run during stream capture; call it once before capturing");
       void* p = nullptr;
       err = cudaGetSymbolAddress(&p, g_route_scratch);
       if (err != cudaSuccess || !p)
         return bad(MOE_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(err));
       g_scratch_ptr[dev] = static_cast<float*>(p);
+      g_scratch_ctx[dev] = current_ctx_id();
     }
     scratch = g_scratch_ptr[dev];
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   err = moe::launch_router_logits(x, w_router, logit_bias, T, H, E, scratch, s);
   if (err != cudaSuccess) return bad(MOE_ERR_CUDA, std::string("router launch: ") + cudaGetErrorString(err));
   err = moe::launch_topk(scratch, T, E, K, topk_idx, topk_w, nullptr, s);

@@ -176,17 +176,32 @@ cudaError_t launch_permute_scatter(const int32_t* idx, const int32_t* rank, cons
 
 // --------------------------------------------------------------- FFN plan --
 // List = every expert in index order; experts with pairs but no registered
-// weights are flagged and given no tiles.
+// weights are flagged and given no tiles. Their pairs are dropped: their
+// y_pair rows are written as zeros and, when inv is given (the forward), their
+// inv entries become -1 so the combine leaves them out, as for a bad expert id.
+__device__ void drop_pair_range(int p0, int p1, const int32_t* __restrict__ perm_src,
+                                const int32_t* __restrict__ perm_k, int K, int32_t* __restrict__ inv,
+                                float4* __restrict__ y_pair, int H4) {
+  const int64_t n = (int64_t)(p1 - p0) * H4;
+  for (int64_t q = threadIdx.x; q < n; q += blockDim.x)
+    y_pair[(size_t)p0 * H4 + q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (inv)
+    for (int p = p0 + (int)threadIdx.x; p < p1; p += blockDim.x) inv[(size_t)perm_src[p] * K + perm_k[p]] = -1;
+}
+
 __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restrict__ offsets,
                                                          const int32_t* __restrict__ map_of, int E, int bn,
                                                          int32_t* __restrict__ list_expert,
                                                          int32_t* __restrict__ list_map,
                                                          int32_t* __restrict__ nt_prefix, int* status,
-                                                         int* __restrict__ sched, int sched_n) {
+                                                         int* __restrict__ sched, int sched_n, DropArgs drop) {
   __shared__ int sh[33];
+  __shared__ int s_missing;
   pdl_wait();
   pdl_trigger();
   const int e = threadIdx.x;
+  if (e == 0) s_missing = 0;
+  __syncthreads();
   for (int i = e; i < sched_n; i += blockDim.x) sched[i] = 0;  // counters of the fused decode FFN
   int nt = 0;
   if (e < E) {
@@ -195,22 +210,43 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
     nt = (cnt + bn - 1) / bn;
     if (cnt > 0 && m < 0) {
       flag_status(status, MOE_DEV_NO_SLOT);
+      s_missing = 1;
       nt = 0;
     }
     list_expert[e] = e;
     list_map[e] = m < 0 ? 0 : m;
   }
   int total;
-  const int pre = block_exclusive_scan_1024(nt, sh, &total);
+  const int pre = block_exclusive_scan_1024(nt, sh, &total);  // its barriers also publish s_missing
   if (e < E) nt_prefix[e] = pre;
   if (e == 0) nt_prefix[E] = total;
+  if (!s_missing || !drop.y_pair) return;  // block-uniform
+  for (int x = 0; x < E; ++x) {
+    const int p0 = offsets[x], p1 = offsets[x + 1];
+    if (p1 > p0 && map_of[x] < 0)
+      drop_pair_range(p0, p1, drop.perm_src, drop.perm_k, drop.K, drop.inv, reinterpret_cast<float4*>(drop.y_pair),
+                      drop.H / 4);
+  }
 }
 
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
                             int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched,
-                            int sched_n) {
+                            int sched_n, const DropArgs& drop) {
   return launch_ex(ffn_plan_kernel, dim3(1), dim3(1024), 0, s, pdl, offsets, map_of, E, bn, list_expert, list_map,
-                   nt_prefix, status, sched, sched ? sched_n : 0);
+                   nt_prefix, status, sched, sched ? sched_n : 0, drop);
+}
+
+// Pairs [p0, p1) of one unregistered expert on the host-synchronised path:
+// dropped as above.
+__global__ void __launch_bounds__(1024) drop_pairs_kernel(int p0, int p1, DropArgs drop) {
+  drop_pair_range(p0, p1, drop.perm_src, drop.perm_k, drop.K, drop.inv, reinterpret_cast<float4*>(drop.y_pair),
+                  drop.H / 4);
+}
+
+cudaError_t launch_drop_pairs(int p0, int p1, const DropArgs& drop, cudaStream_t s) {
+  if (p1 <= p0) return cudaSuccess;
+  drop_pairs_kernel<<<1, 1024, 0, s>>>(p0, p1, drop);
+  return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------- gather --
@@ -311,7 +347,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
     }
     if (i == 0) offsets[E] = total;
     if (i < P) {
-      inv[i] = p;
+      // with a plan (the forward), a pair of an unregistered expert is dropped: the combine skips inv = -1
+      inv[i] = (map_of && e >= 0 && map_of[e] < 0) ? -1 : p;
       if (p >= 0) {
         perm_src[p] = i / K;
         perm_k[p] = i - (i / K) * K;

@@ -454,12 +454,14 @@ __global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16
   bool ok = mbar_wait(bar, 0);
   ok = __syncthreads_and(ok);
   if (!ok && threadIdx.x == 0) {
-    // the copies did not land in time: flag it and give them one more bounded
-    // wait (they write this CTA's shared memory); the CTA then skips its
+    // the copies did not land in time: flag it. They write this CTA's shared
+    // memory, so they must land before the CTA exits: keep waiting, in bounded
+    // rounds of the same limit (a few more at most). The CTA then skips its
     // logits but still takes part in the top-k arrival count, which must
-    // return to zero
+    // return to zero.
     flag_status(status, MOE_DEV_TIMEOUT);
-    mbar_wait(bar, 0);
+    for (int round = 0; round < 4 && !mbar_wait(bar, 0); ++round) {
+    }
   }
   if (ok && e < E) {
     const float* wrow = ws + (size_t)warp * H;

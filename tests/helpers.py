@@ -19,7 +19,7 @@ class LayerCase:
     """Seeded inputs of one MoE layer on a CUDA device, plus a MoeLayer holding them."""
 
     def __init__(self, T, H, E, K, I, seed=0, zipf=None, wdtype=0, n_spare=0, hot=None, device="cuda",
-                 first_token=0):
+                 first_token=0, unregistered=()):
         import mixture_experts_layer_24_b200 as M
         self.T, self.H, self.E, self.K, self.I, self.seed, self.wdtype = T, H, E, K, I, seed, wdtype
         self.dev = torch.device(device)
@@ -46,6 +46,8 @@ class LayerCase:
         self.layer = M.MoeLayer(H, E, K, I, wdtype=wdtype, n_spare_slots=n_spare, device=self.dev)
         self.host = {}
         for e in range(E):
+            if e in unregistered:
+                continue
             resident = hot is None or e in hot
             if self.q is None:
                 g, d, sg, sd = self.w_gu[e], self.w_dn[e], None, None
@@ -73,18 +75,18 @@ class LayerCase:
         return xu, wr, bias
 
     def expert_arrays(self, experts):
+        """The oracle's copy of the experts' weights: the seeded bf16 draws, and for
+        FP8 their codes and 128x128 block scales from the oracle's own quantiser
+        (never the GPU's codes)."""
         gu, dn, sgu, sdn = {}, {}, {}, {}
         for e in experts:
             e = int(e)
+            g, d = oracle.as_u16(self.w_gu[e]), oracle.as_u16(self.w_dn[e])
             if self.q is None:
-                gu[e] = oracle.as_u16(self.w_gu[e])
-                dn[e] = oracle.as_u16(self.w_dn[e])
+                gu[e], dn[e] = g, d
             else:
-                qg, sg, qd, sd = self.q[e]
-                gu[e] = qg.cpu().numpy()
-                dn[e] = qd.cpu().numpy()
-                sgu[e] = sg.cpu().numpy()
-                sdn[e] = sd.cpu().numpy()
+                gu[e], sgu[e] = oracle.quant_e4m3(g, 128)
+                dn[e], sdn[e] = oracle.quant_e4m3(d, 128)
         return gu, dn, sgu, sdn
 
     def oracle_forward(self, tokens=None, threads=0):
@@ -110,3 +112,25 @@ def assert_close_out(got_u16: np.ndarray, ref_u16: np.ndarray, rel: float):
     scale = np.max(np.abs(r))
     assert err <= rel * scale, f"max|err| {err:.4g} > {rel} * max|ref| {scale:.4g}"
     return err / scale
+
+
+def oracle_layer_out(x_u16, wr, bias, K, E, H, I, seed, fp8=False, threads=0):
+    """Oracle outputs [rows, H] (bf16 bits) of the layer whose experts are
+    synth.expert_weights(e, H, I, seed) for the token rows x_u16 (uint16 [rows, H]).
+    The weights are drawn again on the host for the experts these rows route to
+    (and, for FP8, quantised by the oracle), so nothing comes from the GPU."""
+    _, idx, _ = oracle.route(x_u16, wr, bias, K, threads)
+    gu, dn, sgu, sdn = {}, {}, {}, {}
+    for e in np.unique(idx):
+        e = int(e)
+        g, d = synth.expert_weights(e, H, I, seed=seed)
+        g, d = oracle.as_u16(g), oracle.as_u16(d)
+        if fp8:
+            gu[e], sgu[e] = oracle.quant_e4m3(g, 128)
+            dn[e], sdn[e] = oracle.quant_e4m3(d, 128)
+        else:
+            gu[e], dn[e] = g, d
+    if fp8:
+        return oracle.forward(x_u16, wr, bias, K, E, gu, dn, dtype="fp8", scales=(sgu, sdn), threads=threads)["out"]
+    return oracle.forward(x_u16, wr, bias, K, E, gu, dn, threads=threads)["out"]
+

@@ -56,6 +56,7 @@ def test_reference_arm_prints_the_contract_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] >= 3 and d["value"] > 0
     assert d["config"]["workload"] == "decode_sweep_bf16"
+    assert d["config"] == bench.workload_config("decode_sweep_bf16", bench.DECODE_BATCHES, 1)  # our arm's config
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0

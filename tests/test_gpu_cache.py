@@ -7,7 +7,9 @@ to an all-resident layer over the same weights: the same kernels read the
 same bytes (vLLM-Moet, topairepos.com page, hybrid results table, row
 "identity"). A repeated batch finds every one of its experts in the cache and
 copies nothing; a batch that routes more host experts than there are slots
-takes the per-call staging path and still matches.
+takes the per-call staging path and still matches. Every call's output is
+also checked against the CPU oracle (max|err| <= 2e-2 * max|ref| for bf16,
+4e-2 for FP8), with the weights drawn and quantised on the host.
 """
 
 import numpy as np
@@ -16,6 +18,9 @@ import torch
 
 import oracle
 import synth
+from helpers import assert_close_out, oracle_layer_out
+
+TOL = {0: 2e-2, 1: 4e-2}
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +84,8 @@ def test_lru_cache_bit_identical_and_hits(wdtype):
         torch.cuda.synchronize()
         assert cache.status() == 0 and ref.status() == 0
         assert np.array_equal(oracle.as_u16(a), oracle.as_u16(b)), f"call {i} (T={T}) differs"
+        ref_o = oracle_layer_out(oracle.as_u16(x), wr.cpu().numpy(), None, K, E, H, I, seed=5, fp8=wdtype == 1)
+        assert_close_out(oracle.as_u16(b), ref_o, TOL[wdtype])
         st = cache.stats()
         assert st["last_routed_cold"] == st["last_touched"]  # every expert lives on the host
         if st["last_routed_cold"] <= N_SLOTS:

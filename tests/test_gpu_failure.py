@@ -40,3 +40,98 @@ def test_bounded_wait_times_out_and_the_context_stays_usable():
     with pytest.raises(M.MoeError):
         M.moe_debug_wait_flag(ctx, flag, 3_000_000_000)  # above the 2 s bound: refused on the host
     case.close()
+
+
+# --------------------------------------------------- unregistered expert --
+
+import numpy as np  # noqa: E402
+
+
+def _oracle_without(case, missing):
+    """Oracle output with every pair routed to `missing` dropped: each token's sum
+    runs over its other pairs, k ascending (the missing expert is every token's
+    top-1 here, so each token keeps K - 1 pairs)."""
+    xu, wr, bias = case.oracle_inputs()
+    _, idx, w = oracle.route(xu, wr, bias, case.K)
+    keep = idx != missing
+    assert np.all(keep.sum(axis=1) == case.K - 1)
+    pt = np.nonzero(keep)[0].astype(np.int32)  # row-major: token, then k ascending
+    pe = idx[keep]
+    pw = w[keep].astype(np.float32)
+    gu, dn, sgu, sdn = case.expert_arrays(np.unique(pe))
+    if case.q is None:
+        y = oracle.ffn_bf16(xu, pt, pe, pw, gu, dn, case.E)
+    else:
+        y = oracle.ffn_fp8(xu, pt, pe, pw, gu, sgu, dn, sdn, case.E)
+    return oracle.combine(y, np.arange(case.T * (case.K - 1), dtype=np.int32).reshape(case.T, case.K - 1))
+
+
+@pytest.mark.parametrize("T,wdtype,host", [(4, 0, False),     # decode: FFN planned inside the kernel
+                                           (100, 0, False),   # one-launch permutation + plan
+                                           (400, 0, False),   # rank/scan/scatter, then the plan kernel
+                                           (8, 1, False),     # FP8, one-launch FFN
+                                           (8, 0, True)])     # host-resident experts: host-side staging
+def test_unregistered_expert_is_flagged_and_dropped(T, wdtype, host):
+    """Routing to an expert that has no registered weights sets MOE_DEV_NO_SLOT
+    and drops those pairs: each token's output is the oracle's sum over its
+    other pairs. Registering the expert afterwards restores the full layer."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import mixture_experts_layer_24_b200 as M
+    H, E, K, I = 512, 16, 4, 256
+    missing = 5
+    hot = set(range(0, E, 2)) if host else None  # odd experts in pinned host memory
+    case = LayerCase(T, H, E, K, I, seed=40 + T, wdtype=wdtype, unregistered=(missing,), hot=hot,
+                     n_spare=8 if host else 0)
+    bias = torch.zeros(E, dtype=torch.float32)
+    bias[missing] = 64.0  # far above the logits' spread: every token's top-1
+    case.bias = bias.to(case.dev)
+    tol = 4e-2 if wdtype else 2e-2
+    out = case.forward()
+    torch.cuda.synchronize()
+    st = case.layer.status()
+    assert st & M.binding.MOE_DEV_NO_SLOT, st
+    assert not st & M.binding.MOE_DEV_TIMEOUT
+    assert_close_out(oracle.as_u16(out), _oracle_without(case, missing), tol)
+    # register it: the same context now runs the whole layer
+    g, d = case.w_gu[missing], case.w_dn[missing]
+    if case.q is None:
+        case.layer.register(missing, g, d)
+    else:
+        qg, sg, qd, sd = case.q[missing]
+        case.layer.register(missing, qg, qd, sg, sd)
+    out = case.forward()
+    torch.cuda.synchronize()
+    assert case.layer.status() == 0
+    assert_close_out(oracle.as_u16(out), case.oracle_forward()["out"], tol)
+    case.close()
+
+
+def test_unregistered_expert_rows_are_zero_in_expert_ffn():
+    """moe_expert_ffn on its own: the y_pair rows of pairs routed to an
+    unregistered expert are written as zeros (the others match the oracle)."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import mixture_experts_layer_24_b200 as M
+    H, E, K, I, T, missing = 512, 16, 4, 256, 300, 9
+    case = LayerCase(T, H, E, K, I, seed=77, unregistered=(missing,))
+    bias = torch.zeros(E, dtype=torch.float32)
+    bias[missing] = 64.0
+    case.bias = bias.to(case.dev)
+    idx, w = case.layer.route(case.x, case.wr, case.bias)
+    counts, offsets, ps, pk, inv = case.layer.permute(idx)
+    y = case.layer.expert_ffn(case.x, ps, pk, offsets, w)
+    torch.cuda.synchronize()
+    assert case.layer.status() & M.binding.MOE_DEV_NO_SLOT
+    off = offsets.cpu().numpy()
+    yn = y.cpu().numpy()
+    assert off[missing + 1] - off[missing] == T
+    assert not np.any(yn[off[missing]:off[missing + 1]])
+    # the other rows: the oracle's y for the same sorted pairs
+    ps_n, pk_n, idx_n, w_n = ps.cpu().numpy(), pk.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
+    rows = np.r_[0:off[missing], off[missing + 1]:off[E]]
+    pe = idx_n[ps_n[rows], pk_n[rows]]
+    gu, dn, _, _ = case.expert_arrays(np.unique(pe))
+    ref = oracle.ffn_bf16(oracle.as_u16(case.x), ps_n[rows], pe, w_n[ps_n[rows], pk_n[rows]], gu, dn, E)
+    assert np.max(np.abs(yn[rows] - ref)) <= 2e-2 * np.max(np.abs(ref))
+    case.close()

@@ -294,11 +294,18 @@ def test_empty_batch_is_a_no_op():
     case.close()
 
 
-def test_graph_replay_matches_eager():
+@pytest.mark.parametrize("T,wdtype", [(1, 0), (8, 0), (64, 0), (100, 0), (8, 1), (64, 1)])
+def test_graph_replay_matches_eager(T, wdtype):
     """A forward captured in a CUDA graph (kernels chained by programmatic
-    dependent launch) gives the eager bits, replay after replay."""
-    case = LayerCase(64, 512, 16, 4, 256, seed=12)
+    dependent launch) gives the eager bits, replay after replay, and the
+    oracle's output within tolerance. T = 1 .. 64 (bf16) are the decode
+    batches that run planned from the router's top-k in one FFN launch (the
+    launches bench.py replays); 100 tokens take the permutation and separate
+    GEMMs; FP8 8 tokens take the one-launch FP8 FFN, 64 the separate ones."""
+    case = LayerCase(T, 512, 16, 4, 256, seed=12, wdtype=wdtype)
+    tol = TOL_FP8 if wdtype else TOL_BF16
     ref = oracle.as_u16(case.forward())
+    assert_close_out(ref, case.oracle_forward()["out"], tol)
     g, out = case.layer.capture(case.x, case.wr, case.bias)
     for _ in range(3):
         out.zero_()
@@ -306,10 +313,12 @@ def test_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert np.array_equal(oracle.as_u16(out), ref)
     # new input contents, same buffer
-    case.x.copy_(synth.tokens(64, 512, seed=13, device="cuda"))
+    case.x.copy_(synth.tokens(T, 512, seed=13, device="cuda"))
     g.replay()
     torch.cuda.synchronize()
-    assert np.array_equal(oracle.as_u16(out), oracle.as_u16(case.forward()))
+    got = oracle.as_u16(out)
+    assert np.array_equal(got, oracle.as_u16(case.forward()))
+    assert_close_out(got, case.oracle_forward()["out"], tol)
     assert case.layer.status() == 0
     case.close()
 
