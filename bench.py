@@ -713,6 +713,80 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
     return out
 
 
+def run_ep(args):
+    """Expert parallelism (--ep): experts split by range over the N ranks (384/N
+    each), every rank routes its own tokens (the decode sweep, or a 4096-token
+    chunk) and the pairs travel to the experts' GPUs and back by NCCL
+    all-to-all (mixture_experts_layer_24_b200.ep). Per-rank work is fixed as N
+    grows ("weak"); value = tokens of all ranks / max rank time. Each forward
+    reads the per-expert counts on the host once (the all-to-all split sizes),
+    so it is not graph-captured."""
+    from mixture_experts_layer_24_b200 import build as B
+    from mixture_experts_layer_24_b200 import ep
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    if rank == 0:
+        B.build()
+    dist_barrier(world)
+    steps = ep.LibmoeSteps(H, E, K, I, rank, world, device=device)
+    keep = []
+    for e in range(steps.e0, steps.e0 + steps.E_loc):
+        g, d = synth.expert_weights(e, H, I, seed=SEED, device=device)
+        steps.register(e, g, d)
+        keep.append((g, d))
+    wr = synth.router_weight(E, H, seed=SEED, device=device)
+    bias = synth.zipf_logit_bias(E, ZIPF_S, seed=SEED).to(device)
+    comm = ep.TorchComm() if world > 1 else ep.LocalComm.group(1)[0]
+    batches, firsts = sweep_inputs(args.workload, rank)
+    xs = [synth.tokens(b, H, seed=SEED, device=device, first_token=f) for b, f in zip(batches, firsts)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    def one_pass():
+        ms = 0.0
+        for x in xs:
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            ep.ep_forward(steps, comm, x, wr, bias)
+            b.record()
+            b.synchronize()
+            ms += a.elapsed_time(b)
+        return ms
+
+    for _ in range(args.warmup):
+        one_pass()
+    if steps.status():
+        raise SystemExit("device status after warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    ms = sum(one_pass() for _ in range(args.steps))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist_barrier(world)
+    ms_max = dist_max(world, ms, device)
+    total_tokens = dist_sum(world, sum(batches) * args.steps, device)
+    workload = "decode_sweep_bf16" if args.workload == "decode" else "prefill4096_bf16"
+    cfg = workload_config(workload, batches, world)
+    cfg["parallelism"] = f"ep{world} (experts split by range, NCCL all-to-all of pairs)"
+    line = {"metric": METRIC, "value": total_tokens / (ms_max / 1000.0), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg, "clocks": clk}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    steps.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -723,6 +797,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
+    ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
     ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "r4096"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
@@ -732,6 +807,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.ep:
+        return run_ep(args)
     return run_ours(args)
 
 

@@ -161,6 +161,46 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* slots, const void* x, cons
                          const float* logit_bias, int T, void* out, void* ws, size_t ws_bytes,
                          moe_stream_t stream);
 
+/* ---- expert parallelism ------------------------------------------------
+ * Experts split into G contiguous ranges, one per GPU (GPU g holds experts
+ * [g*E/G, (g+1)*E/G)); every pair is computed on the GPU that holds its
+ * expert and its y_pair row comes back to the token's GPU, where the combine
+ * runs in the usual order. The pages split each expert across their GPUs and
+ * sum the slices over NCCL (vLLM-Moet, topairepos.com page, hybrid results
+ * table, row "the step"; model table, "one expert as its 576-row slices"); a
+ * cross-GPU sum would change the order of a token's additions, so here whole
+ * pairs move instead and a token's output bits do not depend on G. The
+ * exchange itself (two all-to-alls of rows, one of counts) is the caller's:
+ * NCCL through torch.distributed in the Python binding (ep.py).
+ *
+ * Token GPU, after moe_route and moe_permute (context with all E experts):
+ *   moe_ep_pack: x_send[p] = x[perm_src[p]] (bf16 [T*K, H]) and
+ *   w_send[p] = topk_w[perm_src[p], perm_k[p]] (fp32 [T*K]) for the valid
+ *   sorted pairs p < offsets[E]. Rows for GPU g are the range
+ *   offsets[g*E/G] .. offsets[(g+1)*E/G]. x, x_send 16-byte aligned. */
+moe_status_t moe_ep_pack(moe_ctx_t* ctx, const void* x, const float* topk_w, const int32_t* perm_src,
+                         const int32_t* perm_k, const int32_t* offsets, int T, void* x_send, float* w_send,
+                         moe_stream_t stream);
+
+/* Expert GPU (a context with its E_loc = E/G experts and top_k = 1): the
+ * received rows arrive grouped by source GPU (n_src of them) and, within a
+ * source, by local expert; recv_counts [n_src][E_loc] gives each group's rows.
+ * Writes the plan that sorts them by (local expert, source, arrival):
+ * offsets [E_loc+1], perm_src [R] (sorted place -> received row), perm_k [R]
+ * (zeros: each received row is one pair) and inv [R] (received row -> sorted
+ * place), R = the sum of recv_counts. Feed x_recv, perm_src, perm_k, offsets
+ * and w_recv (as topk_w [R, 1]) to moe_expert_ffn with T = R.
+ * n_src * E_loc <= 1024. */
+moe_status_t moe_ep_recv_plan(moe_ctx_t* ctx, const int32_t* recv_counts, int n_src, int32_t* offsets,
+                              int32_t* perm_src, int32_t* perm_k, int32_t* inv, moe_stream_t stream);
+
+/* fp32 row gather, dst[i, :] = src[idx[i], :] for i < n_rows, rows of H
+ * (the context's hidden size) floats: on the expert GPU, with idx = inv from
+ * moe_ep_recv_plan, it puts moe_expert_ffn's rows back in arrival order for
+ * the return all-to-all. src, dst 16-byte aligned. */
+moe_status_t moe_ep_gather_rows(moe_ctx_t* ctx, const float* src, const int32_t* idx, int n_rows, float* dst,
+                                moe_stream_t stream);
+
 /* FP8 block quantiser (used for weights with block_rows = 128 and for
  * activations with block_rows = 1): per block of block_rows x 128 elements,
  * s = amax / 448 (IEEE fp32 divide; 1 if the block is all zero) and

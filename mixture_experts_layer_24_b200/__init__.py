@@ -7,6 +7,8 @@ ABI in ``include/moe.h``); this package is argument marshalling only:
   wrappers that take torch tensors (PyTorch supplies device memory and
   streams, nothing else).
 * :mod:`.build`   -- nvcc build of ``libmoe.so`` in-tree.
+* :mod:`.ep`      -- the expert-parallel schedule over several GPUs (which
+  libmoe call comes when, and the NCCL all-to-alls between them).
 
 Importing the package does not load the library; the first call of a binding
 function does, and raises if ``libmoe.so`` is missing (there is no fallback).
@@ -26,6 +28,9 @@ from .binding import (  # noqa: F401
     moe_ctx_create,
     moe_ctx_destroy,
     moe_debug_wait_flag,
+    moe_ep_gather_rows,
+    moe_ep_pack,
+    moe_ep_recv_plan,
     moe_expert_ffn,
     moe_forward,
     moe_get_device_status,

@@ -34,7 +34,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy",
-           "moe_debug_wait_flag"]
+           "moe_debug_wait_flag", "moe_ep_pack", "moe_ep_recv_plan", "moe_ep_gather_rows"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
@@ -92,6 +92,9 @@ def lib():
         "moe_profile_read": ([P, I, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], S),
         "moe_route_noalloc": ([P, P, P, I, I, I, I, P, P, P], S),
         "moe_debug_wait_flag": ([P, P, ctypes.c_int64, P], S),
+        "moe_ep_pack": ([P, P, P, P, P, P, I, P, P, P], S),
+        "moe_ep_recv_plan": ([P, P, I, P, P, P, P, P], S),
+        "moe_ep_gather_rows": ([P, P, P, I, P, P], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -176,6 +179,20 @@ def moe_combine(ctx, y_pair, inv, T, out, stream=None):
 def moe_forward(ctx, slots, x, w_router, logit_bias, T, out, ws, stream=None):
     _check(lib().moe_forward(ctx, slots, _p(x), _p(w_router), _p(logit_bias), T, _p(out), _p(ws), _nbytes(ws),
                              _s(stream)), "moe_forward")
+
+
+def moe_ep_pack(ctx, x, topk_w, perm_src, perm_k, offsets, T, x_send, w_send, stream=None):
+    _check(lib().moe_ep_pack(ctx, _p(x), _p(topk_w), _p(perm_src), _p(perm_k), _p(offsets), T, _p(x_send),
+                             _p(w_send), _s(stream)), "moe_ep_pack")
+
+
+def moe_ep_recv_plan(ctx, recv_counts, n_src, offsets, perm_src, perm_k, inv, stream=None):
+    _check(lib().moe_ep_recv_plan(ctx, _p(recv_counts), n_src, _p(offsets), _p(perm_src), _p(perm_k), _p(inv),
+                                  _s(stream)), "moe_ep_recv_plan")
+
+
+def moe_ep_gather_rows(ctx, src, idx, n_rows, dst, stream=None):
+    _check(lib().moe_ep_gather_rows(ctx, _p(src), _p(idx), n_rows, _p(dst), _s(stream)), "moe_ep_gather_rows")
 
 
 def moe_quantize_e4m3(src, rows, cols, block_rows, q, scales, stream=None):

@@ -1013,6 +1013,54 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
   return MOE_OK;
 }
 
+// ---------------------------------------------------- expert parallelism --
+
+moe_status_t moe_ep_pack(moe_ctx_t* ctx, const void* x, const float* topk_w, const int32_t* perm_src,
+                         const int32_t* perm_k, const int32_t* offsets, int T, void* x_send, float* w_send,
+                         moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  moe_status_t st = check_T(ctx, T);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!x || !topk_w || !perm_src || !perm_k || !offsets || !x_send || !w_send)
+    return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(x_send)) % 16)
+    return fail(MOE_ERR_INVALID_ARG, "x and x_send must be 16-byte aligned");
+  const moe_config_t& c = ctx->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Prof p(ctx, MOE_PROF_GATHER, s);
+  MOE_CUDA(launch_ep_pack(x, topk_w, perm_src, perm_k, offsets, c.n_experts, c.top_k, T * c.top_k, c.hidden, x_send,
+                          w_send, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_recv_plan(moe_ctx_t* ctx, const int32_t* recv_counts, int n_src, int32_t* offsets,
+                              int32_t* perm_src, int32_t* perm_k, int32_t* inv, moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  if (!recv_counts || !offsets || !perm_src || !perm_k || !inv) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if (n_src <= 0) return fail(MOE_ERR_INVALID_ARG, "n_src must be positive");
+  if ((long long)n_src * ctx->cfg.n_experts > 1024)
+    return fail(MOE_ERR_UNSUPPORTED, "n_src * E must be <= 1024 (E = this context's experts)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Prof p(ctx, MOE_PROF_PERMUTE, s);
+  MOE_CUDA(launch_ep_recv_plan(recv_counts, n_src, ctx->cfg.n_experts, offsets, perm_src, perm_k, inv, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_gather_rows(moe_ctx_t* ctx, const float* src, const int32_t* idx, int n_rows, float* dst,
+                                moe_stream_t stream) {
+  if (!ctx) return fail(MOE_ERR_INVALID_ARG, "NULL context");
+  if (n_rows < 0) return fail(MOE_ERR_INVALID_ARG, "n_rows must be >= 0");
+  if (n_rows == 0) return MOE_OK;
+  if (!src || !idx || !dst) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % 16)
+    return fail(MOE_ERR_INVALID_ARG, "src and dst must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Prof p(ctx, MOE_PROF_GATHER, s);
+  MOE_CUDA(launch_ep_gather_rows_f32(src, idx, n_rows, ctx->cfg.hidden, dst, s));
+  return MOE_OK;
+}
+
 moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                                moe_stream_t stream) {
   if (rows < 0 || cols <= 0 || cols % 128) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0 and cols % 128 == 0");

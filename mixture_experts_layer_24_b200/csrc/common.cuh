@@ -238,6 +238,36 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
 }
 
+// ---------------------------------------------------------------- scan --
+// Exclusive scan of up to 1024 values held one per thread (blockDim = 1024).
+__device__ inline int block_exclusive_scan_1024(int v, int* sh /* >= 32 ints */, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) sh[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int s = sh[lane];
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += n;
+    }
+    sh[lane] = si - s;  // exclusive prefix of warp totals
+    if (lane == 31) sh[32] = si;
+  }
+  __syncthreads();
+  const int res = sh[w] + incl - v;
+  *total = sh[32];
+  __syncthreads();
+  return res;
+}
+
 // ---------------------------------------------------------------- misc --
 
 __device__ __forceinline__ void flag_status(int* status, int bit) {

@@ -199,6 +199,17 @@ cudaError_t launch_combine(const float* y, const int32_t* inv, int T, int K, int
                            bool pdl);
 cudaError_t launch_quant_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                               cudaStream_t s);
+// Expert parallelism (ep.cu): rows in sorted order for the all-to-all, the
+// plan of the rows an expert GPU receives, and the fp32 row gather that puts
+// results back in arrival order.
+cudaError_t launch_ep_pack(const void* x, const float* topk_w, const int32_t* perm_src, const int32_t* perm_k,
+                           const int32_t* offsets, int E, int K, int P, int H, void* x_send, float* w_send,
+                           cudaStream_t s);
+cudaError_t launch_ep_recv_plan(const int32_t* recv_counts, int G, int E_loc, int32_t* offsets_loc, int32_t* perm,
+                                int32_t* perm_k, int32_t* inv, cudaStream_t s);
+cudaError_t launch_ep_gather_rows_f32(const float* src, const int32_t* idx, int n_rows, int H, float* dst,
+                                      cudaStream_t s);
+
 // Sets the text moe_last_error() returns on this thread.
 void record_error(const char* msg);
 

@@ -78,35 +78,6 @@ cudaError_t launch_permute_rank(const int32_t* idx, int T, int K, int E, int chu
                    rank, chunk_counts, status);
 }
 
-// Exclusive scan of up to 1024 values held one per thread (blockDim = 1024).
-__device__ int block_exclusive_scan_1024(int v, int* sh /* >= 32 ints */, int* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += n;
-  }
-  if (lane == 31) sh[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    int s = sh[lane];
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int n = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += n;
-    }
-    sh[lane] = si - s;  // exclusive prefix of warp totals
-    if (lane == 31) sh[32] = si;
-  }
-  __syncthreads();
-  const int res = sh[w] + incl - v;
-  *total = sh[32];
-  __syncthreads();
-  return res;
-}
-
 __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ chunk_counts, int n_chunks,
                                                              int E, int32_t* __restrict__ counts,
                                                              int32_t* __restrict__ offsets) {

@@ -5,9 +5,9 @@ in the launch configuration bench.py times.
 - Outputs: checked on a seeded sample of tokens against the oracle (a token's
   output depends on that token alone, which the invariance tests check).
 - Batch invariance across the decode/prefill tile-width switch.
-- Hot/cold residency: bit-identical to the all-resident run, over a chain of
-  layers (vLLM-Moet page, hybrid results table, row "identity": calls, rows,
-  0 differ).
+- Hot/cold residency: bit-identical to the all-resident run over 8 layers
+  (vLLM-Moet page, hybrid results table, row "identity": calls, rows,
+  0 differ), and the oracle on sampled tokens.
 - FP8 block-scaled experts at full size.
 """
 
@@ -155,31 +155,32 @@ def test_batch_invariance_across_tile_widths(full_bf16):
 
 
 def test_hot_cold_bit_identical_to_all_resident():
-    """The hot/cold configuration as stated: 8 chained layers (layer l has its
-    own seed), each with 120 hot experts picked greedily from a seeded routing
-    histogram and the other 264 in pinned host memory behind 32 spare slots;
-    decode B=1, B=4 and a 4096-token prefill chunk. Each layer's output feeds
-    the next. Checked, at every layer:
+    """The hot/cold configuration as stated: 8 layers (layer l has its own
+    seed: router, Zipf prior, experts and input tokens), each with 120 hot
+    experts picked greedily from a seeded routing histogram and the other 264
+    in pinned host memory behind 32 spare slots; decode B=1, B=4 and a
+    4096-token prefill chunk per layer. Layer inputs are seeded N(0,1) tokens
+    rather than the previous layer's raw output: without the residual and norm
+    of a real model between them, chained layers shrink the activations by
+    orders of magnitude per layer. Checked, at every layer:
       - bit identity with the all-resident layer (vLLM-Moet page, hybrid results
         table, row "identity": calls, rows, 0 differ);
       - batch invariance: the B=1 and B=4 tokens are the first tokens of the
         4096 chunk and give the same bits there;
-      - the oracle, on sampled tokens carried through the same 8 layers on the
-        CPU (the oracle's own outputs feed its next layer), within 2e-2.
+      - the oracle, on sampled tokens, within 2e-2.
     One layer's host store (13.3 GB pinned) exists at a time."""
     _need_cuda()
     import mixture_experts_layer_24_b200 as M
     from helpers import oracle_layer_out
     dev = torch.device("cuda")
     n_layers, n_hot, n_spare = 8, 120, 32
-    xb = synth.tokens(4096, H, seed=3, device=dev, first_token=90000)
-    inputs = {1: xb[:1].contiguous(), 4: xb[:4].contiguous(), 4096: xb}
     sample = np.array([0, 3, 1000, 4095])
-    ora = oracle.as_u16(xb)[sample]  # the oracle's own chain of sampled tokens
     calls = rows = differ = 0
     cold_total = 0
     for layer_i in range(n_layers):
         seed = 10 + layer_i
+        xb = synth.tokens(4096, H, seed=seed, device=dev, first_token=90000)
+        inputs = {1: xb[:1].contiguous(), 4: xb[:4].contiguous(), 4096: xb}
         full = FullLayer(seed=seed)
         # seeded routing histogram -> hot set
         hx = synth.tokens(2048, H, seed=seed, device=dev, first_token=700000)
@@ -207,12 +208,12 @@ def test_hot_cold_bit_identical_to_all_resident():
         o4096 = oracle.as_u16(outs[4096])
         assert np.array_equal(oracle.as_u16(outs[1]), o4096[:1]), f"layer {layer_i}: B=1 differs from the chunk"
         assert np.array_equal(oracle.as_u16(outs[4]), o4096[:4]), f"layer {layer_i}: B=4 differs from the chunk"
-        ora = oracle_layer_out(ora, full.wr.cpu().numpy(), full.bias.cpu().numpy(), K, E, H, I, seed)
+        ora = oracle_layer_out(oracle.as_u16(xb)[sample], full.wr.cpu().numpy(), full.bias.cpu().numpy(), K, E, H,
+                               I, seed)
         assert_close_out(o4096[sample], ora, TOL_BF16)
         split.close()
         full.close()
-        inputs = {T: outs[T] for T in inputs}  # chain: this layer's output feeds the next
-        del store, ref
+        del store, ref, outs, inputs, xb
         torch.cuda.empty_cache()
     assert cold_total > 0, "no cold expert was exercised"
     assert calls == 3 * n_layers
