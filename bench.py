@@ -485,6 +485,7 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep):
 
     if args.workload == "decode" and not args.quick:
         br.update(fp8_breakdown(keep, wr, bias, flush, stream, device, hbm))
+        br.update(fp4_breakdown(keep, wr, bias, flush, stream, device, hbm))
         br.update(hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm))
 
     # --- end to end through the public API, host buffers ---
@@ -609,6 +610,46 @@ def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
             "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
     if layer.status():
         out["fp8_device_status"] = layer.status()
+    layer.close()
+    del qkeep
+    torch.cuda.empty_cache()
+    return out
+
+
+def fp4_breakdown(keep, wr, bias, flush, stream, device, hbm):
+    """The same layer with MXFP4 experts (E2M1 codes and E8M0 scales per 32
+    elements, quantised on the GPU from the bf16 weights by the MX quantiser):
+    decode B=1, 8, 64 and a 4096-token chunk. Bytes per touched expert: the
+    packed codes (3 I H / 2) and the scale bytes (3 I H / 32)."""
+    import mixture_experts_layer_24_b200 as M
+    layer = M.MoeLayer(H, E, K, I, wdtype=M.MOE_MXFP4, device=device)
+    qkeep = []
+    for e in range(E):
+        g, d = keep[e]
+        qg = torch.empty((2 * I, H // 2), dtype=torch.uint8, device=device)
+        sg = torch.empty((2 * I, H // 32), dtype=torch.uint8, device=device)
+        qd = torch.empty((H, I // 2), dtype=torch.uint8, device=device)
+        sd = torch.empty((H, I // 32), dtype=torch.uint8, device=device)
+        M.moe_quantize_mx(g, 2 * I, H, 0, qg, sg)
+        M.moe_quantize_mx(d, H, I, 0, qd, sd)
+        layer.register(e, qg, qd, sg, sd)
+        qkeep.append((qg, qd, sg, sd))
+    torch.cuda.synchronize()
+    layer.workspace(4096)
+    fp4_bytes = 3 * I * H // 2 + 3 * I * H // 32
+    out = {}
+    for T in (1, 8, 64, 4096):
+        x = synth.tokens(T, H, seed=SEED, device=device, first_token=600000)
+        time_forwards(layer, [x], wr, bias, flush, stream, 2)
+        reps = 5 if T < 4096 else 3
+        ms = time_forwards(layer, [x], wr, bias, flush, stream, reps) / reps
+        t = touched_experts(layer, x, wr, bias)
+        nbytes = t * fp4_bytes + E * H * 4 + T * H * 4
+        out[f"fp4_B{T}" if T < 4096 else "fp4_prefill4096"] = {
+            "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
+            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+    if layer.status():
+        out["fp4_device_status"] = layer.status()
     layer.close()
     del qkeep
     torch.cuda.empty_cache()

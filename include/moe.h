@@ -73,8 +73,17 @@ typedef enum {
 
 typedef enum {
   MOE_BF16 = 0,          /* bf16 expert weights */
-  MOE_FP8_E4M3_B128 = 1  /* e4m3 expert weights with fp32 scales per 128x128 block;
+  MOE_FP8_E4M3_B128 = 1, /* e4m3 expert weights with fp32 scales per 128x128 block;
                             activations quantised to e4m3 per token per 128 columns */
+  MOE_MXFP4 = 2          /* OCP MXFP4 expert weights: E2M1 codes packed two per byte
+                            (element 2i in the low nibble) with one E8M0 scale byte
+                            per 32 elements along K; activations and h quantised to
+                            MX e4m3 (per token per 32 columns) inside the layer; the
+                            tensor cores apply both scales (kind::mxf8f6f4.block_scale).
+                            The pages' checkpoint ships FP4 experts (vLLM-Moet,
+                            topairepos.com page, hybrid results table, row "quality,
+                            paired against the native FP4 reference"); they name no
+                            block format, and this is the open one. HBM-resident only. */
 } moe_wdtype_t;
 
 enum { MOE_LOC_HBM = 0, MOE_LOC_HOST_PINNED = 1 };
@@ -210,6 +219,17 @@ moe_status_t moe_ep_gather_rows(moe_ctx_t* ctx, const float* src, const int32_t*
 moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_rows, uint8_t* q, float* scales,
                                moe_stream_t stream);
 
+/* MX quantiser (OCP Microscaling; the MXFP4 path's weights and activations):
+ * per 32 consecutive elements of a row, X = 2^(floor(log2 amax) - emax)
+ * (emax 2 for E2M1, 8 for E4M3; clamped to 2^-127 .. 2^127, 2^-127 for an
+ * all-zero block) and q = encode(v / X), round to nearest even, saturating.
+ *   src [rows, cols] bf16, cols % 32 == 0 (16-byte aligned rows);
+ *   elem 0 (E2M1): q [rows, cols/2] packed, element 2i in the low nibble;
+ *   elem 1 (E4M3): q [rows, cols];
+ *   scales [rows, cols/32] E8M0 bytes (exponent + 127). Bit-exact. */
+moe_status_t moe_quantize_mx(const void* src, int rows, int cols, int elem, uint8_t* q, uint8_t* scales,
+                             moe_stream_t stream);
+
 /* moe_route_noalloc -- the router (logits, top-k, weights; same kernels, same
  * order and results as moe_route) for callers that cannot allocate device
  * memory: engines that reserve HBM up front and hand it out only through
@@ -247,9 +267,13 @@ moe_status_t moe_slots_destroy(moe_slots_t* slots);
  * cudaHostRegister), borrowed and kept pinned by the caller.
  * bf16: w_gu [2I, H], w_dn [H, I] bf16; s_gu, s_dn must be NULL.
  * FP8: w_gu [2I, H], w_dn [H, I] e4m3; s_gu [2I/128, H/128], s_dn [H/128, I/128] fp32.
+ * MXFP4 (HBM only): w_gu [2I, H/2], w_dn [H, I/2] packed E2M1 bytes, 32-byte
+ * aligned; s_gu [2I, H/32], s_dn [H, I/32] E8M0 bytes (uint8). The table
+ * copies the scales into the tensor cores' block layout (memory it owns);
+ * the codes are borrowed.
  * Device pointers must be 16-byte aligned. Synchronous. */
 moe_status_t moe_slots_register(moe_slots_t* slots, int expert, const void* w_gu, const void* w_dn,
-                                const float* s_gu, const float* s_dn, int location);
+                                const void* s_gu, const void* s_dn, int location);
 
 /* Reports where `expert` lives: *location = MOE_LOC_* or -1 if unregistered;
  * *slot = its resident index, or -1 for host-resident experts. */

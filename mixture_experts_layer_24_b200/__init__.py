@@ -17,6 +17,7 @@ function does, and raises if ``libmoe.so`` is missing (there is no fallback).
 from .binding import (  # noqa: F401
     MOE_BF16,
     MOE_FP8_E4M3_B128,
+    MOE_MXFP4,
     MOE_LOC_HBM,
     MOE_LOC_HOST_PINNED,
     MOE_SLOTS_LRU,
@@ -40,6 +41,7 @@ from .binding import (  # noqa: F401
     moe_profile_enable,
     moe_profile_read,
     moe_quantize_e4m3,
+    moe_quantize_mx,
     moe_route,
     moe_route_noalloc,
     moe_slots_create,

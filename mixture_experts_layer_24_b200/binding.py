@@ -18,6 +18,7 @@ _LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_BF16 = 0
 MOE_FP8_E4M3_B128 = 1
+MOE_MXFP4 = 2
 MOE_LOC_HBM = 0
 MOE_LOC_HOST_PINNED = 1
 MOE_SLOTS_LRU = 0
@@ -34,7 +35,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy",
-           "moe_debug_wait_flag", "moe_ep_pack", "moe_ep_recv_plan", "moe_ep_gather_rows"]
+           "moe_debug_wait_flag", "moe_ep_pack", "moe_ep_recv_plan", "moe_ep_gather_rows", "moe_quantize_mx"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
@@ -95,6 +96,7 @@ def lib():
         "moe_ep_pack": ([P, P, P, P, P, P, I, P, P, P], S),
         "moe_ep_recv_plan": ([P, P, I, P, P, P, P, P], S),
         "moe_ep_gather_rows": ([P, P, P, I, P, P], S),
+        "moe_quantize_mx": ([P, I, I, I, P, P, P], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -198,6 +200,11 @@ def moe_ep_gather_rows(ctx, src, idx, n_rows, dst, stream=None):
 def moe_quantize_e4m3(src, rows, cols, block_rows, q, scales, stream=None):
     _check(lib().moe_quantize_e4m3(_p(src), rows, cols, block_rows, _p(q), _p(scales), _s(stream)),
            "moe_quantize_e4m3")
+
+
+def moe_quantize_mx(src, rows, cols, elem, q, scales, stream=None):
+    """MX quantiser: elem 0 = E2M1 (q packed two per byte), 1 = E4M3; E8M0 scales per 32 elements."""
+    _check(lib().moe_quantize_mx(_p(src), rows, cols, elem, _p(q), _p(scales), _s(stream)), "moe_quantize_mx")
 
 
 def moe_slots_create(ctx, n_spare_slots: int):
@@ -327,7 +334,12 @@ class MoeLayer:
         else:
             raise ValueError(f"unknown location {location}")
         H, I = self.H, self.I
-        if self.wdtype == MOE_FP8_E4M3_B128:
+        if self.wdtype == MOE_MXFP4:
+            check_tensor(w_gu, "w_gu", torch.uint8, (2 * I, H // 2), dev, pinned)
+            check_tensor(w_dn, "w_dn", torch.uint8, (H, I // 2), dev, pinned)
+            check_tensor(s_gu, "s_gu", torch.uint8, (2 * I, H // 32), dev, pinned)
+            check_tensor(s_dn, "s_dn", torch.uint8, (H, I // 32), dev, pinned)
+        elif self.wdtype == MOE_FP8_E4M3_B128:
             check_tensor(w_gu, "w_gu", torch.uint8, (2 * I, H), dev, pinned)
             check_tensor(w_dn, "w_dn", torch.uint8, (H, I), dev, pinned)
             check_tensor(s_gu, "s_gu", torch.float32, (2 * I // 128, H // 128), dev, pinned)

@@ -154,6 +154,7 @@ struct moe_slots {
   int64_t tick = 0;
   cudaEvent_t ev_done = nullptr;    // after the most recent call's GEMMs (they may read the slots)
   bool ev_done_valid = false;
+  std::vector<uint8_t*> sf_blk;     // [E] MXFP4: the expert's E8M0 scales in the block layout (owned here)
   std::mutex mu;
 };
 
@@ -164,12 +165,16 @@ namespace {
 struct WsLayout {
   size_t logits, rank, chunk_counts, topk_idx, topk_w, counts, offsets, perm_src, perm_k, inv;
   size_t list_expert, list_map, nt_prefix, sched, x_perm, x_scale, h, hq, h_scale, y_pair, total;
+  size_t x_sfb, h_sfb;  // MXFP4: activation scales in the tensor cores' block layout, per N tile
 };
 
 WsLayout ws_layout(const moe_config_t& c, int T) {
   WsLayout L{};
   const size_t P = (size_t)T * c.top_k, E = c.n_experts, H = c.hidden, I = c.intermediate;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
+  const bool mx = c.wdtype == MOE_MXFP4;
+  const size_t bn = (size_t)ffn_block_n(T, c.wdtype);
+  const size_t n_tiles = (P + bn - 1) / bn + std::min(E, P);  // N tiles of a plan, at most
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -190,11 +195,13 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
   L.list_map = take((2 * E + 64) * 4);
   L.nt_prefix = take((2 * E + 64) * 4);
   L.sched = take((size_t)fused_sched_entries((int)E) * 4);
-  L.x_perm = take(P * H * (fp8 ? 1 : 2));
+  L.x_perm = take(P * H * ((fp8 || mx) ? 1 : 2));
   L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
-  L.h = take(P * I * 2);
-  L.hq = take(fp8 ? P * I : 0);
+  L.h = take(mx ? 0 : P * I * 2);
+  L.hq = take((fp8 || mx) ? P * I : 0);
   L.h_scale = take(fp8 ? P * (I / 128) * 4 : 0);
+  L.x_sfb = take(mx ? n_tiles * (H / 128) * 512 : 0);
+  L.h_sfb = take(mx ? n_tiles * (I / 128) * 512 : 0);
   L.y_pair = take(P * H * 4);
   L.total = o;
   return L;
@@ -203,7 +210,8 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
 moe_status_t check_cfg(const moe_config_t& c) {
   if (c.hidden <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.intermediate <= 0)
     return fail(MOE_ERR_INVALID_ARG, "config sizes must be positive");
-  if (c.wdtype != MOE_BF16 && c.wdtype != MOE_FP8_E4M3_B128) return fail(MOE_ERR_INVALID_ARG, "unknown wdtype");
+  if (c.wdtype != MOE_BF16 && c.wdtype != MOE_FP8_E4M3_B128 && c.wdtype != MOE_MXFP4)
+    return fail(MOE_ERR_INVALID_ARG, "unknown wdtype");
   if (c.flags & ~MOE_FLAG_NO_PDL) return fail(MOE_ERR_INVALID_ARG, "unknown flag bits");
   if (c.hidden % 128 || c.intermediate % 128) return fail(MOE_ERR_UNSUPPORTED, "H and I must be multiples of 128");
   if (c.hidden > 8192 || c.intermediate > 8192) return fail(MOE_ERR_UNSUPPORTED, "H and I must be <= 8192");
@@ -261,11 +269,34 @@ moe_status_t encode_3d_bf16(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uin
   return MOE_OK;
 }
 
+// Packed E2M1 codes [rows, inner] (two per byte), box {128 elements, 128 rows}:
+// the copy lands unpacked (16 codes per 16 bytes) with the 128-byte swizzle.
+moe_status_t encode_2d_fp4(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner / 2};
+  const cuuint32_t box[2] = {128u, 128u};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(ptr), dims, strides,
+                                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (E2M1) failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
 moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void* dn, const float* sgu,
                         const float* sdn) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   std::memset(me, 0, sizeof(*me));
+  if (c.wdtype == MOE_MXFP4) {  // sgu / sdn: the blocked E8M0 scales
+    moe_status_t st = encode_2d_fp4(ctx, &me->gu, gu, c.hidden, 2ull * c.intermediate);
+    if (st != MOE_OK) return st;
+    st = encode_2d_fp4(ctx, &me->dn, dn, c.intermediate, c.hidden);
+    if (st != MOE_OK) return st;
+    me->s_gu = sgu;
+    me->s_dn = sdn;
+    return MOE_OK;
+  }
   if (!fp8) {
     for (int kc = 1; kc <= 2; ++kc) {
       moe_status_t st = encode_3d_bf16(ctx, kc == 1 ? &me->gu : &me->gu2, gu, c.hidden, 2ull * c.intermediate, 128, kc);
@@ -295,6 +326,49 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
+  if (c.wdtype == MOE_MXFP4) {
+    // both GEMMs on the block-scaled tensor cores; gate/up writes h as MX e4m3 codes and blocked scales
+    ActMaps xm, hm;
+    std::memset(&xm, 0, sizeof(xm));
+    std::memset(&hm, 0, sizeof(hm));
+    for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
+      moe_status_t st = encode_2d(ctx, &xm.m[i], at<void>(ws, W.x_perm), true, c.hidden, P, rows);
+      if (st != MOE_OK) return st;
+      st = encode_2d(ctx, &hm.m[i], at<void>(ws, W.hq), true, c.intermediate, P, rows);
+      if (st != MOE_OK) return st;
+    }
+    GemmArgs a{};
+    a.maps = sl->d_maps;
+    a.list_expert = list_expert;
+    a.list_map = list_map;
+    a.nt_prefix = nt_prefix;
+    a.offsets = offsets;
+    a.L = L;
+    a.H = c.hidden;
+    a.I = c.intermediate;
+    a.K = c.top_k;
+    a.h_out = at<void>(ws, W.hq);
+    a.h_sfb = at<uint8_t>(ws, W.h_sfb);
+    a.act_sfb = at<uint8_t>(ws, W.x_sfb);
+    a.y_out = y_pair;
+    a.topk_w = topk_w;
+    a.perm_src = perm_src;
+    a.perm_k = perm_k;
+    a.status = ctx->d_status;
+    a.plan_ready = (pdl && plan_ready_gu) ? 1 : 0;
+    a.num_sms = ctx->num_sms;
+    {
+      Prof p(ctx, MOE_PROF_GATE_UP, s);
+      MOE_CUDA(launch_ffn_mxfp4(kGateUp, bn, xm, a, (c.intermediate / 128) * max_ntiles, s, pdl));
+    }
+    a.act_sfb = at<uint8_t>(ws, W.h_sfb);
+    a.plan_ready = pdl ? 1 : 0;  // the plan is at least two launches back from the down GEMM
+    {
+      Prof p(ctx, MOE_PROF_DOWN, s);
+      MOE_CUDA(launch_ffn_mxfp4(kDown, bn, hm, a, (c.hidden / 128) * max_ntiles, s, pdl));
+    }
+    return MOE_OK;
+  }
   CUtensorMap xmap, hmap;
   ActMaps xmaps, hmaps;  // one activation map per tile box height 16 .. bn
   std::memset(&xmaps, 0, sizeof(xmaps));
@@ -687,6 +761,23 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   // pairs routed to an expert with no registered weights: zero rows, and inv = -1 in the forward
   const DropArgs drop{perm_src, perm_k, c.top_k, const_cast<int32_t*>(inv), y_pair, c.hidden};
 
+  if (sl->n_host == 0 && c.wdtype == MOE_MXFP4) {
+    sl->stats.last_cold = 0;
+    sl->stats.last_touched = -1;
+    if (!planned) {
+      Prof p(ctx, MOE_PROF_PERMUTE, s);
+      MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl,
+                               at<int>(ws, W.sched), fused_sched_entries(E), drop));
+    }
+    {
+      // MX e4m3 activation rows in sorted-pair order, scales in the block layout of their N tile
+      Prof pg(ctx, MOE_PROF_GATHER, s);
+      MOE_CUDA(launch_quant_mx_pairs(x, perm_src, offsets, np, E, bn, P, c.hidden, at<uint8_t>(ws, W.x_perm),
+                                     at<uint8_t>(ws, W.x_sfb), s, planned ? pdl : ctx->chain));
+    }
+    return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
+                     s, ctx->chain, planned ? pdl : true);
+  }
   if (sl->n_host == 0) {
     sl->stats.last_cold = 0;
     sl->stats.last_touched = -1;
@@ -1004,7 +1095,7 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
   bool planned = false;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   if ((st = permute_impl(ctx, idx, T, counts, offsets, ps, pk, inv, ws, s, chain, resident ? sl->d_map_of : nullptr,
-                         ffn_block_n(T, c.wdtype), x, (resident && !fp8) ? at<void>(ws, W.x_perm) : nullptr,
+                         ffn_block_n(T, c.wdtype), x, (resident && c.wdtype == MOE_BF16) ? at<void>(ws, W.x_perm) : nullptr,
                          &planned)) != MOE_OK)
     return st;
   if ((st = ffn_impl(ctx, sl, x, ps, pk, offsets, w, T, y, ws, s, chain, planned, inv)) != MOE_OK) return st;
@@ -1071,11 +1162,25 @@ moe_status_t moe_quantize_e4m3(const void* src, int rows, int cols, int block_ro
   return MOE_OK;
 }
 
+moe_status_t moe_quantize_mx(const void* src, int rows, int cols, int elem, uint8_t* q, uint8_t* scales,
+                             moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0 and cols % 32 == 0");
+  if (elem != 0 && elem != 1) return fail(MOE_ERR_INVALID_ARG, "elem must be 0 (E2M1) or 1 (E4M3)");
+  if (rows == 0) return MOE_OK;
+  if (!src || !q || !scales) return fail(MOE_ERR_INVALID_ARG, "NULL tensor");
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(q)) % 16)
+    return fail(MOE_ERR_INVALID_ARG, "src and q must be 16-byte aligned");
+  MOE_CUDA(launch_quant_mx(src, rows, cols, elem, q, scales, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
 // ----------------------------------------------------------------- slots --
 
 moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
   if (!out || !ctx || n_spare < 0) return fail(MOE_ERR_INVALID_ARG, "bad argument");
   *out = nullptr;
+  if (ctx->cfg.wdtype == MOE_MXFP4 && n_spare > 0)
+    return fail(MOE_ERR_UNSUPPORTED, "MXFP4 experts are HBM-resident only (no spare slots)");
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   moe_slots_t* sl = new moe_slots_t();
@@ -1087,6 +1192,7 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
   sl->dn.assign(sl->E, nullptr);
   sl->sgu.assign(sl->E, nullptr);
   sl->sdn.assign(sl->E, nullptr);
+  sl->sf_blk.assign(sl->E, nullptr);
   sl->h_maps.assign(sl->E + n_spare, MapEntry{});
   sl->h_map_of.assign(sl->E, -1);
   const size_t esz = fp8 ? 1 : 2;
@@ -1154,23 +1260,50 @@ moe_status_t moe_slots_destroy(moe_slots_t* sl) {
   if (sl->spare) cudaFree(sl->spare);
   if (sl->d_maps) cudaFree(sl->d_maps);
   if (sl->d_map_of) cudaFree(sl->d_map_of);
+  for (uint8_t* b : sl->sf_blk)
+    if (b) cudaFree(b);
   delete sl;
   return MOE_OK;
 }
 
-moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, const void* w_dn, const float* s_gu,
-                                const float* s_dn, int location) {
+moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, const void* w_dn, const void* s_gu_,
+                                const void* s_dn_, int location) {
   if (!sl) return fail(MOE_ERR_INVALID_ARG, "NULL slot table");
   if (expert < 0 || expert >= sl->E) return fail(MOE_ERR_SLOT, "expert index out of range");
   if (!w_gu || !w_dn) return fail(MOE_ERR_INVALID_ARG, "NULL weights");
-  const bool fp8 = sl->ctx->cfg.wdtype == MOE_FP8_E4M3_B128;
-  if (fp8 != (s_gu != nullptr) || fp8 != (s_dn != nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "scales must be given for FP8 weights and only for them");
+  const moe_config_t& c = sl->ctx->cfg;
+  const bool scaled = c.wdtype != MOE_BF16;
+  if (scaled != (s_gu_ != nullptr) || scaled != (s_dn_ != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "scales must be given for FP8 and MXFP4 weights and only for them");
   if (location != MOE_LOC_HBM && location != MOE_LOC_HOST_PINNED) return fail(MOE_ERR_INVALID_ARG, "bad location");
+  if (c.wdtype == MOE_MXFP4 && location != MOE_LOC_HBM)
+    return fail(MOE_ERR_UNSUPPORTED, "MXFP4 experts are HBM-resident only");
+  const float* s_gu = static_cast<const float*>(s_gu_);
+  const float* s_dn = static_cast<const float*>(s_dn_);
   std::lock_guard<std::mutex> lock(sl->mu);
   if (location == MOE_LOC_HBM) {
-    if ((reinterpret_cast<uintptr_t>(w_gu) | reinterpret_cast<uintptr_t>(w_dn)) % 16)
-      return fail(MOE_ERR_INVALID_ARG, "device weights must be 16-byte aligned");
+    const uintptr_t align = c.wdtype == MOE_MXFP4 ? 32 : 16;  // packed E2M1 tensor maps need 32-byte bases
+    if ((reinterpret_cast<uintptr_t>(w_gu) | reinterpret_cast<uintptr_t>(w_dn)) % align)
+      return fail(MOE_ERR_INVALID_ARG, c.wdtype == MOE_MXFP4 ? "MXFP4 weights must be 32-byte aligned"
+                                                             : "device weights must be 16-byte aligned");
+    if (c.wdtype == MOE_MXFP4) {
+      // the scales, rearranged once into the block layout the tensor cores read (owned by the table)
+      const int H = c.hidden, I = c.intermediate;
+      const size_t gu_blk = (size_t)(2 * I / 128) * (H / 128) * 512, dn_blk = (size_t)(H / 128) * (I / 128) * 512;
+      uint8_t* blk = nullptr;
+      if (cudaMalloc(&blk, gu_blk + dn_blk) != cudaSuccess) return fail(MOE_ERR_OOM, "cudaMalloc of MXFP4 scales failed");
+      cudaError_t err = launch_mx_block_scales(static_cast<const uint8_t*>(s_gu_), 2 * I, H, blk, nullptr);
+      if (err == cudaSuccess) err = launch_mx_block_scales(static_cast<const uint8_t*>(s_dn_), H, I, blk + gu_blk, nullptr);
+      if (err == cudaSuccess) err = cudaStreamSynchronize(nullptr);
+      if (err != cudaSuccess) {
+        cudaFree(blk);
+        return fail(MOE_ERR_CUDA, std::string("MXFP4 scale layout: ") + cudaGetErrorString(err));
+      }
+      if (sl->sf_blk[expert]) cudaFree(sl->sf_blk[expert]);
+      sl->sf_blk[expert] = blk;
+      s_gu = reinterpret_cast<const float*>(blk);
+      s_dn = reinterpret_cast<const float*>(blk + gu_blk);
+    }
     MapEntry me;
     moe_status_t st = make_entry(sl->ctx, &me, w_gu, w_dn, s_gu, s_dn);
     if (st != MOE_OK) return st;

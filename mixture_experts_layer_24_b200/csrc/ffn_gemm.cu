@@ -29,14 +29,9 @@
 // K blocks in increasing order.
 #include "common.cuh"
 #include "internal.h"
+#include "tile.cuh"
 
 namespace moe {
-
-constexpr uint32_t kABytes = 128 * 128;  // one 128-row x 128-byte operand tile
-
-__host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
-  return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512;
-}
 
 // bf16: one pipeline stage holds kKC consecutive 64-wide K chunks, fetched by
 // one 3-D TMA copy per operand (the per-copy cost of the TMA unit, not the
@@ -79,55 +74,11 @@ struct Fp8Cfg {
   static_assert(kStages >= 2 && NP >= 2, "FP8 pipeline needs two stages and two partial buffers");
 };
 
-struct TileInfo {
-  int e, mapi, mt, row0, nvalid, nti;  // nti: N tiles of this expert (readers of each weight tile)
-  int ng;                              // global index of the tile's N tile (nt_prefix[expert slot] + nt)
-};
-
-// The (expert, 128-row tile, N tile) of tile index `tile` (no range or status checks).
-__device__ __forceinline__ void decode_tile_at(const GemmArgs& a, int m_tiles, int bn, int tile, TileInfo& ti) {
-  int lo = 0, hi = a.L;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (a.nt_prefix[mid] * m_tiles <= tile) lo = mid;
-    else hi = mid;
-  }
-  const int nti = a.nt_prefix[lo + 1] - a.nt_prefix[lo];
-  const int local = tile - a.nt_prefix[lo] * m_tiles;
-  const int mt = local / nti, nt = local - mt * nti;
-  ti.e = a.list_expert[lo];
-  ti.mapi = a.list_map[lo];
-  ti.mt = mt;
-  ti.row0 = a.offsets[ti.e] + nt * bn;
-  ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
-  ti.nti = nti;
-  ti.ng = a.nt_prefix[lo] + nt;
-}
-
-__device__ __forceinline__ void tensormap_acquire(const void* map) {
-  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
-}
-
 // ====================================================================== bf16
 // Persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ... The
 // shared-memory pipeline runs on across tile boundaries (stage and phase come
 // from one running K-step count), and the accumulator lives in one of NBUF
 // TMEM buffers so that the epilogue of tile j overlaps the MMAs of tile j+1.
-
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Per-tile MMA width: the smallest of 16, 32, 64, 128 (<= BN) that holds
-// the tile's pairs; its index selects the activation map of that box height.
-__device__ __forceinline__ int tile_width_index(int nvalid, int bn) {
-  int w = 16, i = 0;
-  while (w < nvalid && w < bn) {
-    w <<= 1;
-    ++i;
-  }
-  return i;
-}
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ ActMaps act,
@@ -2077,6 +2028,7 @@ int ffn_block_n(int T, int wdtype) {
   // slower on a 4096-token chunk).
   int bn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
   if (wdtype == MOE_FP8_E4M3_B128 && bn > 64) bn = 64;
+  if (wdtype == MOE_MXFP4 && bn > kMxfp4MaxBn) bn = kMxfp4MaxBn;
   return bn;
 }
 

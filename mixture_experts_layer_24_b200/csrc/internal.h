@@ -13,12 +13,16 @@
 
 namespace moe {
 
-// Per-slot TMA descriptors of one expert's weights (and FP8 scales), kept in
-// a device array that the FFN kernels index by slot.
+// Per-slot TMA descriptors of one expert's weights (and FP8 / MXFP4 scales),
+// kept in a device array that the FFN kernels index by slot.
 struct alignas(64) MapEntry {
-  // bf16: 3-D maps (64 elements, rows, K/64 chunks), box {64, 128, kc} with
-  //       kc = 1 (gu, dn) and kc = 2 (gu2, dn2);
-  // FP8:  2-D maps in gu / dn, box {128 B of K, 128 rows}.
+  // bf16:  3-D maps (64 elements, rows, K/64 chunks), box {64, 128, kc} with
+  //        kc = 1 (gu, dn) and kc = 2 (gu2, dn2);
+  // FP8:   2-D maps in gu / dn, box {128 B of K, 128 rows};
+  // MXFP4: 2-D maps in gu / dn over the packed E2M1 codes (two per byte),
+  //        box {128 elements, 128 rows}, landing unpacked (16 codes per 16 B);
+  //        s_gu / s_dn point at the E8M0 scales in the tensor cores' 512-byte
+  //        block layout, [rows/128][K/128][512] bytes.
   CUtensorMap gu;   // w_gu [2I, H]
   CUtensorMap dn;   // w_dn [H, I]
   CUtensorMap gu2;
@@ -79,6 +83,8 @@ struct GemmArgs {
                               // (read it, and start streaming weights, before pdl_wait)
   int* sched;                 // fused decode FFN: [0] tile counter, [1 + n] finished gate/up
                               // tiles of global N tile n (zeroed by the plan kernel)
+  const uint8_t* act_sfb;     // MXFP4: the activation operand's E8M0 scales, blocked per N tile
+  uint8_t* h_sfb;             // MXFP4 gate/up: h's scales, written blocked per N tile for the down GEMM
   int stages;                 // pipeline depth (set by the launcher)
   int est_tiles;              // host-side bound on the tiles of this launch
   int num_sms;
@@ -209,6 +215,19 @@ cudaError_t launch_ep_recv_plan(const int32_t* recv_counts, int G, int E_loc, in
                                 int32_t* perm_k, int32_t* inv, cudaStream_t s);
 cudaError_t launch_ep_gather_rows_f32(const float* src, const int32_t* idx, int n_rows, int H, float* dst,
                                       cudaStream_t s);
+
+// MXFP4 (mx.cu, ffn_mxfp4.cu).
+cudaError_t launch_quant_mx(const void* src, int rows, int cols, int elem_e4m3, uint8_t* q, uint8_t* scales,
+                            cudaStream_t s);
+cudaError_t launch_mx_block_scales(const uint8_t* scales, int rows, int K, uint8_t* blocked, cudaStream_t s);
+cudaError_t launch_quant_mx_pairs(const void* x, const int32_t* perm_src, const int32_t* offsets,
+                                  const int32_t* nt_prefix, int E, int bn, int P, int H, uint8_t* xq, uint8_t* sfb,
+                                  cudaStream_t s, bool pdl);
+// One MXFP4 GEMM (gate/up + SwiGLU + MX quantisation of h, or down * weight)
+// over the tile list; act_maps: e4m3 activation maps of box heights 16..bn.
+cudaError_t launch_ffn_mxfp4(int mode, int bn, const ActMaps& act_maps, const GemmArgs& a, int max_tiles,
+                             cudaStream_t s, bool pdl);
+constexpr int kMxfp4MaxBn = 64;
 
 // Sets the text moe_last_error() returns on this thread.
 void record_error(const char* msg);
