@@ -425,9 +425,11 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep):
     dn_ms, dn_n = prof["down"]
     fu_ms, fu_n = prof["ffn_fused"]
     if fu_n:
-        # decode batches run both GEMMs in one launch: its bytes are gate/up + down
-        dom_bytes, dom_ms, dom_n = gu_bytes + dn_bytes, fu_ms, fu_n
-        dom_name = "ffn fused gate/up + SwiGLU + down x weight (tcgen05, one launch)"
+        # decode batches run both GEMMs and the combine in one launch: its bytes are gate/up + down + the
+        # combine's reads of the y_pair rows and writes of the outputs
+        comb_bytes = sum(b * K * H * 4 + b * H * 2 for b in batches)
+        dom_bytes, dom_ms, dom_n = gu_bytes + dn_bytes + comb_bytes, fu_ms, fu_n
+        dom_name = "ffn decode: gate/up + SwiGLU + down x weight + combine (tcgen05, one launch)"
     else:
         dom_bytes, dom_ms, dom_n = gu_bytes, gu_ms, gu_n
         dom_name = "ffn gate/up GEMM + SwiGLU (tcgen05)"

@@ -1171,6 +1171,17 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
       d.perm_src[p] = s_psrc[p];
       d.perm_k[p] = s_pk[p];
     }
+    if (d.out) {  // a token all of whose pairs are dropped gets no down tile: its output is zero
+      for (int t = 0; t < d.T; ++t) {
+        bool any = false;
+        for (int k = 0; k < K; ++k) {
+          const int e = s_e[t * K + k];
+          any |= e >= 0 && d.map_of[e] >= 0;
+        }
+        if (!any)
+          for (int o = tid; o < a.H; o += 192) static_cast<__nv_bfloat16*>(d.out)[(size_t)t * a.H + o] = __float2bfloat16_rn(0.0f);
+      }
+    }
   }
 
   const int Gt = L * mg, total = Gt + L * md;
@@ -1463,6 +1474,40 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(buf));
+      if (!gu && d.out) {
+        // Combine inside the launch: a (token, 128-column block) is complete when the down tiles of all its
+        // valid pairs have stored their y rows; the tile that completes it sums the token's pairs, k
+        // ascending from the first valid one, and rounds once to bf16 (the combine kernel's arithmetic).
+        __threadfence();         // this thread's y stores before the count (release)
+        named_bar_sync(1, 128);  // every epilogue thread's stores are fenced
+        if (r < cnt) {
+          const int t = s_psrc[row0 + r];
+          int kv = 0;
+          for (int k = 0; k < K; ++k) {
+            const int e2 = s_e[t * K + k];
+            kv += (e2 >= 0 && d.map_of[e2] >= 0) ? 1 : 0;
+          }
+          const int prev = atomicAdd(d.comb_cnt + t * md + mt, 1);
+          s_t2p[r] = prev == kv - 1 ? t : -1;  // s_t2p is free during a down tile
+        }
+        named_bar_sync(1, 128);
+        __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(d.out);
+        for (int n = 0; n < cnt; ++n) {
+          const int t = s_t2p[n];
+          if (t < 0) continue;  // block-uniform
+          __threadfence();      // the other tiles' y rows (acquire, after their fenced counts)
+          float acc = 0.0f;
+          bool have = false;
+          for (int k = 0; k < K; ++k) {
+            const int e2 = s_e[t * K + k];
+            if (e2 < 0 || d.map_of[e2] < 0) continue;
+            const float yv = __ldcg(a.y_out + (size_t)s_inv[t * K + k] * a.H + mt * 128 + r);
+            acc = have ? acc + yv : yv;
+            have = true;
+          }
+          outp[(size_t)t * a.H + mt * 128 + r] = __float2bfloat16_rn(acc);
+        }
+      }
       if (gu) {
         __threadfence();
         named_bar_sync(1, 128);
