@@ -425,8 +425,10 @@ class MoeLayer:
 
         Returns (graph, out): graph.replay() recomputes out from the current
         contents of x. Valid while x, w_router, logit_bias and the registered
-        weights stay where they are; residency must be all-HBM (the hot/cold
-        path synchronises with the host and cannot be captured)."""
+        weights stay where they are. With host-resident experts, only batches
+        whose T * top_k fits in the spare slots can be captured (their cache
+        bookkeeping and copies run on the device); larger ones synchronise with
+        the host."""
         T = x.shape[0]
         ws = torch.empty(max(moe_workspace_size(self.ctx, T), 256), dtype=torch.uint8, device=self.device)
         out = torch.empty((T, self.H), dtype=torch.bfloat16, device=self.device)

@@ -155,6 +155,16 @@ struct moe_slots {
   cudaEvent_t ev_done = nullptr;    // after the most recent call's GEMMs (they may read the slots)
   bool ev_done_valid = false;
   std::vector<uint8_t*> sf_blk;     // [E] MXFP4: the expert's E8M0 scales in the block layout (owned here)
+  // The LRU state lives on the device (decode batches run it there, residency.cu); the vectors above
+  // mirror it for the host-synchronised path, which pulls it before and pushes it after its own use.
+  void* d_res = nullptr;
+  ResidencyDev rdev{};
+  std::vector<HostRec> h_host;      // [E] device-visible addresses of host records
+  std::vector<char> unmapped;       // [E] host record without a device address
+  int n_unmapped = 0;
+  bool last_dev = false;            // the most recent call ran the device-side path
+  int64_t* h_lru = nullptr;         // pinned staging: pull half, push half
+  size_t h_lru_words = 0;           // int64 words per half
   std::mutex mu;
 };
 
@@ -316,6 +326,64 @@ moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void
   return MOE_OK;
 }
 
+
+// ---- the slot table's LRU state between host and device. Staging half (words): [0] tick, [1..8] stats,
+// [9 .. 9+n_spare) slot ticks, then int32 slot_expert [n_spare], expert_slot [E], map_of [E].
+int64_t* lru_half(moe_slots_t* sl, int half) { return sl->h_lru + (size_t)half * sl->h_lru_words; }
+
+// Queues the device state's copy into the pull half (the caller synchronises before lru_unpack).
+moe_status_t lru_pull_async(moe_slots_t* sl, cudaStream_t s) {
+  if (!sl->d_res) return MOE_OK;
+  int64_t* h = lru_half(sl, 0);
+  int32_t* h32 = reinterpret_cast<int32_t*>(h + 9 + sl->n_spare);
+  MOE_CUDA(cudaMemcpyAsync(h, sl->rdev.tick, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaMemcpyAsync(h + 1, sl->rdev.stats, 8 * sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaMemcpyAsync(h + 9, sl->rdev.slot_tick, sl->n_spare * sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaMemcpyAsync(h32, sl->rdev.slot_expert, sl->n_spare * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  MOE_CUDA(cudaMemcpyAsync(h32 + sl->n_spare, sl->rdev.expert_slot, sl->E * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                           s));
+  return MOE_OK;
+}
+
+void lru_unpack(moe_slots_t* sl) {
+  if (!sl->d_res) return;
+  const int64_t* h = lru_half(sl, 0);
+  const int32_t* h32 = reinterpret_cast<const int32_t*>(h + 9 + sl->n_spare);
+  sl->tick = h[0];
+  for (int i = 0; i < sl->n_spare; ++i) {
+    sl->slot_tick[i] = h[9 + i];
+    sl->slot_expert[i] = h32[i];
+  }
+  for (int e = 0; e < sl->E; ++e) sl->expert_slot[e] = h32[sl->n_spare + e];
+}
+
+// Queues the host mirror's copy to the device, with the expert -> map-entry table it implies.
+moe_status_t lru_push_async(moe_slots_t* sl, cudaStream_t s) {
+  if (!sl->d_res) return MOE_OK;
+  int64_t* h = lru_half(sl, 1);
+  int32_t* h32 = reinterpret_cast<int32_t*>(h + 9 + sl->n_spare);
+  h[0] = sl->tick;
+  for (int i = 0; i < sl->n_spare; ++i) {
+    h[9 + i] = sl->slot_tick[i];
+    h32[i] = sl->slot_expert[i];
+  }
+  for (int e = 0; e < sl->E; ++e) {
+    h32[sl->n_spare + e] = sl->expert_slot[e];
+    const int m = sl->loc[e] == MOE_LOC_HBM ? e
+                  : (sl->loc[e] == MOE_LOC_HOST_PINNED && sl->expert_slot[e] >= 0) ? sl->E + sl->expert_slot[e]
+                                                                                   : -1;
+    h32[sl->n_spare + sl->E + e] = m;
+    sl->h_map_of[e] = m;
+  }
+  MOE_CUDA(cudaMemcpyAsync(sl->rdev.tick, h, sizeof(int64_t), cudaMemcpyHostToDevice, s));
+  MOE_CUDA(cudaMemcpyAsync(sl->rdev.slot_tick, h + 9, sl->n_spare * sizeof(int64_t), cudaMemcpyHostToDevice, s));
+  MOE_CUDA(cudaMemcpyAsync(sl->rdev.slot_expert, h32, sl->n_spare * sizeof(int32_t), cudaMemcpyHostToDevice, s));
+  MOE_CUDA(cudaMemcpyAsync(sl->rdev.expert_slot, h32 + sl->n_spare, sl->E * sizeof(int32_t), cudaMemcpyHostToDevice,
+                           s));
+  MOE_CUDA(cudaMemcpyAsync(sl->d_map_of, h32 + sl->n_spare + sl->E, sl->E * sizeof(int32_t), cudaMemcpyHostToDevice,
+                           s));
+  return MOE_OK;
+}
 
 // Runs the two GEMMs (and, for FP8, the quantiser of h between them) for one
 // expert list whose arrays live in the workspace at list offset `lo`.
@@ -728,6 +796,16 @@ moe_status_t ffn_decode_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, con
   return MOE_OK;
 }
 
+// Decode batches with host-resident experts whose pairs cannot route to more host experts than there are
+// spare slots: the cache bookkeeping and the copies run on the device (residency.cu), no host round trip.
+bool residency_device_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, int T) {
+  const moe_config_t& c = ctx->cfg;
+  return c.wdtype == MOE_BF16 && sl->n_host > 0 && sl->d_res && sl->policy == MOE_SLOTS_LRU &&
+         sl->n_unmapped == 0 && (long long)T * c.top_k <= sl->n_spare && T >= 1 && T <= kDecodeMaxT &&
+         (long long)T * c.top_k <= kDecodeMaxPairs && ((uintptr_t)x % 16) == 0 &&
+         ffn_decode_smem_bytes(T, c.n_experts) <= 232448;
+}
+
 bool decode_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, int T) {
   const moe_config_t& c = ctx->cfg;
   return c.wdtype == MOE_BF16 && sl->n_host == 0 && T >= 1 && T <= kDecodeMaxT &&
@@ -820,7 +898,10 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   // ---- hot/cold: read the per-expert offsets back, stage the routed cold experts
   int32_t* hoff = sl->h_pinned;
   MOE_CUDA(cudaMemcpyAsync(hoff, offsets, sizeof(int32_t) * (E + 1), cudaMemcpyDeviceToHost, s));
+  if ((st = lru_pull_async(sl, s)) != MOE_OK) return st;  // the cache state the device-side path left
   MOE_CUDA(cudaStreamSynchronize(s));
+  lru_unpack(sl);
+  sl->last_dev = false;
   std::vector<int> hot, cold;
   int touched = 0;
   for (int e = 0; e < E; ++e) {
@@ -921,7 +1002,7 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     }
     MOE_CUDA(cudaEventRecord(sl->ev_done, s));
     sl->ev_done_valid = true;
-    return MOE_OK;
+    return lru_push_async(sl, s);
   }
   // per-call staging (or more routed host experts than slots): every slot is overwritten, the cache empties
   std::fill(sl->slot_expert.begin(), sl->slot_expert.end(), -1);
@@ -1001,7 +1082,7 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
   }
   MOE_CUDA(cudaEventRecord(sl->ev_done, s));
   sl->ev_done_valid = true;
-  return MOE_OK;
+  return lru_push_async(sl, s);
 }
 
 }  // namespace
@@ -1082,6 +1163,24 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
   float* y = at<float>(ws, W.y_pair);
   const bool resident = sl->n_host == 0;
   const bool chain = ctx->chain;
+  if (residency_device_path_ok(ctx, sl, x, T)) {
+    // decode with host-resident experts: router -> cache plan -> copies of the missed experts (none when
+    // every routed expert is resident or cached) -> FFN planned from the top-k, combine inside
+    int* sched = at<int>(ws, W.sched);
+    const int sched_n = fused_sched_entries(c.n_experts) + T * (c.hidden / 128);
+    if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n)) != MOE_OK) return st;
+    {
+      Prof p(ctx, MOE_PROF_PERMUTE, s);
+      MOE_CUDA(launch_residency_plan(idx, T * c.top_k, c.n_experts, sl->rdev, sl->d_map_of, s, chain));
+    }
+    {
+      Prof p(ctx, MOE_PROF_GATHER, s);
+      MOE_CUDA(launch_residency_copy(sl->rdev, sl->spare, ctx->num_sms, s, chain));
+    }
+    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched, out)) != MOE_OK) return st;
+    sl->last_dev = true;
+    return MOE_OK;
+  }
   if (decode_path_ok(ctx, sl, x, T)) {
     // decode: router (which also zeroes the FFN's counters and combine counts) -> FFN planned from the
     // top-k, with the combine inside the same launch
@@ -1233,6 +1332,54 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
   sl->slot_expert.assign(n_spare, -1);
   sl->expert_slot.assign(sl->E, -1);
   sl->slot_tick.assign(n_spare, -1);
+  sl->h_host.assign(sl->E, HostRec{});
+  sl->unmapped.assign(sl->E, 0);
+  if (n_spare > 0) {
+    // the LRU state on the device: loc, host records, slot_expert, slot_tick, expert_slot, tick, copy list, stats
+    const size_t E_ = sl->E;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+      const size_t at = o;
+      o += align256(bytes);
+      return at;
+    };
+    const size_t o_loc = take(E_ * 4), o_host = take(E_ * sizeof(HostRec)), o_se = take(n_spare * 4),
+                 o_st = take(n_spare * 8), o_es = take(E_ * 4), o_tick = take(8), o_cn = take(4),
+                 o_ce = take(n_spare * 4), o_cs = take(n_spare * 4), o_stats = take(8 * 8);
+    uint8_t* d = nullptr;
+    if (cudaMalloc(&d, o) != cudaSuccess) return cleanup(MOE_ERR_OOM, "cudaMalloc of the residency state failed");
+    sl->d_res = d;
+    ResidencyDev& r = sl->rdev;
+    r.loc = reinterpret_cast<const int32_t*>(d + o_loc);
+    r.host = reinterpret_cast<const HostRec*>(d + o_host);
+    r.slot_expert = reinterpret_cast<int32_t*>(d + o_se);
+    r.slot_tick = reinterpret_cast<long long*>(d + o_st);
+    r.expert_slot = reinterpret_cast<int32_t*>(d + o_es);
+    r.tick = reinterpret_cast<long long*>(d + o_tick);
+    r.copy_n = reinterpret_cast<int32_t*>(d + o_cn);
+    r.copy_e = reinterpret_cast<int32_t*>(d + o_ce);
+    r.copy_slot = reinterpret_cast<int32_t*>(d + o_cs);
+    r.stats = reinterpret_cast<long long*>(d + o_stats);
+    r.status_word = ctx->d_status;
+    r.n_spare = n_spare;
+    r.slot_bytes = sl->slot_bytes;
+    r.part_off[0] = 0;
+    r.part_off[1] = sl->off_dn;
+    r.part_off[2] = sl->off_sgu;
+    r.part_off[3] = sl->off_sdn;
+    r.part_bytes[0] = sl->bytes_gu;
+    r.part_bytes[1] = sl->bytes_dn;
+    r.part_bytes[2] = sl->bytes_sgu;
+    r.part_bytes[3] = sl->bytes_sdn;
+    if (cudaMemset(d, 0xff, o) != cudaSuccess ||  // -1 everywhere ...
+        cudaMemset(d + o_host, 0, E_ * sizeof(HostRec)) != cudaSuccess ||
+        cudaMemset(d + o_tick, 0, 8) != cudaSuccess || cudaMemset(d + o_cn, 0, 4) != cudaSuccess ||
+        cudaMemset(d + o_stats, 0, 64) != cudaSuccess)  // ... except the records, tick, copy count, stats
+      return cleanup(MOE_ERR_CUDA, "cudaMemset of the residency state failed");
+    sl->h_lru_words = 9 + (size_t)n_spare + (2 * (size_t)n_spare + 2 * E_ + 1) / 2 + 1;
+    if (cudaHostAlloc(&sl->h_lru, 2 * sl->h_lru_words * sizeof(int64_t), cudaHostAllocDefault) != cudaSuccess)
+      return cleanup(MOE_ERR_OOM, "cudaHostAlloc of the residency staging failed");
+  }
   for (int i = 0; i < n_spare; ++i) {
     uint8_t* slot = sl->spare + (size_t)i * sl->slot_bytes;
     moe_status_t st = make_entry(ctx, &sl->h_maps[sl->E + i], slot, slot + sl->off_dn,
@@ -1264,6 +1411,8 @@ moe_status_t moe_slots_destroy(moe_slots_t* sl) {
   if (sl->spare) cudaFree(sl->spare);
   if (sl->d_maps) cudaFree(sl->d_maps);
   if (sl->d_map_of) cudaFree(sl->d_map_of);
+  if (sl->d_res) cudaFree(sl->d_res);
+  if (sl->h_lru) cudaFreeHost(sl->h_lru);
   for (uint8_t* b : sl->sf_blk)
     if (b) cudaFree(b);
   delete sl;
@@ -1285,6 +1434,13 @@ moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, c
   const float* s_gu = static_cast<const float*>(s_gu_);
   const float* s_dn = static_cast<const float*>(s_dn_);
   std::lock_guard<std::mutex> lock(sl->mu);
+  if (sl->d_res) {  // the cache state as the device-side path left it
+    MOE_CUDA(cudaDeviceSynchronize());
+    moe_status_t st = lru_pull_async(sl, nullptr);
+    if (st != MOE_OK) return st;
+    MOE_CUDA(cudaDeviceSynchronize());
+    lru_unpack(sl);
+  }
   if (location == MOE_LOC_HBM) {
     const uintptr_t align = c.wdtype == MOE_MXFP4 ? 32 : 16;  // packed E2M1 tensor maps need 32-byte bases
     if ((reinterpret_cast<uintptr_t>(w_gu) | reinterpret_cast<uintptr_t>(w_dn)) % align)
@@ -1331,6 +1487,34 @@ moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, c
   sl->sgu[expert] = s_gu;
   sl->sdn[expert] = s_dn;
   MOE_CUDA(cudaMemcpy(sl->d_map_of + expert, &sl->h_map_of[expert], sizeof(int32_t), cudaMemcpyHostToDevice));
+  if (sl->d_res) {
+    // device side: where the expert lives, its record's device-visible addresses (pinned host memory is
+    // mapped into the device's address space), and the cache state
+    HostRec hr{};
+    char unm = 0;
+    if (location == MOE_LOC_HOST_PINNED) {
+      const void* parts[4] = {w_gu, w_dn, s_gu, s_dn};
+      for (int i = 0; i < 4; ++i) {
+        if (!parts[i]) continue;
+        void* dp = nullptr;
+        if (cudaHostGetDevicePointer(&dp, const_cast<void*>(parts[i]), 0) != cudaSuccess || !dp) {
+          cudaGetLastError();  // not mapped: this expert keeps the host-synchronised path
+          unm = 1;
+          break;
+        }
+        hr.p[i] = dp;
+      }
+    }
+    sl->n_unmapped += (int)unm - (int)sl->unmapped[expert];
+    sl->unmapped[expert] = unm;
+    sl->h_host[expert] = hr;
+    MOE_CUDA(cudaMemcpy(const_cast<int32_t*>(sl->rdev.loc) + expert, &location, sizeof(int32_t),
+                        cudaMemcpyHostToDevice));
+    MOE_CUDA(cudaMemcpy(const_cast<HostRec*>(sl->rdev.host) + expert, &hr, sizeof(HostRec), cudaMemcpyHostToDevice));
+    moe_status_t st = lru_push_async(sl, nullptr);
+    if (st != MOE_OK) return st;
+    MOE_CUDA(cudaDeviceSynchronize());
+  }
   return MOE_OK;
 }
 
@@ -1347,15 +1531,43 @@ moe_status_t moe_slots_set_policy(moe_slots_t* sl, int policy) {
   if (policy != MOE_SLOTS_LRU && policy != MOE_SLOTS_PER_CALL) return fail(MOE_ERR_INVALID_ARG, "bad policy");
   std::lock_guard<std::mutex> lock(sl->mu);
   sl->policy = policy;
+  if (sl->d_res) {
+    MOE_CUDA(cudaDeviceSynchronize());
+    moe_status_t st = lru_pull_async(sl, nullptr);  // keeps the tick
+    if (st != MOE_OK) return st;
+    MOE_CUDA(cudaDeviceSynchronize());
+    lru_unpack(sl);
+  }
   std::fill(sl->slot_expert.begin(), sl->slot_expert.end(), -1);
   std::fill(sl->expert_slot.begin(), sl->expert_slot.end(), -1);
   std::fill(sl->slot_tick.begin(), sl->slot_tick.end(), -1);
+  if (sl->d_res) {
+    moe_status_t st = lru_push_async(sl, nullptr);
+    if (st != MOE_OK) return st;
+    MOE_CUDA(cudaDeviceSynchronize());
+  }
   return MOE_OK;
 }
 
 moe_status_t moe_slots_stats(const moe_slots_t* sl, moe_slots_stats_t* stats) {
   if (!sl || !stats) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
   *stats = sl->stats;
+  if (sl->d_res) {
+    // counts of the device-side path: [0] last touched, [1] last routed host, [2] last hits, [3] last misses,
+    // [4] hits, [5] misses (cumulative)
+    int64_t dst[8];
+    MOE_CUDA(cudaDeviceSynchronize());
+    MOE_CUDA(cudaMemcpy(dst, sl->rdev.stats, sizeof(dst), cudaMemcpyDeviceToHost));
+    if (sl->last_dev) {
+      stats->last_touched = (int32_t)dst[0];
+      stats->last_routed_cold = (int32_t)dst[1];
+      stats->last_hits = (int32_t)dst[2];
+      stats->last_cold = (int32_t)dst[3];
+    }
+    stats->cache_hits += dst[4];
+    stats->cold_staged += dst[5];
+    stats->bytes_staged += dst[5] * (int64_t)(sl->bytes_gu + sl->bytes_dn + sl->bytes_sgu + sl->bytes_sdn);
+  }
   return MOE_OK;
 }
 

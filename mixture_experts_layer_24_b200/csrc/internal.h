@@ -231,6 +231,32 @@ cudaError_t launch_ffn_mxfp4(int mode, int bn, const ActMaps& act_maps, const Ge
                              cudaStream_t s, bool pdl);
 constexpr int kMxfp4MaxBn = 64;
 
+// Host-resident experts on the device path (residency.cu): the slot table's
+// LRU state in device memory, and the device-visible addresses of every host
+// expert's pinned record (gate/up, down, FP8 scales).
+struct HostRec {
+  const void* p[4];
+};
+struct ResidencyDev {
+  const int32_t* loc;      // [E] MOE_LOC_* or -1
+  const HostRec* host;     // [E]
+  int32_t* slot_expert;    // [n_spare] expert held, -1 empty
+  long long* slot_tick;    // [n_spare] call that last used the slot, -1 never
+  int32_t* expert_slot;    // [E] its spare slot, -1 not cached
+  long long* tick;         // calls so far (shared with the host-synchronised path)
+  int32_t* copy_n;         // misses of the current call ...
+  int32_t* copy_e;         // [n_spare] ... their experts ...
+  int32_t* copy_slot;      // [n_spare] ... and slots
+  long long* stats;        // [8] last touched, last routed host, last hits, last misses, hits, misses
+  int* status_word;
+  int n_spare;
+  size_t slot_bytes;
+  size_t part_off[4], part_bytes[4];
+};
+cudaError_t launch_residency_plan(const int32_t* idx, int P, int E, const ResidencyDev& rd, int32_t* map_of,
+                                  cudaStream_t s, bool pdl);
+cudaError_t launch_residency_copy(const ResidencyDev& rd, uint8_t* spare, int num_sms, cudaStream_t s, bool pdl);
+
 // Sets the text moe_last_error() returns on this thread.
 void record_error(const char* msg);
 

@@ -138,3 +138,35 @@ def test_reregistering_an_expert_drops_its_cached_copy():
     assert cache.stats()["last_cold"] >= 1  # e was copied again
     ref.close()
     cache.close()
+
+
+def test_device_side_cache_in_a_cuda_graph():
+    """Decode batches whose pairs fit in the spare slots keep the whole cache
+    bookkeeping on the device (plan, copies of the missed experts, FFN), so the
+    forward can be captured once and replayed: over replays with new tokens the
+    cache fills, hits and evicts inside the graph, and every output equals the
+    all-resident layer's bits and the oracle within 2e-2."""
+    _need_cuda()
+    import mixture_experts_layer_24_b200 as M
+    ref, cache, wr, bias, keep = _layers(0, M.MOE_SLOTS_LRU)
+    dev = torch.device("cuda")
+    T = 2  # 8 pairs <= 12 slots: the device-side path
+    x = synth.tokens(T, H, seed=5, device=dev, first_token=9000)
+    g, out = cache.capture(x, wr, bias)
+    seen_hits = 0
+    for i, first in enumerate([9000, 9100, 9000, 9200, 9300, 9100, 9400, 9000]):
+        x.copy_(synth.tokens(T, H, seed=5, device=dev, first_token=first))
+        g.replay()
+        a = ref.forward(x, wr, bias)
+        torch.cuda.synchronize()
+        assert cache.status() == 0 and ref.status() == 0
+        got = oracle.as_u16(out)
+        assert np.array_equal(got, oracle.as_u16(a)), f"replay {i} differs"
+        assert_close_out(got, oracle_layer_out(oracle.as_u16(x), wr.cpu().numpy(), None, K, E, H, I, seed=5), TOL[0])
+        st = cache.stats()
+        assert st["last_hits"] + st["last_cold"] == st["last_routed_cold"]
+        seen_hits += st["last_hits"]
+    assert seen_hits > 0
+    assert cache.stats()["cold_staged"] > N_SLOTS  # the graph's own copies refilled evicted slots
+    ref.close()
+    cache.close()
