@@ -531,7 +531,8 @@ def run_profile_case(kind):
     touched) and 64 tokens; "t1": 8 experts (top-8 of 8, all touched, 400 MB)
     and one token -- the per-launch shape of batch-1 decode; "p2048": 48
     experts and a 2048-token prefill chunk under the Zipf logit prior;
-    "f64" / "f2048": "t64" / "p2048" with e4m3 experts; "r4096": the router
+    "f64" / "f2048": "t64" / "p2048" with e4m3 experts; "m64" / "m2048": with MXFP4
+    experts; "r4096": the router
     alone (384 experts, 4096 tokens, Zipf prior), three calls."""
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
@@ -548,13 +549,21 @@ def run_profile_case(kind):
         print(json.dumps({"profile_case": f"router E={E} H={H} K={K} T=4096", "status": st}))
         layer.close()
         return 1 if st else 0
-    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64), "f2048": (48, 2048)}[kind]
+    E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64), "f2048": (48, 2048),
+                "m64": (32, 64), "m2048": (48, 2048)}[kind]
     fp8 = kind in ("f64", "f2048")
-    layer = M.MoeLayer(H, E_s, K, I, wdtype=M.MOE_FP8_E4M3_B128 if fp8 else M.MOE_BF16, device=device)
+    mx = kind in ("m64", "m2048")
+    wd = M.MOE_FP8_E4M3_B128 if fp8 else (M.MOE_MXFP4 if mx else M.MOE_BF16)
+    layer = M.MoeLayer(H, E_s, K, I, wdtype=wd, device=device)
     keep = []
     for e in range(E_s):
         g, d = synth.expert_weights(e, H, I, seed=SEED, device=device)
-        if fp8:
+        if mx:
+            w = quantize_expert_mx(M, g, d, device)
+            del g, d
+            layer.register(e, *w)
+            keep.append(w)
+        elif fp8:
             w = quantize_expert(M, g, d, device)
             del g, d
             layer.register(e, *w)
@@ -563,13 +572,14 @@ def run_profile_case(kind):
             layer.register(e, g, d)
             keep.append((g, d))
     wr = synth.router_weight(E_s, H, seed=SEED, device=device)
-    bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind in ("p2048", "f2048") else None
+    bias = synth.zipf_logit_bias(E_s, ZIPF_S, seed=SEED).to(device) if kind in ("p2048", "f2048", "m2048") else None
     x = synth.tokens(T_s, H, seed=SEED, device=device)
     for _ in range(3):
         layer.forward(x, wr, bias)
     torch.cuda.synchronize()
     st = layer.status()
-    print(json.dumps({"profile_case": f"E={E_s} H={H} I={I} K={K} T={T_s} {'e4m3' if fp8 else 'bf16'}", "status": st}))
+    print(json.dumps({"profile_case": f"E={E_s} H={H} I={I} K={K} T={T_s} {'e4m3' if fp8 else ('mxfp4' if mx else 'bf16')}",
+                      "status": st}))
     layer.close()
     return 1 if st else 0
 
@@ -583,6 +593,18 @@ def quantize_expert(M, g, d, device):
     sd = torch.empty((H // 128, I // 128), dtype=torch.float32, device=device)
     M.moe_quantize_e4m3(g, 2 * I, H, 128, qg, sg)
     M.moe_quantize_e4m3(d, H, I, 128, qd, sd)
+    return qg, qd, sg, sd
+
+
+def quantize_expert_mx(M, g, d, device):
+    """(codes_gu, codes_dn, scales_gu, scales_dn): packed E2M1 codes and E8M0
+    scales per 32 elements, quantised on the GPU by the library's MX quantiser."""
+    qg = torch.empty((2 * I, H // 2), dtype=torch.uint8, device=device)
+    sg = torch.empty((2 * I, H // 32), dtype=torch.uint8, device=device)
+    qd = torch.empty((H, I // 2), dtype=torch.uint8, device=device)
+    sd = torch.empty((H, I // 32), dtype=torch.uint8, device=device)
+    M.moe_quantize_mx(g, 2 * I, H, 0, qg, sg)
+    M.moe_quantize_mx(d, H, I, 0, qd, sd)
     return qg, qd, sg, sd
 
 
@@ -627,15 +649,9 @@ def fp4_breakdown(keep, wr, bias, flush, stream, device, hbm):
     layer = M.MoeLayer(H, E, K, I, wdtype=M.MOE_MXFP4, device=device)
     qkeep = []
     for e in range(E):
-        g, d = keep[e]
-        qg = torch.empty((2 * I, H // 2), dtype=torch.uint8, device=device)
-        sg = torch.empty((2 * I, H // 32), dtype=torch.uint8, device=device)
-        qd = torch.empty((H, I // 2), dtype=torch.uint8, device=device)
-        sd = torch.empty((H, I // 32), dtype=torch.uint8, device=device)
-        M.moe_quantize_mx(g, 2 * I, H, 0, qg, sg)
-        M.moe_quantize_mx(d, H, I, 0, qd, sd)
-        layer.register(e, qg, qd, sg, sd)
-        qkeep.append((qg, qd, sg, sd))
+        w = quantize_expert_mx(M, keep[e][0], keep[e][1], device)
+        layer.register(e, *w)
+        qkeep.append(w)
     torch.cuda.synchronize()
     layer.workspace(4096)
     fp4_bytes = 3 * I * H // 2 + 3 * I * H // 32
@@ -841,7 +857,7 @@ def main():
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
     ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "r4096"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "m64", "m2048", "r4096"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:
