@@ -1023,8 +1023,9 @@ struct DecodeCfg {
   static constexpr uint32_t kAcc = 2 * TP;
   static constexpr uint32_t kTmemCols = tmem_cols_for(2 * kAcc);
   static constexpr int kMaxPairs = 512;
-  // plan: s_e, s_psrc, s_pk [kMaxPairs]; s_cnt[E], s_off[E+1], s_list[E]; s_t2p[TP]; scan[8]; s_run[E]; s_inv[kMaxPairs]
-  static size_t plan_bytes(int E) { return 4 * (4 * (size_t)kMaxPairs + 4 * (size_t)E + 1 + TP + 8); }
+  // plan: s_e, s_psrc, s_pk [kMaxPairs]; s_cnt[E], s_off[E+1], s_list[E]; s_t2p[TP]; scan[8]; s_run[E];
+  // s_inv[kMaxPairs]; combine: s_vp[kMaxPairs] (sorted row of each kept pair, -1 dropped), s_kv[TP] (kept pairs)
+  static size_t plan_bytes(int E) { return 4 * (5 * (size_t)kMaxPairs + 4 * (size_t)E + 1 + 2 * TP + 8); }
   static size_t smem(int E) {
     return 1024 + (size_t)kStages * kStageBytes + 8 * (2 * kStages + 4 + 2 * kRing) + 4 * kRing + 16 + 4 * TP +
            plan_bytes(E);
@@ -1101,6 +1102,8 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
   int* s_scan = s_t2p + TP;                               // [8]
   int* s_run = s_scan + 8;                                // [E] running count per expert (ranks)
   int* s_inv = s_run + E;                                 // [kMaxPairs] sorted place of pair i
+  int* s_vp = s_inv + C::kMaxPairs;                       // [kMaxPairs] sorted place of pair i if kept, else -1
+  int* s_kv = s_vp + C::kMaxPairs;                        // [TP] kept pairs of token t
 
   // ---------------------------------------------------------------- plan
   for (int i = tid; i < E; i += 192) s_cnt[i] = 0;
@@ -1159,8 +1162,15 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
     }
   }
   __syncthreads();
+  for (int i = tid; i < P; i += 192) s_vp[i] = (s_e[i] >= 0 && d.map_of[s_e[i]] >= 0) ? s_inv[i] : -1;
+  __syncthreads();
+  for (int t = tid; t < d.T; t += 192) {
+    int kv = 0;
+    for (int k = 0; k < K; ++k) kv += s_vp[t * K + k] >= 0 ? 1 : 0;
+    s_kv[t] = kv;
+  }
   if (blockIdx.x == 0)  // a pair of an unregistered expert is dropped: the combine skips inv = -1
-    for (int i = tid; i < P; i += 192) d.inv[i] = (s_e[i] >= 0 && d.map_of[s_e[i]] < 0) ? -1 : s_inv[i];
+    for (int i = tid; i < P; i += 192) d.inv[i] = s_vp[i];
   if (blockIdx.x == 0) {
     for (int e = tid; e < E; e += 192) {
       d.counts[e] = s_cnt[e];
@@ -1172,15 +1182,10 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
       d.perm_k[p] = s_pk[p];
     }
     if (d.out) {  // a token all of whose pairs are dropped gets no down tile: its output is zero
-      for (int t = 0; t < d.T; ++t) {
-        bool any = false;
-        for (int k = 0; k < K; ++k) {
-          const int e = s_e[t * K + k];
-          any |= e >= 0 && d.map_of[e] >= 0;
-        }
-        if (!any)
+      __syncthreads();  // s_kv is complete
+      for (int t = 0; t < d.T; ++t)
+        if (s_kv[t] == 0)
           for (int o = tid; o < a.H; o += 192) static_cast<__nv_bfloat16*>(d.out)[(size_t)t * a.H + o] = __float2bfloat16_rn(0.0f);
-      }
     }
   }
 
@@ -1482,30 +1487,36 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
         named_bar_sync(1, 128);  // every epilogue thread's stores are fenced
         if (r < cnt) {
           const int t = s_psrc[row0 + r];
-          int kv = 0;
-          for (int k = 0; k < K; ++k) {
-            const int e2 = s_e[t * K + k];
-            kv += (e2 >= 0 && d.map_of[e2] >= 0) ? 1 : 0;
-          }
           const int prev = atomicAdd(d.comb_cnt + t * md + mt, 1);
-          s_t2p[r] = prev == kv - 1 ? t : -1;  // s_t2p is free during a down tile
+          s_t2p[r] = prev == s_kv[t] - 1 ? t : -1;  // s_t2p is free during a down tile
         }
         named_bar_sync(1, 128);
+        bool any = false;
+        for (int n = 0; n < cnt; ++n) any |= s_t2p[n] >= 0;
+        if (any) __threadfence();  // the other tiles' y rows (acquire, after their fenced counts)
         __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(d.out);
+        const int o = mt * 128 + r;
         for (int n = 0; n < cnt; ++n) {
           const int t = s_t2p[n];
           if (t < 0) continue;  // block-uniform
-          __threadfence();      // the other tiles' y rows (acquire, after their fenced counts)
+          const int* vp = s_vp + t * K;
           float acc = 0.0f;
           bool have = false;
-          for (int k = 0; k < K; ++k) {
-            const int e2 = s_e[t * K + k];
-            if (e2 < 0 || d.map_of[e2] < 0) continue;
-            const float yv = __ldcg(a.y_out + (size_t)s_inv[t * K + k] * a.H + mt * 128 + r);
-            acc = have ? acc + yv : yv;
-            have = true;
+          for (int k0 = 0; k0 < K; k0 += 8) {  // eight rows' loads in flight, then the adds, k ascending
+            float yv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int p = k0 + u < K ? vp[k0 + u] : -1;
+              yv[u] = p >= 0 ? __ldcg(a.y_out + (size_t)p * a.H + o) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              if (k0 + u >= K || vp[k0 + u] < 0) continue;
+              acc = have ? acc + yv[u] : yv[u];
+              have = true;
+            }
           }
-          outp[(size_t)t * a.H + mt * 128 + r] = __float2bfloat16_rn(acc);
+          outp[(size_t)t * a.H + o] = __float2bfloat16_rn(acc);
         }
       }
       if (gu) {

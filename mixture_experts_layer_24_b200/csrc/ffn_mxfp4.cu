@@ -175,14 +175,33 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
         const uint8_t* sfa1 = sfa + (size_t)(m_tiles + ti.mt) * KB * 512;  // up rows start at row I
         const uint8_t* sfb = a.act_sfb + (size_t)ti.ng * KB * 512;
         tensormap_acquire(wmap);
+        int kb = 0;
         if (first) {
           first = false;
-          if (a.plan_ready) {  // the activations come from the previous kernel
+          // the plan is complete: the first stages' weights and weight scales go out before waiting for the
+          // kernel that writes the activations and their scales
+          const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
+          for (int j = 0; j < npre; ++j) {
+            const uint32_t st = base + j * STAGE;
+            mbar_arrive_expect_tx(full(j), stage_tx);
+            tma_load_2d_hint(st, wmap, full(j), j * 128, ti.mt * 128, pol_w);
+            if (MODE == kGateUp) tma_load_2d_hint(st + C::kAOp, wmap, full(j), j * 128, a.I + ti.mt * 128, pol_w);
+            bulk_load(st + C::kSfOff, sfa0 + (size_t)j * 512, 512, full(j));
+            if (MODE == kGateUp) bulk_load(st + C::kSfOff + 512, sfa1 + (size_t)j * 512, 512, full(j));
+          }
+          if (a.plan_ready) {
             pdl_wait();
             pdl_trigger();
           }
+          for (int j = 0; j < npre; ++j) {
+            const uint32_t st = base + j * STAGE;
+            tma_load_2d(st + C::kBOff, amap, full(j), j * 128, ti.row0);
+            bulk_load(st + C::kSfOff + NA * 512, sfb + (size_t)j * 512, 512, full(j));
+          }
+          kb = npre;
+          issued = npre;
         }
-        for (int kb = 0; kb < KB; ++kb, ++issued) {
+        for (; kb < KB; ++kb, ++issued) {
           const int s = issued % S;
           if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
             *abort_flag = 1;
