@@ -425,11 +425,9 @@ def extras(layer, wr, bias, xs, batches, flush, stream, args, device, keep):
     dn_ms, dn_n = prof["down"]
     fu_ms, fu_n = prof["ffn_fused"]
     if fu_n:
-        # decode batches run both GEMMs and the combine in one launch: its bytes are gate/up + down + the
-        # combine's reads of the y_pair rows and writes of the outputs
-        comb_bytes = sum(b * K * H * 4 + b * H * 2 for b in batches)
-        dom_bytes, dom_ms, dom_n = gu_bytes + dn_bytes + comb_bytes, fu_ms, fu_n
-        dom_name = "ffn decode: gate/up + SwiGLU + down x weight + combine (tcgen05, one launch)"
+        # decode batches run both GEMMs in one launch: its bytes are gate/up + down
+        dom_bytes, dom_ms, dom_n = gu_bytes + dn_bytes, fu_ms, fu_n
+        dom_name = "ffn fused gate/up + SwiGLU + down x weight (tcgen05, one launch)"
     else:
         dom_bytes, dom_ms, dom_n = gu_bytes, gu_ms, gu_n
         dom_name = "ffn gate/up GEMM + SwiGLU (tcgen05)"
@@ -608,6 +606,17 @@ def quantize_expert_mx(M, g, d, device):
     return qg, qd, sg, sd
 
 
+def layer_kernel_us(layer, x, wr, bias, flush, stream, reps):
+    """Per-kernel device time (us per forward) of one layer's forwards, from the library's own events."""
+    import mixture_experts_layer_24_b200 as M
+    M.moe_profile_enable(layer.ctx, True)
+    M.moe_profile_read(layer.ctx, reset=True)
+    time_forwards(layer, [x], wr, bias, flush, stream, reps)
+    pr = M.moe_profile_read(layer.ctx, reset=True)
+    M.moe_profile_enable(layer.ctx, False)
+    return {k: round(1000 * v[0] / reps, 2) for k, v in pr.items() if v[1]}
+
+
 def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
     """The same layer with e4m3 experts (128x128 block scales, quantised on the
     GPU from the bf16 weights): decode B=1, 8, 64 and a 4096-token chunk."""
@@ -631,7 +640,8 @@ def fp8_breakdown(keep, wr, bias, flush, stream, device, hbm):
         nbytes = t * fp8_bytes + E * H * 4 + T * H * 4
         out[f"fp8_B{T}" if T < 4096 else "fp8_prefill4096"] = {
             "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
-            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm,
+            "kernel_us": layer_kernel_us(layer, x, wr, bias, flush, stream, 2)}
     if layer.status():
         out["fp8_device_status"] = layer.status()
     layer.close()
@@ -665,7 +675,8 @@ def fp4_breakdown(keep, wr, bias, flush, stream, device, hbm):
         nbytes = t * fp4_bytes + E * H * 4 + T * H * 4
         out[f"fp4_B{T}" if T < 4096 else "fp4_prefill4096"] = {
             "us_per_layer": 1000 * ms, "tokens_per_s": T / (ms / 1000), "touched_experts": t,
-            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm}
+            "hbm_roofline_frac": (nbytes / (ms / 1000) / 1e9) / hbm,
+            "kernel_us": layer_kernel_us(layer, x, wr, bias, flush, stream, 2)}
     if layer.status():
         out["fp4_device_status"] = layer.status()
     layer.close()
@@ -716,6 +727,7 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
 
     def stream_of(layer, T, n_fill=4, n_time=20, base=610000):
         ms_tot, bound_tot, hits, routed, copied, touched_tot = 0.0, 0.0, 0, 0, 0, 0
+        ms_nocopy = []  # forwards that copied nothing (every routed host expert was cached, or none routed)
         for i in range(n_fill + n_time):
             x = synth.tokens(T, H, seed=SEED, device=device, first_token=base + 1000 * i)
             ms = time_forwards(layer, [x], wr, bias, flush, stream, 1)
@@ -723,6 +735,8 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
                 continue
             st = layer.stats()
             ms_tot += ms
+            if st["last_cold"] == 0:
+                ms_nocopy.append(ms)
             hits += st["last_hits"]
             routed += st["last_routed_cold"]
             copied += st["last_cold"]
@@ -732,6 +746,8 @@ def hotcold_breakdown(keep, wr, bias, flush, stream, device, hbm, n_hot=120, n_s
         return {"us_per_layer": 1000 * ms_tot / n_time, "tokens_per_s": T * n_time / (ms_tot / 1000),
                 "touched_experts_mean": touched_tot / n_time, "host_experts_routed_mean": routed / n_time,
                 "copied_experts_mean": copied / n_time, "hit_rate": hits / routed if routed else None,
+                "us_per_layer_no_copy": 1000 * statistics.median(ms_nocopy) if ms_nocopy else None,
+                "forwards_no_copy": len(ms_nocopy),
                 "roofline_frac": bound_tot / (ms_tot / 1000) if ms_tot > 0 else None,
                 "sample": f"{n_time} forwards over new tokens after {n_fill} that fill the cache"}
 

@@ -204,8 +204,7 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
   L.list_expert = take((2 * E + 64) * 4);
   L.list_map = take((2 * E + 64) * 4);
   L.nt_prefix = take((2 * E + 64) * 4);
-  // the fused FFN's counters, then the decode kernel's combine counts [kDecodeMaxT][H/128]
-  L.sched = take(((size_t)fused_sched_entries((int)E) + (size_t)kDecodeMaxT * (H / 128)) * 4);
+  L.sched = take((size_t)fused_sched_entries((int)E) * 4);
   L.x_perm = take(P * H * ((fp8 || mx) ? 1 : 2));
   L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
   L.h = take(mx ? 0 : P * I * 2);
@@ -749,7 +748,7 @@ moe_status_t permute_impl(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_
 // Decode FFN planned inside the kernel from the router's top-k (no permutation
 // kernel, no gathered x). The caller checked decode_path_ok().
 moe_status_t ffn_decode_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* idx, const float* topk_w,
-                             int T, float* y_pair, void* ws, cudaStream_t s, int* sched, void* out) {
+                             int T, float* y_pair, void* ws, cudaStream_t s, int* sched) {
   const moe_config_t& c = ctx->cfg;
   const WsLayout W = ws_layout(c, T);
   const int E = c.n_experts, P = T * c.top_k;
@@ -788,8 +787,6 @@ moe_status_t ffn_decode_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, con
   d.perm_src = at<int32_t>(ws, W.perm_src);
   d.perm_k = at<int32_t>(ws, W.perm_k);
   d.inv = at<int32_t>(ws, W.inv);
-  d.out = out;
-  d.comb_cnt = sched + fused_sched_entries(E);
   Prof p(ctx, MOE_PROF_FFN_FUSED, s);
   MOE_CUDA(launch_ffn_decode(xmap, hmaps, a, d, (c.intermediate / 128 + c.hidden / 128) * std::min(E, P), s,
                              ctx->chain));
@@ -1165,9 +1162,9 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
   const bool chain = ctx->chain;
   if (residency_device_path_ok(ctx, sl, x, T)) {
     // decode with host-resident experts: router -> cache plan -> copies of the missed experts (none when
-    // every routed expert is resident or cached) -> FFN planned from the top-k, combine inside
+    // every routed expert is resident or cached) -> FFN planned from the top-k -> combine
     int* sched = at<int>(ws, W.sched);
-    const int sched_n = fused_sched_entries(c.n_experts) + T * (c.hidden / 128);
+    const int sched_n = 1 + std::min(c.n_experts, T * c.top_k);
     if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n)) != MOE_OK) return st;
     {
       Prof p(ctx, MOE_PROF_PERMUTE, s);
@@ -1177,19 +1174,20 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
       Prof p(ctx, MOE_PROF_GATHER, s);
       MOE_CUDA(launch_residency_copy(sl->rdev, sl->spare, ctx->num_sms, s, chain));
     }
-    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched, out)) != MOE_OK) return st;
+    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched)) != MOE_OK) return st;
     sl->last_dev = true;
+    Prof p(ctx, MOE_PROF_COMBINE, s);
+    MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, chain));
     return MOE_OK;
   }
   if (decode_path_ok(ctx, sl, x, T)) {
-    // decode: router (which also zeroes the FFN's counters and combine counts) -> FFN planned from the
-    // top-k, with the combine inside the same launch
+    // decode: router (which also zeroes the FFN's counters) -> FFN planned from the top-k -> combine
     int* sched = at<int>(ws, W.sched);
-    const int sched_n = fused_sched_entries(c.n_experts) + T * (c.hidden / 128);
+    const int sched_n = 1 + std::min(c.n_experts, T * c.top_k);
     if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n)) != MOE_OK) return st;
-    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched, out)) != MOE_OK) return st;
-    (void)inv;
-    (void)chain;
+    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched)) != MOE_OK) return st;
+    Prof p(ctx, MOE_PROF_COMBINE, s);
+    MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, chain));
     return MOE_OK;
   }
   // route (first kernel: ordinary stream order with whatever came before)

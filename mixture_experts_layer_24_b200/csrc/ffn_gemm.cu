@@ -1023,9 +1023,8 @@ struct DecodeCfg {
   static constexpr uint32_t kAcc = 2 * TP;
   static constexpr uint32_t kTmemCols = tmem_cols_for(2 * kAcc);
   static constexpr int kMaxPairs = 512;
-  // plan: s_e, s_psrc, s_pk [kMaxPairs]; s_cnt[E], s_off[E+1], s_list[E]; s_t2p[TP]; scan[8]; s_run[E];
-  // s_inv[kMaxPairs]; combine: s_vp[kMaxPairs] (sorted row of each kept pair, -1 dropped), s_kv[TP] (kept pairs)
-  static size_t plan_bytes(int E) { return 4 * (5 * (size_t)kMaxPairs + 4 * (size_t)E + 1 + 2 * TP + 8); }
+  // plan: s_e, s_psrc, s_pk [kMaxPairs]; s_cnt[E], s_off[E+1], s_list[E]; s_t2p[TP]; scan[8]; s_run[E]; s_inv[kMaxPairs]
+  static size_t plan_bytes(int E) { return 4 * (4 * (size_t)kMaxPairs + 4 * (size_t)E + 1 + TP + 8); }
   static size_t smem(int E) {
     return 1024 + (size_t)kStages * kStageBytes + 8 * (2 * kStages + 4 + 2 * kRing) + 4 * kRing + 16 + 4 * TP +
            plan_bytes(E);
@@ -1102,8 +1101,6 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
   int* s_scan = s_t2p + TP;                               // [8]
   int* s_run = s_scan + 8;                                // [E] running count per expert (ranks)
   int* s_inv = s_run + E;                                 // [kMaxPairs] sorted place of pair i
-  int* s_vp = s_inv + C::kMaxPairs;                       // [kMaxPairs] sorted place of pair i if kept, else -1
-  int* s_kv = s_vp + C::kMaxPairs;                        // [TP] kept pairs of token t
 
   // ---------------------------------------------------------------- plan
   for (int i = tid; i < E; i += 192) s_cnt[i] = 0;
@@ -1162,15 +1159,8 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
     }
   }
   __syncthreads();
-  for (int i = tid; i < P; i += 192) s_vp[i] = (s_e[i] >= 0 && d.map_of[s_e[i]] >= 0) ? s_inv[i] : -1;
-  __syncthreads();
-  for (int t = tid; t < d.T; t += 192) {
-    int kv = 0;
-    for (int k = 0; k < K; ++k) kv += s_vp[t * K + k] >= 0 ? 1 : 0;
-    s_kv[t] = kv;
-  }
   if (blockIdx.x == 0)  // a pair of an unregistered expert is dropped: the combine skips inv = -1
-    for (int i = tid; i < P; i += 192) d.inv[i] = s_vp[i];
+    for (int i = tid; i < P; i += 192) d.inv[i] = (s_e[i] >= 0 && d.map_of[s_e[i]] < 0) ? -1 : s_inv[i];
   if (blockIdx.x == 0) {
     for (int e = tid; e < E; e += 192) {
       d.counts[e] = s_cnt[e];
@@ -1180,12 +1170,6 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
     for (int p = tid; p < s_off[E]; p += 192) {
       d.perm_src[p] = s_psrc[p];
       d.perm_k[p] = s_pk[p];
-    }
-    if (d.out) {  // a token all of whose pairs are dropped gets no down tile: its output is zero
-      __syncthreads();  // s_kv is complete
-      for (int t = 0; t < d.T; ++t)
-        if (s_kv[t] == 0)
-          for (int o = tid; o < a.H; o += 192) static_cast<__nv_bfloat16*>(d.out)[(size_t)t * a.H + o] = __float2bfloat16_rn(0.0f);
     }
   }
 
@@ -1479,46 +1463,6 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_decode_kernel(const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty(buf));
-      if (!gu && d.out) {
-        // Combine inside the launch: a (token, 128-column block) is complete when the down tiles of all its
-        // valid pairs have stored their y rows; the tile that completes it sums the token's pairs, k
-        // ascending from the first valid one, and rounds once to bf16 (the combine kernel's arithmetic).
-        __threadfence();         // this thread's y stores before the count (release)
-        named_bar_sync(1, 128);  // every epilogue thread's stores are fenced
-        if (r < cnt) {
-          const int t = s_psrc[row0 + r];
-          const int prev = atomicAdd(d.comb_cnt + t * md + mt, 1);
-          s_t2p[r] = prev == s_kv[t] - 1 ? t : -1;  // s_t2p is free during a down tile
-        }
-        named_bar_sync(1, 128);
-        bool any = false;
-        for (int n = 0; n < cnt; ++n) any |= s_t2p[n] >= 0;
-        if (any) __threadfence();  // the other tiles' y rows (acquire, after their fenced counts)
-        __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(d.out);
-        const int o = mt * 128 + r;
-        for (int n = 0; n < cnt; ++n) {
-          const int t = s_t2p[n];
-          if (t < 0) continue;  // block-uniform
-          const int* vp = s_vp + t * K;
-          float acc = 0.0f;
-          bool have = false;
-          for (int k0 = 0; k0 < K; k0 += 8) {  // eight rows' loads in flight, then the adds, k ascending
-            float yv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int p = k0 + u < K ? vp[k0 + u] : -1;
-              yv[u] = p >= 0 ? __ldcg(a.y_out + (size_t)p * a.H + o) : 0.0f;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              if (k0 + u >= K || vp[k0 + u] < 0) continue;
-              acc = have ? acc + yv[u] : yv[u];
-              have = true;
-            }
-          }
-          outp[(size_t)t * a.H + o] = __float2bfloat16_rn(acc);
-        }
-      }
       if (gu) {
         __threadfence();
         named_bar_sync(1, 128);
@@ -1889,6 +1833,65 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
         accg[i] = 0.0f;
         accu[i] = 0.0f;
       }
+      if constexpr (HALF <= 16) {
+        // Narrow tiles (decode): each warp loads only its own HALF columns, for G K blocks at once, then
+        // promotes them in K order; one TMEM round trip per G blocks instead of per block. A warp whose
+        // columns are all past the tile's pairs loads nothing.
+        constexpr int G = HALF <= 8 ? 4 : 2;
+        const bool mine = c0 < ti.nvalid;  // warp-uniform
+        for (int kb0 = 0; kb0 < KB; kb0 += G) {
+          const int ng = KB - kb0 < G ? KB - kb0 : G;
+          if (!aborted) {
+            bool ok = !*abort_flag;
+            for (int g = 0; g < ng && ok; ++g) ok = mbar_wait(pfull((kp + g) % NP), ((kp + g) / NP) & 1);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+              aborted = true;
+              if (lane == 0) {
+                *abort_flag = 1;
+                flag_status(a.status, MOE_DEV_TIMEOUT);
+              }
+            }
+          }
+          if (!aborted && mine) {
+            tc_fence_after();
+            uint32_t pg[G][HALF], pu[G][HALF];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              if (g < ng) {
+                const uint32_t pbase = tl + static_cast<uint32_t>(((kp + g) % NP) * 2 * BN) + c0;
+                if constexpr (HALF == 8) {
+                  tmem_ld8(pbase, pg[g]);
+                  if (gu) tmem_ld8(pbase + BN, pu[g]);
+                } else {
+                  tmem_ld16(pbase, pg[g]);
+                  if (gu) tmem_ld16(pbase + BN, pu[g]);
+                }
+              }
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              if (g < ng) {
+                const int kb = kb0 + g;
+                const float swg = s_w[kb];
+                const float swu = gu ? s_w[KB + kb] : 0.0f;
+#pragma unroll
+                for (int q = 0; q < HALF; ++q) {
+                  const float sa = s_act[(c0 + q) * KB + kb];
+                  accg[q] = fmaf(__uint_as_float(pg[g][q]), sa * swg, accg[q]);
+                  if (gu) accu[q] = fmaf(__uint_as_float(pu[g][q]), sa * swu, accu[q]);
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0)
+            for (int g = 0; g < ng; ++g) mbar_arrive(pempty((kp + g) % NP));
+          kp += ng;
+        }
+      } else {
       for (int kb = 0; kb < KB; ++kb, ++kp) {
         const int pb = kp % NP;
         if (!aborted) {
@@ -1933,6 +1936,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pempty(pb));
+      }
       }
       if (gu) {
         // h = bf16(silu(g) * u), then its e4m3 block code: amax over the tile's 128 rows per pair

@@ -127,8 +127,6 @@ struct DecodeArgs {
   int32_t* perm_src;        // [P]
   int32_t* perm_k;          // [P]
   int32_t* inv;             // [P]
-  void* out;                // [T, H] bf16: when set, the combine runs inside the launch (no combine kernel)
-  int* comb_cnt;            // [T * H/128] completion counts per (token, 128-column block), zeroed by the router
 };
 cudaError_t launch_ffn_decode(const CUtensorMap& xmap, const ActMaps& hmaps, const GemmArgs& a, const DecodeArgs& d,
                               int max_tiles, cudaStream_t s, bool pdl);
