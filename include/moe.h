@@ -83,7 +83,8 @@ typedef enum {
                             The pages' checkpoint ships FP4 experts (vLLM-Moet,
                             topairepos.com page, hybrid results table, row "quality,
                             paired against the native FP4 reference"); they name no
-                            block format, and this is the open one. HBM-resident only. */
+                            block format, and this is the open one. HBM-resident only;
+                            H and I multiples of 256. */
 } moe_wdtype_t;
 
 enum { MOE_LOC_HBM = 0, MOE_LOC_HOST_PINNED = 1 };

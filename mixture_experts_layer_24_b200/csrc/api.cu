@@ -225,6 +225,8 @@ moe_status_t check_cfg(const moe_config_t& c) {
   if (c.flags & ~MOE_FLAG_NO_PDL) return fail(MOE_ERR_INVALID_ARG, "unknown flag bits");
   if (c.hidden % 128 || c.intermediate % 128) return fail(MOE_ERR_UNSUPPORTED, "H and I must be multiples of 128");
   if (c.hidden > 8192 || c.intermediate > 8192) return fail(MOE_ERR_UNSUPPORTED, "H and I must be <= 8192");
+  if (c.wdtype == MOE_MXFP4 && ((c.hidden % (128 * kMxKC)) || (c.intermediate % (128 * kMxKC))))
+    return fail(MOE_ERR_UNSUPPORTED, "MXFP4 needs H and I multiples of 256 (two 128-deep K blocks per stage)");
   if (c.top_k > 32 || c.top_k > c.n_experts || c.n_experts > 1024)
     return fail(MOE_ERR_UNSUPPORTED, "need 1 <= K <= 32 and K <= E <= 1024");
   return MOE_OK;
@@ -279,17 +281,35 @@ moe_status_t encode_3d_bf16(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uin
   return MOE_OK;
 }
 
-// Packed E2M1 codes [rows, inner] (two per byte), box {128 elements, 128 rows}:
-// the copy lands unpacked (16 codes per 16 bytes) with the 128-byte swizzle.
-moe_status_t encode_2d_fp4(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
-  const cuuint64_t dims[2] = {inner, rows};
-  const cuuint64_t strides[1] = {inner / 2};
-  const cuuint32_t box[2] = {128u, 128u};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(ptr), dims, strides,
+// Packed E2M1 codes [rows, inner] (two per byte) as (128 elements, rows,
+// inner/128 blocks), box {128, 128, kMxKC}: one copy brings kMxKC K blocks of a
+// 128-row tile, each landing unpacked (16 codes per 16 bytes) with the
+// 128-byte swizzle.
+moe_status_t encode_3d_fp4(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows) {
+  const cuuint64_t dims[3] = {128, rows, inner / 128};
+  const cuuint64_t strides[2] = {inner / 2, 64};
+  const cuuint32_t box[3] = {128u, 128u, (cuuint32_t)kMxKC};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides,
                                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (E2M1) failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
+// Byte rows [rows, inner] (e4m3 codes) as (128 bytes, rows, inner/128 blocks),
+// box {128, box_rows, kMxKC}: kMxKC K blocks per copy, each a swizzled
+// box_rows x 128 B block.
+moe_status_t encode_3d_u8(moe_ctx_t* ctx, CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t rows,
+                          uint32_t box_rows) {
+  const cuuint64_t dims[3] = {128, rows, inner / 128};
+  const cuuint64_t strides[2] = {inner, 128};
+  const cuuint32_t box[3] = {128u, box_rows, (cuuint32_t)kMxKC};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = ctx->encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (3-D bytes) failed: " + std::to_string((int)r));
   return MOE_OK;
 }
 
@@ -299,9 +319,9 @@ moe_status_t make_entry(moe_ctx_t* ctx, MapEntry* me, const void* gu, const void
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   std::memset(me, 0, sizeof(*me));
   if (c.wdtype == MOE_MXFP4) {  // sgu / sdn: the blocked E8M0 scales
-    moe_status_t st = encode_2d_fp4(ctx, &me->gu, gu, c.hidden, 2ull * c.intermediate);
+    moe_status_t st = encode_3d_fp4(ctx, &me->gu, gu, c.hidden, 2ull * c.intermediate);
     if (st != MOE_OK) return st;
-    st = encode_2d_fp4(ctx, &me->dn, dn, c.intermediate, c.hidden);
+    st = encode_3d_fp4(ctx, &me->dn, dn, c.intermediate, c.hidden);
     if (st != MOE_OK) return st;
     me->s_gu = sgu;
     me->s_dn = sdn;
@@ -400,9 +420,9 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     std::memset(&xm, 0, sizeof(xm));
     std::memset(&hm, 0, sizeof(hm));
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
-      moe_status_t st = encode_2d(ctx, &xm.m[i], at<void>(ws, W.x_perm), true, c.hidden, P, rows);
+      moe_status_t st = encode_3d_u8(ctx, &xm.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows);
       if (st != MOE_OK) return st;
-      st = encode_2d(ctx, &hm.m[i], at<void>(ws, W.hq), true, c.intermediate, P, rows);
+      st = encode_3d_u8(ctx, &hm.m[i], at<void>(ws, W.hq), c.intermediate, P, rows);
       if (st != MOE_OK) return st;
     }
     GemmArgs a{};
@@ -1450,8 +1470,9 @@ moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, c
       const size_t gu_blk = (size_t)(2 * I / 128) * (H / 128) * 512, dn_blk = (size_t)(H / 128) * (I / 128) * 512;
       uint8_t* blk = nullptr;
       if (cudaMalloc(&blk, gu_blk + dn_blk) != cudaSuccess) return fail(MOE_ERR_OOM, "cudaMalloc of MXFP4 scales failed");
-      cudaError_t err = launch_mx_block_scales(static_cast<const uint8_t*>(s_gu_), 2 * I, H, blk, nullptr);
-      if (err == cudaSuccess) err = launch_mx_block_scales(static_cast<const uint8_t*>(s_dn_), H, I, blk + gu_blk, nullptr);
+      cudaError_t err = launch_mx_block_scales(static_cast<const uint8_t*>(s_gu_), 2 * I, H, I, blk, nullptr);
+      if (err == cudaSuccess)
+        err = launch_mx_block_scales(static_cast<const uint8_t*>(s_dn_), H, I, 0, blk + gu_blk, nullptr);
       if (err == cudaSuccess) err = cudaStreamSynchronize(nullptr);
       if (err != cudaSuccess) {
         cudaFree(blk);

@@ -18,14 +18,19 @@
 // weight rows x BN pairs per tile), persistent CTAs over (expert, row tile,
 // N tile), K blocks in increasing order, no split-K, per-tile MMA width
 // 16..BN, two TMEM accumulators so one tile's epilogue overlaps the next
-// tile's MMAs. One stage is one 128-wide K block:
-//   [A gate 16 KB][A up 16 KB (gate/up only)][B: BN x 128 B]
-//   [scales A gate 512 B][scales A up 512 B][scales B 512 B]
-// A (E2M1) arrives by TMA in the tensor cores' unpacked layout (16 codes per
-// 16 bytes, the 128-byte swizzle); HBM moves 4 bits per weight. The scale
-// blocks arrive by bulk copy and go to TMEM with tcgen05.cp (32x128b, copied
-// to all four lane quarters); the four 32-deep MMAs of a stage read scale
-// byte j = 0..3 of each row's word.
+// tile's MMAs. One stage is kMxKC (2) consecutive 128-deep K blocks:
+//   [A gate: KC x 16 KB][A up: KC x 16 KB (gate/up only)][B: KC x W x 128 B]
+//   [scales A: KC x (gate 512 B, up 512 B)][scales B: KC x 512 B]
+// fetched by five copies (four for down): one 3-D TMA copy per operand brings
+// all KC blocks, and the weight scales of gate and up for KC blocks sit
+// together in global memory (mx.cu), as do the activation scales, so one bulk
+// copy each brings them. The TMA unit's per-copy cost, not the bytes, bounds
+// one SM's streaming rate for small copies: with one K block and six copies
+// per stage the GEMMs streamed 2.5-3.1 TB/s. A (E2M1) arrives in the tensor
+// cores' unpacked layout (16 codes per 16 bytes, the 128-byte swizzle); HBM
+// moves 4 bits per weight. Before the four 32-deep MMAs of each K block its
+// scale blocks go to TMEM with tcgen05.cp (32x128b, copied to all four lane
+// quarters); the MMAs read scale byte j = 0..3 of each row's word.
 #include "common.cuh"
 #include "internal.h"
 #include "tile.cuh"
@@ -81,10 +86,12 @@ __device__ __forceinline__ int mx_scale_exp8(float amax) {
 template <int MODE, int BN>
 struct MxCfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr uint32_t kAOp = kABytes;                // 128 rows x 128 K, unpacked E2M1
+  static constexpr int KC = kMxKC;
+  static constexpr uint32_t kAOp = KC * kABytes;           // KC blocks of 128 rows x 128 K, unpacked E2M1
   static constexpr uint32_t kBOff = NA * kAOp;
-  static constexpr uint32_t kSfOff = kBOff + BN * 128;     // scale blocks: A gate, (A up), B
-  static constexpr uint32_t kStageRaw = kSfOff + (NA + 1) * 512;
+  static constexpr uint32_t kSfOff = kBOff + KC * BN * 128;  // weight scales (KC x NA blocks), then activation
+  static constexpr uint32_t kSfBOff = kSfOff + KC * NA * 512;
+  static constexpr uint32_t kStageRaw = kSfBOff + KC * 512;
   static constexpr uint32_t kStageBytes = (kStageRaw + 1023u) & ~1023u;  // next stage's A stays 1024-aligned
   static constexpr int kStagesFit = (220 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -102,9 +109,11 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
   using C = MxCfg<MODE, BN>;
   constexpr int NA = C::NA, NBUF = C::NBUF, S = C::kStages;
   constexpr uint32_t STAGE = C::kStageBytes, ACC = C::kAcc;
+  constexpr int KC = C::KC;
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
   const int Kdim = MODE == kGateUp ? a.H : a.I;
-  const int KB = Kdim / 128;  // stages (128-wide K blocks) per tile
+  const int KB = Kdim / 128;  // 128-deep K blocks per tile
+  const int KS = KB / KC;     // stages per tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (!a.plan_ready) {
@@ -166,42 +175,43 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
         decode_tile_at(a, m_tiles, BN, tile, ti);
         const int wi = tile_width_index(ti.nvalid, BN);
         const void* amap = &act.m[wi];
-        const uint32_t stage_tx = NA * 8192u + (16u << wi) * 128u + (NA + 1) * 512u;  // A: 128 x 128 x 4 bits
+        // per stage: KC blocks of A (128 x 128 x 4 bits each), of B and of the scales
+        const uint32_t stage_tx = KC * (NA * 8192u + (16u << wi) * 128u + NA * 512u + 512u);
         const uint64_t pol_w = ti.nti > 1 ? pol_shared : pol_once;
         const MapEntry* me = a.maps + ti.mapi;
         const void* wmap = MODE == kGateUp ? static_cast<const void*>(&me->gu) : static_cast<const void*>(&me->dn);
-        const uint8_t* sfa = reinterpret_cast<const uint8_t*>(MODE == kGateUp ? me->s_gu : me->s_dn);
-        const uint8_t* sfa0 = sfa + (size_t)ti.mt * KB * 512;
-        const uint8_t* sfa1 = sfa + (size_t)(m_tiles + ti.mt) * KB * 512;  // up rows start at row I
+        // weight scales: [m tile][K block][NA][512] (gate and up of a K block side by side)
+        const uint8_t* sfa = reinterpret_cast<const uint8_t*>(MODE == kGateUp ? me->s_gu : me->s_dn) +
+                             (size_t)ti.mt * KB * NA * 512;
         const uint8_t* sfb = a.act_sfb + (size_t)ti.ng * KB * 512;
         tensormap_acquire(wmap);
-        int kb = 0;
+        auto issue_w = [&](uint32_t st, int ks) {
+          tma_load_3d_hint(st, wmap, full(issued % S), 0, ti.mt * 128, ks * KC, pol_w);
+          if (MODE == kGateUp) tma_load_3d_hint(st + C::kAOp, wmap, full(issued % S), 0, a.I + ti.mt * 128, ks * KC, pol_w);
+          bulk_load(st + C::kSfOff, sfa + (size_t)ks * KC * NA * 512, KC * NA * 512, full(issued % S));
+        };
+        auto issue_x = [&](uint32_t st, int ks, uint32_t bar) {
+          tma_load_3d(st + C::kBOff, amap, bar, 0, ti.row0, ks * KC);
+          bulk_load(st + C::kSfBOff, sfb + (size_t)ks * KC * 512, KC * 512, bar);
+        };
+        int ks = 0;
         if (first) {
           first = false;
           // the plan is complete: the first stages' weights and weight scales go out before waiting for the
           // kernel that writes the activations and their scales
-          const int npre = a.plan_ready ? (KB < S ? KB : S) : 0;
-          for (int j = 0; j < npre; ++j) {
-            const uint32_t st = base + j * STAGE;
+          const int npre = a.plan_ready ? (KS < S ? KS : S) : 0;
+          for (int j = 0; j < npre; ++j, ++issued) {
             mbar_arrive_expect_tx(full(j), stage_tx);
-            tma_load_2d_hint(st, wmap, full(j), j * 128, ti.mt * 128, pol_w);
-            if (MODE == kGateUp) tma_load_2d_hint(st + C::kAOp, wmap, full(j), j * 128, a.I + ti.mt * 128, pol_w);
-            bulk_load(st + C::kSfOff, sfa0 + (size_t)j * 512, 512, full(j));
-            if (MODE == kGateUp) bulk_load(st + C::kSfOff + 512, sfa1 + (size_t)j * 512, 512, full(j));
+            issue_w(base + j * STAGE, j);
           }
           if (a.plan_ready) {
             pdl_wait();
             pdl_trigger();
           }
-          for (int j = 0; j < npre; ++j) {
-            const uint32_t st = base + j * STAGE;
-            tma_load_2d(st + C::kBOff, amap, full(j), j * 128, ti.row0);
-            bulk_load(st + C::kSfOff + NA * 512, sfb + (size_t)j * 512, 512, full(j));
-          }
-          kb = npre;
-          issued = npre;
+          for (int j = 0; j < npre; ++j) issue_x(base + j * STAGE, j, full(j));
+          ks = npre;
         }
-        for (; kb < KB; ++kb, ++issued) {
+        for (; ks < KS; ++ks, ++issued) {
           const int s = issued % S;
           if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
             *abort_flag = 1;
@@ -210,12 +220,8 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
           }
           const uint32_t st = base + s * STAGE;
           mbar_arrive_expect_tx(full(s), stage_tx);
-          tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
-          if (MODE == kGateUp) tma_load_2d_hint(st + C::kAOp, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
-          tma_load_2d(st + C::kBOff, amap, full(s), kb * 128, ti.row0);
-          bulk_load(st + C::kSfOff, sfa0 + (size_t)kb * 512, 512, full(s));
-          if (MODE == kGateUp) bulk_load(st + C::kSfOff + 512, sfa1 + (size_t)kb * 512, 512, full(s));
-          bulk_load(st + C::kSfOff + NA * 512, sfb + (size_t)kb * 512, 512, full(s));
+          issue_w(st, ks);
+          issue_x(st, ks, full(s));
         }
       }
       // every copy this thread issued has landed before the CTA may exit
@@ -246,7 +252,8 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
         decode_tile_at(a, m_tiles, BN, tile, ti);
         const int width = 16 << tile_width_index(ti.nvalid, BN);
         bool ok = true;
-        for (int kb = 0; kb < KB; ++kb, ++consumed) {
+        const uint32_t chunk_b = (uint32_t)width * 128u;  // a 3-D box lands its K blocks densely
+        for (int ks = 0; ks < KS; ++ks, ++consumed) {
           const int s = consumed % S;
           if (!mbar_wait(full(s), (consumed / S) & 1)) {
             ok = false;
@@ -254,20 +261,24 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
           }
           tc_fence_after();
           const uint32_t st = base + s * STAGE;
-          // this stage's scales to TMEM; tcgen05 operations of one thread run in issue order, so the
-          // copies land after the previous stage's MMAs have read the same columns
-          tc_cp_sf(sf_a0, sf_block_desc(st + C::kSfOff));
-          if (MODE == kGateUp) tc_cp_sf(sf_a1, sf_block_desc(st + C::kSfOff + 512));
-          tc_cp_sf(sf_b, sf_block_desc(st + C::kSfOff + NA * 512));
 #pragma unroll
-          for (uint32_t k = 0; k < 4; ++k) {
-            const uint32_t idesc = mx_instr_desc(width, k);
-            const uint64_t bdesc = sw128_kmajor_desc(st + C::kBOff + k * 32);
-            const uint32_t acc = (kb | (int)k) != 0 ? 1u : 0u;
-            tc_mma_mx(d, sw128_kmajor_desc(st + k * 32), bdesc, idesc, sf_a0 | (k << 30), sf_b | (k << 30), acc);
-            if (MODE == kGateUp)
-              tc_mma_mx(d + BN, sw128_kmajor_desc(st + C::kAOp + k * 32), bdesc, idesc, sf_a1 | (k << 30),
+          for (int c = 0; c < KC; ++c) {
+            // this block's scales to TMEM; tcgen05 operations of one thread run in issue order, so the copies
+            // land after the previous block's MMAs have read the same columns
+            tc_cp_sf(sf_a0, sf_block_desc(st + C::kSfOff + c * NA * 512));
+            if (MODE == kGateUp) tc_cp_sf(sf_a1, sf_block_desc(st + C::kSfOff + c * NA * 512 + 512));
+            tc_cp_sf(sf_b, sf_block_desc(st + C::kSfBOff + c * 512));
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+              const uint32_t idesc = mx_instr_desc(width, k);
+              const uint64_t bdesc = sw128_kmajor_desc(st + C::kBOff + c * chunk_b + k * 32);
+              const uint32_t acc = (ks | c | (int)k) != 0 ? 1u : 0u;
+              tc_mma_mx(d, sw128_kmajor_desc(st + c * kABytes + k * 32), bdesc, idesc, sf_a0 | (k << 30),
                         sf_b | (k << 30), acc);
+              if (MODE == kGateUp)
+                tc_mma_mx(d + BN, sw128_kmajor_desc(st + C::kAOp + c * kABytes + k * 32), bdesc, idesc,
+                          sf_a1 | (k << 30), sf_b | (k << 30), acc);
+            }
           }
           tc_commit(empty(s));
         }

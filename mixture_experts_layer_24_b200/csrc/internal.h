@@ -19,10 +19,10 @@ struct alignas(64) MapEntry {
   // bf16:  3-D maps (64 elements, rows, K/64 chunks), box {64, 128, kc} with
   //        kc = 1 (gu, dn) and kc = 2 (gu2, dn2);
   // FP8:   2-D maps in gu / dn, box {128 B of K, 128 rows};
-  // MXFP4: 2-D maps in gu / dn over the packed E2M1 codes (two per byte),
-  //        box {128 elements, 128 rows}, landing unpacked (16 codes per 16 B);
-  //        s_gu / s_dn point at the E8M0 scales in the tensor cores' 512-byte
-  //        block layout, [rows/128][K/128][512] bytes.
+  // MXFP4: 3-D maps in gu / dn over the packed E2M1 codes (two per byte),
+  //        (128 elements, rows, K/128 blocks), box {128, 128, kMxKC}, each
+  //        block landing unpacked (16 codes per 16 B); s_gu / s_dn point at the
+  //        E8M0 scales in the tensor cores' 512-byte block layout (mx.cu).
   CUtensorMap gu;   // w_gu [2I, H]
   CUtensorMap dn;   // w_dn [H, I]
   CUtensorMap gu2;
@@ -219,7 +219,10 @@ cudaError_t launch_ep_gather_rows_f32(const float* src, const int32_t* idx, int 
 // MXFP4 (mx.cu, ffn_mxfp4.cu).
 cudaError_t launch_quant_mx(const void* src, int rows, int cols, int elem_e4m3, uint8_t* q, uint8_t* scales,
                             cudaStream_t s);
-cudaError_t launch_mx_block_scales(const uint8_t* scales, int rows, int K, uint8_t* blocked, cudaStream_t s);
+cudaError_t launch_mx_block_scales(const uint8_t* scales, int rows, int K, int split_rows, uint8_t* blocked,
+                                   cudaStream_t s);
+// K blocks (128 deep) per pipeline stage of the MXFP4 GEMMs: one 3-D copy per operand brings them all.
+constexpr int kMxKC = 2;
 cudaError_t launch_quant_mx_pairs(const void* x, const int32_t* perm_src, const int32_t* offsets,
                                   const int32_t* nt_prefix, int E, int bn, int P, int H, uint8_t* xq, uint8_t* sfb,
                                   cudaStream_t s, bool pdl);

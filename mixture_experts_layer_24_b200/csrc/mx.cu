@@ -19,9 +19,11 @@
 //   - plain scales are [rows, cols/32] bytes;
 //   - the tensor cores take scales as 512-byte blocks, one per 128 rows x 4
 //     scales (128 K elements): byte 16*(r%32) + 4*(r/32) + j holds row r's
-//     scale j. Weight scales are kept as [rows/128][K/128][512]; activation
-//     scales as [N tile][K/128][512], row r of the block being the tile's
-//     r-th pair.
+//     scale j. Down-projection scales are kept as [H/128][I/128][512]; gate/up
+//     scales as [I/128][H/128][2][512], the gate block of row tile mt beside
+//     the up block of the same tile (rows I + 128 mt ..), so that one copy
+//     brings both for several K blocks; activation scales as
+//     [N tile][K/128][512], row r of the block being the tile's r-th pair.
 #include "common.cuh"
 #include "internal.h"
 
@@ -133,23 +135,33 @@ cudaError_t launch_quant_mx(const void* src, int rows, int cols, int elem_e4m3, 
   return cudaGetLastError();
 }
 
-// Plain weight scales [rows, K/32] -> blocked [rows/128][K/128][512]; one
-// thread per (row, 4-scale word).
+// Plain weight scales [rows, K/32] -> blocked; one thread per (row, 4-scale
+// word). split_rows = 0: [rows/128][K/128][512]; split_rows = I (gate/up,
+// rows = 2I): [I/128][K/128][2][512], rows >= I going to the second block.
 __global__ void __launch_bounds__(256) mx_block_scales_kernel(const uint8_t* __restrict__ s, int rows, int K,
-                                                               uint8_t* __restrict__ blk) {
+                                                               int split_rows, uint8_t* __restrict__ blk) {
   const int nkb = K / 128;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (int64_t)rows * nkb) return;
   const int r = (int)(i / nkb), kb = (int)(i - (int64_t)r * nkb);
   const uint32_t w = *reinterpret_cast<const uint32_t*>(s + (size_t)r * (K / 32) + 4 * kb);
-  const int rt = r / 128, rr = r - rt * 128;
-  *reinterpret_cast<uint32_t*>(blk + ((size_t)rt * nkb + kb) * 512 + 16 * (rr % 32) + 4 * (rr / 32)) = w;
+  const int rr = r % 128;
+  size_t block;
+  if (split_rows > 0) {
+    const int which = r >= split_rows ? 1 : 0;
+    const int mt = (r - which * split_rows) / 128;
+    block = ((size_t)mt * nkb + kb) * 2 + which;
+  } else {
+    block = (size_t)(r / 128) * nkb + kb;
+  }
+  *reinterpret_cast<uint32_t*>(blk + block * 512 + 16 * (rr % 32) + 4 * (rr / 32)) = w;
 }
 
-cudaError_t launch_mx_block_scales(const uint8_t* scales, int rows, int K, uint8_t* blocked, cudaStream_t s) {
+cudaError_t launch_mx_block_scales(const uint8_t* scales, int rows, int K, int split_rows, uint8_t* blocked,
+                                   cudaStream_t s) {
   const int64_t n = (int64_t)rows * (K / 128);
   if (n <= 0) return cudaSuccess;
-  mx_block_scales_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, rows, K, blocked);
+  mx_block_scales_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(scales, rows, K, split_rows, blocked);
   return cudaGetLastError();
 }
 

@@ -69,6 +69,16 @@ def test_host_side_argument_checks(lib):
     assert M.MOE_SLOTS_LRU != M.MOE_SLOTS_PER_CALL
 
 
+def test_mxfp4_shape_limits_checked_on_the_host(lib):
+    """MXFP4 stages hold two 128-deep K blocks: H and I must be multiples of 256,
+    refused before any CUDA call."""
+    import mixture_experts_layer_24_b200 as M
+    for H, I in ((384, 256), (256, 384)):
+        with pytest.raises(M.MoeError) as e:
+            M.moe_ctx_create(H, 8, 2, I, M.MOE_MXFP4)
+        assert e.value.status == 2 and b"256" in lib.moe_last_error()
+
+
 def test_ctx_create_without_gpu_fails_cleanly(lib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")

@@ -110,7 +110,7 @@ def test_mx_quantizer_bit_exact(elem, rows, cols):
 
 
 @pytest.mark.parametrize("T,H,E,K,I,zipf", [(16, 256, 8, 2, 512, None), (1, 512, 8, 4, 256, None),
-                                             (5, 1024, 16, 8, 512, 1.1), (100, 512, 12, 4, 384, None),
+                                             (5, 1024, 16, 8, 512, 1.1), (100, 512, 12, 4, 768, None),
                                              (300, 256, 6, 3, 256, 1.1)])
 def test_forward_mxfp4_matches_oracle(T, H, E, K, I, zipf):
     case = MxCase(T, H, E, K, I, seed=T + 7, zipf=zipf)
