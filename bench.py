@@ -68,7 +68,7 @@ def peaks():
 # time; they are reported only while the sources still hash the same.
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_decode_sweep.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "mixture_experts_layer_24_b200", "csrc", f)
-                  for f in ("ffn_gemm.cu", "common.cuh", "internal.h")]
+                  for f in ("ffn_decode.cu", "common.cuh", "tile.cuh", "internal.h")]
 
 
 def kernel_sources_sha256():

@@ -101,6 +101,9 @@ struct alignas(64) ActMaps {
 // max_tiles bounds the grid (CTAs past the real tile count exit at once).
 cudaError_t launch_ffn_gemm(int mode, int wdtype, int bn, const CUtensorMap& act_map, const ActMaps* act_maps,
                             const GemmArgs& a, int max_tiles, cudaStream_t s, bool pdl);
+// The FP8 GEMMs behind launch_ffn_gemm (bn 16, 32 or 64).
+cudaError_t launch_ffn_fp8(int mode, int bn, const ActMaps& maps, const GemmArgs& a, int max_tiles, cudaStream_t s,
+                           bool pdl);
 
 // Fused decode FFN (bf16, bn <= 64): gate/up and down tiles of one forward in
 // one persistent launch with a dynamic tile queue. xmaps: x_perm with one K

@@ -36,7 +36,7 @@ def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
 
 def test_source_hash_covers_the_kernel_files():
     assert all(os.path.exists(p) for p in bench.KERNEL_SOURCES)
-    assert any(p.endswith("ffn_gemm.cu") for p in bench.KERNEL_SOURCES)
+    assert any(p.endswith("ffn_decode.cu") for p in bench.KERNEL_SOURCES)
     assert len(bench.kernel_sources_sha256()) == 64
 
 
