@@ -529,8 +529,8 @@ def run_profile_case(kind):
     touched) and 64 tokens; "t1": 8 experts (top-8 of 8, all touched, 400 MB)
     and one token -- the per-launch shape of batch-1 decode; "p2048": 48
     experts and a 2048-token prefill chunk under the Zipf logit prior;
-    "f64" / "f2048": "t64" / "p2048" with e4m3 experts; "m64" / "m2048": with MXFP4
-    experts; "r4096": the router
+    "f64" / "f2048" / "f1": "t64" / "p2048" / "t1" with e4m3 experts; "m64" /
+    "m2048" / "m1": with MXFP4 experts; "r4096": the router
     alone (384 experts, 4096 tokens, Zipf prior), three calls."""
     import mixture_experts_layer_24_b200 as M
     device = torch.device("cuda", 0)
@@ -548,9 +548,9 @@ def run_profile_case(kind):
         layer.close()
         return 1 if st else 0
     E_s, T_s = {"t64": (32, 64), "t1": (8, 1), "p2048": (48, 2048), "f64": (32, 64), "f2048": (48, 2048),
-                "m64": (32, 64), "m2048": (48, 2048)}[kind]
-    fp8 = kind in ("f64", "f2048")
-    mx = kind in ("m64", "m2048")
+                "f1": (8, 1), "m64": (32, 64), "m2048": (48, 2048), "m1": (8, 1)}[kind]
+    fp8 = kind in ("f64", "f2048", "f1")
+    mx = kind in ("m64", "m2048", "m1")
     wd = M.MOE_FP8_E4M3_B128 if fp8 else (M.MOE_MXFP4 if mx else M.MOE_BF16)
     layer = M.MoeLayer(H, E_s, K, I, wdtype=wd, device=device)
     keep = []
@@ -873,7 +873,7 @@ def main():
     ap.add_argument("--eager", action="store_true", help="no CUDA graphs in the timed region")
     ap.add_argument("--quick", action="store_true", help="skip the FP8 and hot/cold breakdowns")
     ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
-    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "m64", "m2048", "r4096"],
+    ap.add_argument("--profile-case", nargs="?", const="t64", default=None, choices=["t64", "t1", "p2048", "f64", "f2048", "f1", "m64", "m2048", "m1", "r4096"],
                     help="small ncu case, 3 forwards, no timing: t64 = 32 experts x 64 tokens, t1 = 8 experts x 1 token")
     args = ap.parse_args()
     if args.profile_case:

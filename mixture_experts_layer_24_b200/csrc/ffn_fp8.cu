@@ -13,59 +13,92 @@
 //
 // Warp roles: warps 0..7 epilogue (4 TMEM lane quarters x 2 column groups),
 // warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tile.cuh"
 
 namespace moe {
 
+// One TMEM load of N consecutive fp32 columns of the thread's own lane (N = 8, 16 or 32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32) tmem_ld32(taddr, r);
+  else if constexpr (N == 16) tmem_ld16(taddr, r);
+  else tmem_ld8(taddr, r);
+}
+
 template <int MODE, int BN>
 struct Fp8Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
   static constexpr uint32_t kStageBytes = NA * kABytes + BN * 128;  // one 128-wide K block
   static constexpr int kMaxKB = 64;                                   // K / 128 <= 64 (K <= 8192)
-  // activation scales [BN][KB], weight scales [2][KB], routing weights [BN]
-  static constexpr uint32_t kScaleBytes = BN * kMaxKB * 4 + 2 * kMaxKB * 4 + BN * 4;
-  static constexpr int kStagesRaw = (220 * 1024 - (int)kScaleBytes) / (int)kStageBytes;
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // per tile: the combined scales s_act[pair, kb] * s_w[row block, kb] as [NA][KB][BN] (a warp's columns of one
+  // K block are consecutive, so they load as 16-byte vectors), then the routing weights [BN]
+  __host__ __device__ static constexpr uint32_t scale_bytes(int KB) { return (uint32_t)(NA * KB * BN * 4 + BN * 4); }
+  static int stages(int KB) {
+    const int s = (int)((220 * 1024 - scale_bytes(KB)) / kStageBytes);
+    return s > 8 ? 8 : s;
+  }
   // TMEM buffers of per-K-block partial sums (the MMA runs up to NP blocks ahead of the promotion)
   static constexpr int kNpRaw = 512 / (NA * BN);
   static constexpr int NP = kNpRaw > 8 ? 8 : kNpRaw;
   static constexpr uint32_t kTmemCols = tmem_cols_for(NP * NA * BN);
-  static constexpr size_t kSmem = 1024 + kStages * kStageBytes + kScaleBytes + 8 * (2 * kStages + 2 * NP) + 64;
+  static size_t smem(int KB) { return 1024 + stages(KB) * kStageBytes + scale_bytes(KB) + 8 * (2 * stages(KB) + 2 * NP) + 64; }
   // epilogue warps (4 TMEM lane quarters x EW/4 column groups); 16 at BN = 64
   // measured no faster than 8
   static constexpr int EW = 8;
-  static_assert(kStages >= 2 && NP >= 2, "FP8 pipeline needs two stages and two partial buffers");
+  static constexpr int kThreads = 32 * (EW + 1 + NA);  // + producer + one MMA issuer per accumulator
+  static constexpr int HALF = BN * 4 / EW;             // columns per epilogue warp: 8, 16 or 32
+  static_assert(NP >= 2, "FP8 pipeline needs two partial buffers");
 };
 
 // ======================================================================= fp8
 // Persistent, like the bf16 kernel: one CTA per SM walks tiles blockIdx.x,
 // +gridDim.x, ...; the shared-memory pipeline and a ring of NP TMEM buffers
 // for the per-K-block partial sums run on across tile boundaries. Per tile the
-// epilogue warps stage the tile's activation and weight scales (and, for down,
-// the routing weights) in shared memory, then promote every K block's partial
-// sum in registers, K blocks in increasing order. The MMA width adapts per
-// tile (16 .. BN). After a failed (timed-out) wait a warp stops working but
-// keeps its control flow, so the epilogue warps always meet at the same named
+// epilogue warps build the tile's table of combined scales s_act * s_w (and,
+// for down, the routing weights) in shared memory, then promote every K
+// block's partial sum in registers, K blocks in increasing order: one TMEM
+// load of the warp's columns per operand, one wait, then per column one fma
+// with the table's scale (the same fp32 product the promotion always used,
+// so the results do not change). Gate and up MMAs are issued by two threads
+// (warps EW+1 and EW+2), each committing to the stage and partial barriers
+// (which count both): every tcgen05 instruction holds its issuing thread for
+// tens of cycles, and at BN = 64 the eight MMAs of a K block took about as
+// long to issue as the promotion took. The MMA width adapts per tile
+// (16 .. BN). After a failed (timed-out) wait a warp stops working but keeps
+// its control flow, so the epilogue warps always meet at the same named
 // barriers.
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
+__global__ void __launch_bounds__(Fp8Cfg<MODE, BN>::kThreads, 1)
     ffn_fp8_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
   using C = Fp8Cfg<MODE, BN>;
-  constexpr int NA = C::NA, S = C::kStages, NP = C::NP;
+  constexpr int NA = C::NA, NP = C::NP;
   constexpr uint32_t STAGE = C::kStageBytes;
   constexpr int EW = C::EW;            // epilogue warps: 4 TMEM lane quarters x EW/4 column groups
   constexpr int EPT = 32 * EW;         // epilogue threads
-  constexpr int PW = EW, MW = EW + 1;  // producer warp, MMA warp
-  constexpr int HALF = BN * 4 / EW;    // columns per epilogue warp
-  constexpr int NCH = HALF >= 16 ? HALF / 16 : 1;
-  constexpr int CW = HALF >= 16 ? 16 : HALF;  // columns used per TMEM load
+  constexpr int PW = EW, MW = EW + 1;  // producer warp, first MMA warp
+  constexpr int HALF = C::HALF;        // columns per epilogue warp
 
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
   const int KD = MODE == kGateUp ? a.H : a.I;  // reduction length
   const int KB = KD / 128;
+  const int S = a.stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (!a.plan_ready) {
@@ -83,24 +116,23 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  float* s_act = reinterpret_cast<float*>(gbase + S * STAGE);  // [BN][KB] activation scales of the tile's pairs
-  float* s_w = s_act + BN * C::kMaxKB;                         // [NA][KB] weight scales of the tile's row blocks
-  float* wcol = s_w + 2 * C::kMaxKB;                           // [BN] routing weights (down)
-  const uint32_t bars = base + S * STAGE + C::kScaleBytes;     // full[S], empty[S], pfull[NP], pempty[NP]
+  float* cs = reinterpret_cast<float*>(gbase + S * STAGE);  // [NA][KB][BN] combined scales of the tile
+  float* wcol = cs + NA * KB * BN;                          // [BN] routing weights (down)
+  const uint32_t bars = base + S * STAGE + C::scale_bytes(KB);  // full[S], empty[S], pfull[NP], pempty[NP]
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
   auto pfull = [&](int b) { return bars + 8u * (2 * S + b); };
   auto pempty = [&](int b) { return bars + 8u * (2 * S + NP + b); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + C::kScaleBytes + 8 * (2 * S + 2 * NP));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * STAGE + C::scale_bytes(KB) + 8 * (2 * S + 2 * NP));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(empty(s), NA);
     }
     for (int b = 0; b < NP; ++b) {
-      mbar_init(pfull(b), 1);
+      mbar_init(pfull(b), NA);
       mbar_init(pempty(b), EW);
     }
     *abort_flag = 0;
@@ -119,7 +151,8 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
-      int issued = 0;
+      int issued = 0, ps = 0;
+      uint32_t pphase = 0;
       bool first = true;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         TileInfo ti;
@@ -148,19 +181,26 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
           for (int j = 0; j < npre; ++j) tma_load_2d(base + j * STAGE + NA * kABytes, amap, full(j), j * 128, ti.row0);
           kb = npre;
           issued = npre;
+          ps = npre == S ? 0 : npre;
+          pphase = npre == S ? 1u : 0u;
         }
         for (; kb < KB; ++kb, ++issued) {
-          const int s = issued % S;
-          if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
+          // slot ps = issued % S; its previous fill was round issued / S - 1 (S is a launch value: running
+          // counters instead of divisions)
+          if (issued >= S && !mbar_wait(empty(ps), pphase ^ 1u)) {
             *abort_flag = 1;
             flag_status(a.status, MOE_DEV_TIMEOUT);
             break;
           }
-          const uint32_t st = base + s * STAGE;
-          mbar_arrive_expect_tx(full(s), stage_tx);
-          tma_load_2d_hint(st, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
-          if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(s), kb * 128, a.I + ti.mt * 128, pol_w);
-          tma_load_2d(st + NA * kABytes, amap, full(s), kb * 128, ti.row0);
+          const uint32_t st = base + ps * STAGE;
+          mbar_arrive_expect_tx(full(ps), stage_tx);
+          tma_load_2d_hint(st, wmap, full(ps), kb * 128, ti.mt * 128, pol_w);
+          if (MODE == kGateUp) tma_load_2d_hint(st + kABytes, wmap, full(ps), kb * 128, a.I + ti.mt * 128, pol_w);
+          tma_load_2d(st + NA * kABytes, amap, full(ps), kb * 128, ti.row0);
+          if (++ps == S) {
+            ps = 0;
+            pphase ^= 1u;
+          }
         }
       }
       // every copy this thread issued has landed before the CTA may exit
@@ -169,34 +209,39 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
       pdl_wait();
       pdl_trigger();
     }
-  } else if (warp == MW) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= MW) {
+    // ------------------------------------------------------------ MMA issuers (gate or down; up)
     if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
-    if (lane == 0) {
-      int consumed = 0, kp = 0;
+    const int who = warp - MW;
+    if (lane == 0 && who < NA) {
+      int cslot = 0, kp = 0;  // consumed stage slot (running), K blocks consumed
+      uint32_t cphase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
         decode_tile_at(a, m_tiles, BN, tile, ti);
         const int width = 16 << tile_width_index(ti.nvalid, BN);
         const uint32_t idesc = instr_desc(128, width, 0u);
-        for (int kb = 0; kb < KB; ++kb, ++consumed, ++kp) {
-          const int s = consumed % S, pb = kp % NP;
-          ok = mbar_wait(full(s), (consumed / S) & 1);
+        for (int kb = 0; kb < KB; ++kb, ++kp) {
+          const int pb = kp % NP;
+          ok = mbar_wait(full(cslot), cphase);
           if (ok && kp >= NP) ok = mbar_wait(pempty(pb), ((kp / NP) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t st = base + s * STAGE;
-          const uint32_t d = tmem + static_cast<uint32_t>(pb * NA * BN);
+          const uint32_t st = base + cslot * STAGE;
+          const int s = cslot;
+          if (++cslot == S) {
+            cslot = 0;
+            cphase ^= 1u;
+          }
+          const uint32_t d = tmem + static_cast<uint32_t>(pb * NA * BN + who * BN);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t bdesc = sw128_kmajor_desc(st + NA * kABytes + k * 32);
-            const uint32_t acc = k != 0 ? 1u : 0u;
-            tc_mma_e4m3(d, sw128_kmajor_desc(st + k * 32), bdesc, idesc, acc);
-            if (MODE == kGateUp) tc_mma_e4m3(d + BN, sw128_kmajor_desc(st + kABytes + k * 32), bdesc, idesc, acc);
+            tc_mma_e4m3(d, sw128_kmajor_desc(st + who * kABytes + k * 32), bdesc, idesc, k != 0 ? 1u : 0u);
           }
           tc_commit(empty(s));
           tc_commit(pfull(pb));
@@ -227,15 +272,16 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
       const int width = 16 << tile_width_index(ti.nvalid, BN);
       const MapEntry* me = a.maps + ti.mapi;
       const float* sw = MODE == kGateUp ? me->s_gu : me->s_dn;
-      named_bar_sync(1, EPT);  // the previous tile's readers are done with the scale tables
-      for (int i = et; i < BN * KB; i += EPT) {
-        const int n = i / KB, kb = i - n * KB;
-        s_act[n * KB + kb] = n < ti.nvalid ? a.act_scale[(size_t)(ti.row0 + n) * KB + kb] : 0.0f;
-      }
-      for (int i = et; i < NA * KB; i += EPT) {
-        const int which = i / KB, kb = i - which * KB;
+      named_bar_sync(1, EPT);  // the previous tile's readers are done with the tables
+      // combined scales [which][kb][n] of the tile's pairs, n fastest (each pair's row of activation scales
+      // stays in L1); columns n >= nvalid keep stale values: their sums are never stored
+      const int nv = ti.nvalid;
+      for (int i = et; i < NA * KB * nv; i += EPT) {
+        const int n = i % nv, t = i / nv;
+        const int kb = t % KB, which = t / KB;
         const int rb = which == 0 ? ti.mt : a.I / 128 + ti.mt;  // gate (or down) row block, then up
-        s_w[which * KB + kb] = sw[(size_t)rb * KB + kb];
+        cs[(which * KB + kb) * BN + n] =
+            __ldg(a.act_scale + (size_t)(ti.row0 + n) * KB + kb) * __ldg(sw + (size_t)rb * KB + kb);
       }
       if (MODE == kDown) {
         for (int n = et; n < BN; n += EPT) {
@@ -254,6 +300,7 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
       for (int i = 0; i < HALF; ++i) accg[i] = 0.0f;
 #pragma unroll
       for (int i = 0; i < (MODE == kGateUp ? HALF : 1); ++i) accu[i] = 0.0f;
+      const bool live = c0 < width;  // warp-uniform: the MMA wrote this warp's columns
       for (int kb = 0; kb < KB; ++kb, ++kp) {
         const int pb = kp % NP;
         if (!aborted) {
@@ -267,40 +314,50 @@ __global__ void __launch_bounds__(32 * (Fp8Cfg<MODE, BN>::EW + 2), 1)
             }
           }
         }
-        if (!aborted) {
+        if (!aborted && live) {
           tc_fence_after();
-          const float swg = s_w[kb];
-          const float swu = MODE == kGateUp ? s_w[KB + kb] : 0.0f;
-          const uint32_t pbase = tl + static_cast<uint32_t>(pb * NA * BN);
+          const uint32_t pbase = tl + static_cast<uint32_t>(pb * NA * BN + c0);
+          // NC columns from c0: all HALF, or 16 when the MMA width leaves no more for this warp
+          auto promote = [&](auto nc) {
+            constexpr int NC = decltype(nc)::value;
+            uint32_t pg[NC];
+            [[maybe_unused]] uint32_t pu[MODE == kGateUp ? NC : 1];
+            tmem_ld_cols<NC>(pbase, pg);
+            if constexpr (MODE == kGateUp) tmem_ld_cols<NC>(pbase + BN, pu);
+            tmem_wait_ld();
+            const float4* cg = reinterpret_cast<const float4*>(cs + kb * BN + c0);
 #pragma unroll
-          for (int ch = 0; ch < NCH; ++ch) {
-            const int cstart = CW == 16 ? c0 + ch * 16 : 0;  // first TMEM column of this load
-            if (cstart < width) {                             // warp-uniform
-              uint32_t pg[16], pu[16];
-              tmem_ld16(pbase + cstart, pg);
-              if (MODE == kGateUp) tmem_ld16(pbase + BN + cstart, pu);
-              tmem_wait_ld();
+            for (int q = 0; q < NC / 4; ++q) {
+              const float4 g4 = cg[q];
+              accg[4 * q + 0] = fmaf(__uint_as_float(pg[4 * q + 0]), g4.x, accg[4 * q + 0]);
+              accg[4 * q + 1] = fmaf(__uint_as_float(pg[4 * q + 1]), g4.y, accg[4 * q + 1]);
+              accg[4 * q + 2] = fmaf(__uint_as_float(pg[4 * q + 2]), g4.z, accg[4 * q + 2]);
+              accg[4 * q + 3] = fmaf(__uint_as_float(pg[4 * q + 3]), g4.w, accg[4 * q + 3]);
+            }
+            if constexpr (MODE == kGateUp) {
+              const float4* cu = reinterpret_cast<const float4*>(cs + (KB + kb) * BN + c0);
 #pragma unroll
-              for (int q = 0; q < CW; ++q) {
-                const int col = ch * CW + q;  // index within this warp's half
-                const int n = c0 + col;       // tile column
-                // register holding column n (HALF < 16: the load holds both halves)
-                const uint32_t gb = CW == 16 ? pg[q] : (hf ? pg[(CW + q) & 15] : pg[q]);
-                const float sa = s_act[n * KB + kb];
-                accg[col] = fmaf(__uint_as_float(gb), sa * swg, accg[col]);
-                if (MODE == kGateUp) {
-                  const uint32_t ub = CW == 16 ? pu[q] : (hf ? pu[(CW + q) & 15] : pu[q]);
-                  accu[col] = fmaf(__uint_as_float(ub), sa * swu, accu[col]);
-                }
+              for (int q = 0; q < NC / 4; ++q) {
+                const float4 u4 = cu[q];
+                accu[4 * q + 0] = fmaf(__uint_as_float(pu[4 * q + 0]), u4.x, accu[4 * q + 0]);
+                accu[4 * q + 1] = fmaf(__uint_as_float(pu[4 * q + 1]), u4.y, accu[4 * q + 1]);
+                accu[4 * q + 2] = fmaf(__uint_as_float(pu[4 * q + 2]), u4.z, accu[4 * q + 2]);
+                accu[4 * q + 3] = fmaf(__uint_as_float(pu[4 * q + 3]), u4.w, accu[4 * q + 3]);
               }
             }
+          };
+          if constexpr (HALF == 32) {
+            if (width - c0 <= 16) promote(std::integral_constant<int, 16>{});
+            else promote(std::integral_constant<int, 32>{});
+          } else {
+            promote(std::integral_constant<int, HALF>{});
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pempty(pb));
       }
-      if (!aborted) {
+      if (!aborted && live) {
         if (MODE == kGateUp) {
           const int j = ti.mt * 128 + r;
           __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(a.h_out);
@@ -837,14 +894,18 @@ cudaError_t launch_ffn_fp8_fused(int bn, const ActMaps& xmaps, const ActMaps& hm
 // ==================================================================== launch
 
 template <int MODE, int BN>
-static cudaError_t launch_fp8(const ActMaps& maps, const GemmArgs& a, int grid, cudaStream_t s, bool pdl) {
+static cudaError_t launch_fp8(const ActMaps& maps, GemmArgs a, int grid, cudaStream_t s, bool pdl) {
   using C = Fp8Cfg<MODE, BN>;
+  const int KB = (MODE == kGateUp ? a.H : a.I) / 128;
+  if (KB > C::kMaxKB || C::stages(KB) < 2) return cudaErrorInvalidValue;
+  a.stages = C::stages(KB);
+  const size_t smem = C::smem(KB);
   auto kern = ffn_fp8_kernel<MODE, BN>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
   if (persistent <= 0) return cudaSuccess;
-  return launch_ex(kern, dim3(persistent), dim3(32 * (C::EW + 2)), C::kSmem, s, pdl, maps, a);
+  return launch_ex(kern, dim3(persistent), dim3(C::kThreads), smem, s, pdl, maps, a);
 }
 
 cudaError_t launch_ffn_fp8(int mode, int bn, const ActMaps& maps, const GemmArgs& a, int max_tiles, cudaStream_t s,

@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
   constexpr uint32_t A_OP = kKC * C::kChunkA;  // bytes of one A operand per stage
   constexpr uint32_t B_OFF = NA * A_OP;        // stage: [A gate][A up][B], kKC chunks each
   constexpr uint32_t ACC = NA * BN;            // TMEM columns of one accumulator buffer
-  const int S = a.stages;
+  constexpr int S = C::kStagesMax;  // compile-time depth: no division by a launch value in the K loops
   const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
   const int KB = (MODE == kGateUp ? a.H : a.I) / (64 * kKC);  // K steps per tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

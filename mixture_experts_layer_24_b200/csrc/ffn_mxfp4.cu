@@ -24,13 +24,26 @@
 // fetched by five copies (four for down): one 3-D TMA copy per operand brings
 // all KC blocks, and the weight scales of gate and up for KC blocks sit
 // together in global memory (mx.cu), as do the activation scales, so one bulk
-// copy each brings them. The TMA unit's per-copy cost, not the bytes, bounds
-// one SM's streaming rate for small copies: with one K block and six copies
-// per stage the GEMMs streamed 2.5-3.1 TB/s. A (E2M1) arrives in the tensor
+// copy each brings them (one K block and six copies per stage measured
+// 2.5-3.1 TB/s; the copies alone, without the MMAs, stream these stages at
+// 6.9-7.0 TB/s, so they are not the bound). A (E2M1) arrives in the tensor
 // cores' unpacked layout (16 codes per 16 bytes, the 128-byte swizzle); HBM
 // moves 4 bits per weight. Before the four 32-deep MMAs of each K block its
 // scale blocks go to TMEM with tcgen05.cp (32x128b, copied to all four lane
 // quarters); the MMAs read scale byte j = 0..3 of each row's word.
+//
+// What bounds it: a 32-deep MMA of this kind covers 16 bytes of E2M1 per
+// weight row, half of what a bf16 or e4m3 MMA covers, so a stage of 32 KB of
+// weights takes 16 MMAs and 6 scale copies, and each tcgen05 instruction
+// held its issuing thread about 60 SM cycles whatever the MMA width (clock64
+// stamps around the issue loop: 8 MMAs 470 cycles, 3 copies 160-200). Gate
+// and up are therefore issued by two threads (warps 5 and 6), each with its
+// own scale columns and its own commits (the stage and accumulator barriers
+// count both); that measured 7-11% faster than one issuer.
+//
+// Warp roles: warps 0..3 epilogue (TMEM lane quarters), warp 4 TMA producer,
+// warp 5 MMA issuer (gate, or down), warp 6 MMA issuer (up), warp 5 also
+// allocates TMEM.
 #include "common.cuh"
 #include "internal.h"
 #include "tile.cuh"
@@ -97,15 +110,15 @@ struct MxCfg {
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int NBUF = 2;
   static constexpr uint32_t kAcc = NA * BN;                 // TMEM columns of one accumulator buffer
-  static constexpr uint32_t kSfCol = NBUF * kAcc;           // scale columns after the accumulators
-  static constexpr uint32_t kTmemCols = tmem_cols_for(kSfCol + 4 * (NA + 1));
+  static constexpr uint32_t kSfCol = NBUF * kAcc;           // scale columns after the accumulators:
+  static constexpr uint32_t kTmemCols = tmem_cols_for(kSfCol + 8 * NA);  // per issuer 4 weight + 4 activation
   static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 256 + 4 * BN;
   static_assert(kStages >= 2, "a pipeline needs two stages");
   static_assert(BN <= 64, "two accumulators plus scale columns in 512 TMEM columns");
 };
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
+__global__ void __launch_bounds__(224, 1) ffn_mxfp4_kernel(const __grid_constant__ ActMaps act, const GemmArgs a) {
   using C = MxCfg<MODE, BN>;
   constexpr int NA = C::NA, NBUF = C::NBUF, S = C::kStages;
   constexpr uint32_t STAGE = C::kStageBytes, ACC = C::kAcc;
@@ -144,10 +157,10 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(empty(s), NA);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull(b), 1);
+      mbar_init(tfull(b), NA);
       mbar_init(tempty(b), 4);
     }
     *abort_flag = 0;
@@ -230,14 +243,15 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
       pdl_wait();
       pdl_trigger();
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 5 || warp == 6) {
+    // ------------------------------------------------------------ MMA issuers: warp 5 gate (or down), warp 6 up
     if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
-    if (lane == 0) {
-      const uint32_t sf_a0 = tmem + C::kSfCol, sf_a1 = sf_a0 + 4, sf_b = sf_a0 + 4 * NA;
+    const int who = warp - 5;
+    if (lane == 0 && who < NA) {
+      const uint32_t sf_a = tmem + C::kSfCol + 8 * who, sf_b = sf_a + 4;
       int consumed = 0, j = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
         const int buf = j % NBUF;
@@ -247,12 +261,12 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + buf * ACC;
+        const uint32_t d = tmem + buf * ACC + who * BN;
         TileInfo ti;
         decode_tile_at(a, m_tiles, BN, tile, ti);
         const int width = 16 << tile_width_index(ti.nvalid, BN);
         bool ok = true;
-        const uint32_t chunk_b = (uint32_t)width * 128u;  // a 3-D box lands its K blocks densely
+        const uint32_t chunk_b = (uint32_t)width * 128u;
         for (int ks = 0; ks < KS; ++ks, ++consumed) {
           const int s = consumed % S;
           if (!mbar_wait(full(s), (consumed / S) & 1)) {
@@ -263,21 +277,15 @@ __global__ void __launch_bounds__(192, 1) ffn_mxfp4_kernel(const __grid_constant
           const uint32_t st = base + s * STAGE;
 #pragma unroll
           for (int c = 0; c < KC; ++c) {
-            // this block's scales to TMEM; tcgen05 operations of one thread run in issue order, so the copies
-            // land after the previous block's MMAs have read the same columns
-            tc_cp_sf(sf_a0, sf_block_desc(st + C::kSfOff + c * NA * 512));
-            if (MODE == kGateUp) tc_cp_sf(sf_a1, sf_block_desc(st + C::kSfOff + c * NA * 512 + 512));
+            tc_cp_sf(sf_a, sf_block_desc(st + C::kSfOff + c * NA * 512 + who * 512));
             tc_cp_sf(sf_b, sf_block_desc(st + C::kSfBOff + c * 512));
 #pragma unroll
             for (uint32_t k = 0; k < 4; ++k) {
               const uint32_t idesc = mx_instr_desc(width, k);
               const uint64_t bdesc = sw128_kmajor_desc(st + C::kBOff + c * chunk_b + k * 32);
               const uint32_t acc = (ks | c | (int)k) != 0 ? 1u : 0u;
-              tc_mma_mx(d, sw128_kmajor_desc(st + c * kABytes + k * 32), bdesc, idesc, sf_a0 | (k << 30),
-                        sf_b | (k << 30), acc);
-              if (MODE == kGateUp)
-                tc_mma_mx(d + BN, sw128_kmajor_desc(st + C::kAOp + c * kABytes + k * 32), bdesc, idesc,
-                          sf_a1 | (k << 30), sf_b | (k << 30), acc);
+              tc_mma_mx(d, sw128_kmajor_desc(st + who * C::kAOp + c * kABytes + k * 32), bdesc, idesc,
+                        sf_a | (k << 30), sf_b | (k << 30), acc);
             }
           }
           tc_commit(empty(s));
@@ -394,7 +402,7 @@ static cudaError_t launch_mx(const ActMaps& maps, const GemmArgs& a, int grid, c
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
   const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
-  return launch_ex(kern, dim3(persistent), dim3(192), C::kSmem, s, pdl, maps, a);
+  return launch_ex(kern, dim3(persistent), dim3(224), C::kSmem, s, pdl, maps, a);
 }
 
 cudaError_t launch_ffn_mxfp4(int mode, int bn, const ActMaps& act_maps, const GemmArgs& a, int max_tiles,
