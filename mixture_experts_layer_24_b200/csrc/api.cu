@@ -473,9 +473,9 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     hmap = hmaps.m[0];
   } else {
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
-      st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, kBf16KChunks);
+      st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, kBf16GateUpChunks);
       if (st != MOE_OK) return st;
-      st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, kBf16KChunks);
+      st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, kBf16DownChunks);
       if (st != MOE_OK) return st;
     }
     xmap = xmaps.m[0];

@@ -31,17 +31,16 @@
 namespace moe {
 
 // bf16: one pipeline stage holds kKC consecutive 64-wide K chunks, fetched by
-// one 3-D TMA copy per operand (the per-copy cost of the TMA unit, not the
-// bytes, bounds a single SM's streaming rate for small boxes).
+// one 3-D TMA copy per operand (one chunk for gate/up, two for down: the
+// depths measured fastest).
 template <int MODE, int BN>
 struct Bf16Cfg {
   static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr int KC = kBf16KChunks;
+  static constexpr int KC = MODE == kGateUp ? kBf16GateUpChunks : kBf16DownChunks;
   static constexpr uint32_t kChunkA = kABytes;     // 128 rows x 128 B
   static constexpr uint32_t kChunkB = BN * 128;    // BN rows x 128 B
   static constexpr uint32_t kStageBytes = KC * (NA * kChunkA + kChunkB);
-  // up to 220 KB of stages (227 KB per CTA at most; one CTA per SM): three
-  // two-chunk stages at BN <= 32
+  // up to 220 KB of stages (227 KB per CTA at most; one CTA per SM)
   static constexpr int kStagesFit = (220 * 1024) / kStageBytes;
   static constexpr int kStagesMax = kStagesFit > 8 ? 8 : kStagesFit;
   // two accumulator buffers whenever both fit in TMEM's 512 columns
@@ -58,7 +57,7 @@ struct Bf16Cfg {
 // TMEM buffers so that the epilogue of tile j overlaps the MMAs of tile j+1.
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant__ ActMaps act,
+__global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant__ ActMaps act,
                                                           const GemmArgs a) {
   using C = Bf16Cfg<MODE, BN>;
   constexpr int NA = C::NA, kKC = C::KC, NBUF = C::NBUF;
@@ -99,10 +98,10 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
+      mbar_init(empty(s), NA);  // one commit per MMA issuer
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull(b), 1);
+      mbar_init(tfull(b), NA);
       mbar_init(tempty(b), 4);
     }
     *abort_flag = 0;
@@ -179,13 +178,16 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
       pdl_wait();
       pdl_trigger();
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 5 || warp == 6) {
+    // ------------------------------------------------------------ MMA issuers: warp 5 gate (or down), warp 6 up
+    // (each tcgen05 instruction holds its issuing thread for tens of cycles, about as long as a 128 x 128 x 16
+    // MMA computes, so two threads issue the two accumulators' MMAs)
     if (a.plan_ready) {
       pdl_wait();
       pdl_trigger();
     }
-    if (lane == 0) {
+    const int who = warp - 5;
+    if (lane == 0 && who < NA) {
       int consumed = 0, j = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++j) {
         const int buf = j % NBUF;
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + buf * ACC;
+        const uint32_t d = tmem + buf * ACC + who * BN;
         TileInfo ti;
         decode_tile_at(a, m_tiles, BN, tile, ti);
         const int width = 16 << tile_width_index(ti.nvalid, BN);
@@ -209,16 +211,15 @@ __global__ void __launch_bounds__(192, 1) ffn_bf16_kernel(const __grid_constant_
             break;
           }
           tc_fence_after();
-          const uint32_t st = base + s * STAGE;
+          const uint32_t st = base + s * STAGE + who * A_OP;
+          const uint32_t sb = base + s * STAGE + B_OFF;
 #pragma unroll
           for (int c = 0; c < kKC; ++c) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const uint64_t bdesc = sw128_kmajor_desc(st + B_OFF + c * chunk_b + k * 32);
+              const uint64_t bdesc = sw128_kmajor_desc(sb + c * chunk_b + k * 32);
               const uint32_t acc = (kb | c | k) != 0 ? 1u : 0u;
               tc_mma_bf16(d, sw128_kmajor_desc(st + c * C::kChunkA + k * 32), bdesc, idesc, acc);
-              if (MODE == kGateUp)
-                tc_mma_bf16(d + BN, sw128_kmajor_desc(st + A_OP + c * C::kChunkA + k * 32), bdesc, idesc, acc);
             }
           }
           tc_commit(empty(s));
@@ -722,7 +723,7 @@ static cudaError_t launch_bf16(const ActMaps& maps, GemmArgs a, int grid, cudaSt
   using C = Bf16Cfg<MODE, BN>;
   a.stages = C::kStagesMax;
   const int persistent = grid < a.num_sms ? grid : a.num_sms;  // one CTA per SM walks the tiles
-  return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 192, persistent, maps, a, s, pdl);
+  return launch_kernel(ffn_bf16_kernel<MODE, BN>, C::smem(a.stages), 224, persistent, maps, a, s, pdl);
 }
 
 template <int MODE>

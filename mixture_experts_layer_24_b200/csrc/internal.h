@@ -34,10 +34,12 @@ struct alignas(64) MapEntry {
 enum FfnMode { kGateUp = 0, kDown = 1 };
 
 // 64-wide K chunks per pipeline stage (one 3-D TMA copy per operand) of the
-// bf16 GEMM. Fewer, larger copies stream faster than more, smaller stages:
-// the TMA unit's per-copy cost bounds one SM's rate (measured at BN = 128:
-// one chunk per stage is 5-25% slower than two).
-constexpr int kBf16KChunks = 2;
+// bf16 GEMMs, measured at BN = 128 (4096 and 16384 tokens): gate/up streams
+// two weight operands per chunk, and one-chunk stages (4 of 48 KB in flight
+// instead of 2 of 96 KB) ran 4-10% faster; down stages are half that size,
+// and two-chunk stages (3 of 64 KB) ran 7-24% faster than one-chunk ones.
+constexpr int kBf16GateUpChunks = 1;
+constexpr int kBf16DownChunks = 2;
 
 // Launches `kern` on `s`, with programmatic stream serialisation when pdl is
 // true (the kernel must then follow the pdl_wait / pdl_trigger rule).
