@@ -14,10 +14,11 @@
 // behind any output element is the same whatever BN, the batch or the set of
 // resident experts; only the columns a CTA owns differ.
 //
-// Warp roles (one CTA per tile):
+// Warp roles of the GEMM (one CTA per SM, persistent over tiles):
 //   warps 0..3: epilogue (TMEM -> registers -> global)
-//   next warp: TMA producer (one elected lane)
-//   last warp: TMEM allocator + MMA issuer (one elected lane)
+//   warp 4: TMA producer (one elected lane)
+//   warp 5: TMEM allocator + MMA issuer of gate (or down); warp 6: MMA issuer
+//   of up (one elected lane each; the fused kernels keep one issuer)
 // Gate/up CTAs hold two accumulators, gate rows [j, j+128) and up rows
 // [I+j, I+j+128), so one thread owns g and u of the same (j, pair) and SwiGLU
 // happens in the epilogue without any exchange.

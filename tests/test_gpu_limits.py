@@ -77,3 +77,24 @@ def test_widest_hidden_and_intermediate_past_2_pow_31_elements():
     torch.cuda.synchronize()
     assert np.array_equal(oracle.as_u16(alone)[0], oracle.as_u16(out)[T - 1])
     layer.close()
+
+
+@pytest.mark.parametrize("T", [8, 256])
+def test_fp8_widest_hidden_and_intermediate(T):
+    """FP8 at H = I = 8192: 64 scale blocks along each reduction, the most the
+    FP8 kernels hold. At 256 tokens that is the separate GEMMs with the largest
+    per-tile scale table (four stages); at 8 tokens the fused decode launch.
+    Sampled tokens against the oracle (its own quantisation of the same bf16
+    draws), first and last included."""
+    _need_cuda()
+    import mixture_experts_layer_24_b200 as M
+    from helpers import LayerCase
+    H, E, K, I, seed = 8192, 8, 2, 8192, 73
+    case = LayerCase(T, H, E, K, I, seed=seed, wdtype=M.MOE_FP8_E4M3_B128)
+    out = case.forward()
+    torch.cuda.synchronize()
+    assert case.layer.status() == 0
+    tok = np.array(sorted({0, T // 2, T - 1}))
+    ref = case.oracle_forward(tokens=tok)["out"]
+    assert_close_out(oracle.as_u16(out)[tok], ref, 4e-2)
+    case.close()
