@@ -507,6 +507,7 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     a.status = ctx->d_status;
     a.sched = sched;
     a.num_sms = ctx->num_sms;
+    a.plan_ready = (pdl && plan_ready_gu) ? 1 : 0;  // plan -> quantiser -> this launch
     Prof p(ctx, MOE_PROF_FFN_FUSED, s);
     MOE_CUDA(launch_ffn_fp8_fused(bn, xmaps, hmaps, a, (c.intermediate / 128 + c.hidden / 128) * max_ntiles, s, pdl));
     return MOE_OK;

@@ -431,12 +431,19 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
   const int KBg = a.H / 128, KBd = a.I / 128;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  pdl_wait();  // the plan, the quantised x and the counters come from earlier kernels of the forward
-  pdl_trigger();
+  // The plan and the counters come from a kernel two or more launches back when a.plan_ready is set (the
+  // quantised x from the one just before): then the first weight stages go out before the programmatic wait.
+  if (!a.plan_ready) {
+    pdl_wait();
+    pdl_trigger();
+  }
   const int NT = a.nt_prefix[a.L];
   const int Gt = NT * mg, total = Gt + NT * md;
   const bool stand_down = a.status && (*reinterpret_cast<volatile int*>(a.status) & MOE_DEV_TIMEOUT);
-  if ((int)blockIdx.x >= total || stand_down) return;
+  if ((int)blockIdx.x >= total || stand_down) {
+    if (a.plan_ready) pdl_wait();
+    return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -491,6 +498,7 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
       const uint64_t pol_once = l2_policy_evict_first(), pol_shared = l2_policy_evict_normal();
       int issued = 0;
       int tile = blockIdx.x;
+      bool waited = !a.plan_ready;  // programmatic wait done
       auto fail = [&]() {
         *abort_flag = 1;
         flag_status(a.status, MOE_DEV_TIMEOUT);
@@ -517,7 +525,23 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
           const void* amap = &xact.m[wi];
           const uint32_t tx = 2 * kABytes + (16u << wi) * 128u;
           tensormap_acquire(wmap);
-          for (int kb = 0; kb < KBg; ++kb, ++issued) {
+          int kb = 0;
+          if (!waited) {
+            // first tile: its weight stages before the wait, x (from the previous kernel) after it
+            const int npre = KBg < S ? KBg : S;
+            for (; kb < npre; ++kb) {
+              const uint32_t st = base + kb * STAGE;
+              mbar_arrive_expect_tx(full(kb), tx);
+              tma_load_2d_hint(st, wmap, full(kb), kb * 128, ti.mt * 128, pol_w);
+              tma_load_2d_hint(st + kABytes, wmap, full(kb), kb * 128, a.I + ti.mt * 128, pol_w);
+            }
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
+            for (int q = 0; q < npre; ++q) tma_load_2d(base + q * STAGE + 2 * kABytes, amap, full(q), q * 128, ti.row0);
+            issued = npre;
+          }
+          for (; kb < KBg; ++kb, ++issued) {
             const int s = issued % S;
             if (issued >= S && !mbar_wait(empty(s), ((issued / S) - 1) & 1)) {
               ok = false;
@@ -544,6 +568,11 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
             }
             mbar_arrive_expect_tx(full(s), tx);
             tma_load_2d_hint(base + s * STAGE, wmap, full(s), kb * 128, ti.mt * 128, pol_w);
+          }
+          if (!waited) {
+            pdl_wait();
+            pdl_trigger();
+            waited = true;
           }
           if (ok) {
             const int* dep = a.sched + 1 + ti.ng;
@@ -585,10 +614,21 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
         }
         tile = (int)gridDim.x + atomicAdd(a.sched, 1);
       }
+      if (!waited) {
+        pdl_wait();
+        pdl_trigger();
+      }
       for (int g = issued - S < 0 ? 0 : issued - S; g < issued; ++g) mbar_wait(full(g % S), (g / S) & 1);
+    } else if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     if (lane == 0) {
       int consumed = 0, kp = 0;
       bool ok = true;
@@ -635,6 +675,10 @@ __global__ void __launch_bounds__(320, 1) ffn_fp8_fused_kernel(const __grid_cons
   } else {
     // ------------------------------------------------------------ epilogue (warps 0..7)
     // warp w owns TMEM lanes [32(w%4), +32) and columns [HALF*(w/4), +HALF)
+    if (a.plan_ready) {
+      pdl_wait();
+      pdl_trigger();
+    }
     const int q4 = warp & 3, hf = warp >> 2;
     const int r = q4 * 32 + lane;
     const int et = threadIdx.x;  // 0..255
