@@ -512,10 +512,13 @@ static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, 
                    sched, sched ? sched_n : 0);
 }
 
-// T <= 8: logits + fused top-k in one launch; up to 64 tokens: logits in
-// 8-token groups, then the warp top-k kernel (programmatic launch). Rows that
-// a bulk copy cannot take (not 16-byte aligned, or too large for shared
-// memory) go through the direct kernel.
+// T <= 4: logits + fused top-k in one launch; up to 64 tokens: logits, then
+// the warp top-k kernel (programmatic launch), which measured faster from 8
+// tokens on (the fused top-k runs in the last CTA's four warps, two tokens
+// each at T = 8: 299.0 vs 293.5 us per layer) and slower below (by 0.7-1.9
+// us). The fused form was also slower for the register-tiled kernel at 16 and
+// 64 tokens. Rows that a bulk copy cannot take (not 16-byte aligned, or too
+// large for shared memory) go through the direct kernel.
 cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                                float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
                                cudaStream_t s, bool pdl, int* sched, int sched_n) {
@@ -531,7 +534,12 @@ cudaError_t launch_route_small(const void* x, const float* wr, const float* bias
   if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
   if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
   if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
-  if (T <= 8) return launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
+  if (T <= 8) {
+    const cudaError_t err = launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, status, s, sched,
+                                         sched_n);
+    if (err != cudaSuccess) return err;
+    return launch_topk_warp(logits, T, E, K, idx, w, s, pdl);
+  }
   // more tokens: W rows would be staged once per 8-token group; register
   // tiles reuse each loaded element across 4 tokens and 4 or 8 experts
   cudaError_t err;
