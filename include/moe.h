@@ -325,6 +325,17 @@ moe_status_t moe_plan_hot_set(const int64_t* hist, int E, int n_hot, int32_t* ho
  * non-positive limits return MOE_ERR_INVALID_ARG without launching. */
 moe_status_t moe_debug_wait_flag(moe_ctx_t* ctx, const int32_t* flag, int64_t limit_ns, moe_stream_t stream);
 
+/* Test hook for failure detection on the host: the library's own allocations
+ * of the given kind -- MOE_ALLOC_DEVICE (cudaMalloc: context words, slot
+ * tables, spare slots, residency state, MXFP4 scale blocks), MOE_ALLOC_PINNED
+ * (cudaHostAlloc: the slot tables' pinned staging words) or MOE_ALLOC_ANY --
+ * let `skip` succeed and then fail the next n as if the memory were exhausted.
+ * The calls that make them return MOE_ERR_OOM and release what they had
+ * allocated. Process-wide; n = 0 disarms it. Negative counts or an unknown
+ * kind return MOE_ERR_INVALID_ARG. The hook itself touches no device. */
+enum { MOE_ALLOC_ANY = 0, MOE_ALLOC_DEVICE = 1, MOE_ALLOC_PINNED = 2 };
+moe_status_t moe_debug_fail_allocs(int kind, int skip, int n);
+
 /* Copies the device status word to *status (synchronises the context's
  * device); reset != 0 clears it afterwards. */
 moe_status_t moe_get_device_status(moe_ctx_t* ctx, int32_t* status, int reset);

@@ -28,6 +28,10 @@ from .binding import (  # noqa: F401
     moe_combine,
     moe_ctx_create,
     moe_ctx_destroy,
+    MOE_ALLOC_ANY,
+    MOE_ALLOC_DEVICE,
+    MOE_ALLOC_PINNED,
+    moe_debug_fail_allocs,
     moe_debug_wait_flag,
     moe_ep_gather_rows,
     moe_ep_pack,

@@ -35,7 +35,8 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_workspace_size", "moe_route
            "moe_slots_destroy", "moe_slots_register", "moe_slots_query", "moe_slots_stats",
            "moe_plan_hot_set", "moe_get_device_status", "moe_last_error", "moe_launch_count",
            "moe_profile_enable", "moe_profile_read", "moe_route_noalloc", "moe_slots_set_policy",
-           "moe_debug_wait_flag", "moe_ep_pack", "moe_ep_recv_plan", "moe_ep_gather_rows", "moe_quantize_mx"]
+           "moe_debug_wait_flag", "moe_ep_pack", "moe_ep_recv_plan", "moe_ep_gather_rows", "moe_quantize_mx",
+           "moe_debug_fail_allocs"]
 
 PROF_KINDS = ["router", "topk", "permute", "gather", "gate_up", "down", "quant", "combine", "ffn_fused"]
 
@@ -97,6 +98,7 @@ def lib():
         "moe_ep_recv_plan": ([P, P, I, P, P, P, P, P], S),
         "moe_ep_gather_rows": ([P, P, P, I, P, P], S),
         "moe_quantize_mx": ([P, I, I, I, P, P, P], S),
+        "moe_debug_fail_allocs": ([I, I, I], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -258,6 +260,16 @@ def moe_debug_wait_flag(ctx, flag, limit_ns: int, stream=None):
     _check(lib().moe_debug_wait_flag(ctx, _p(flag), int(limit_ns), _s(stream)), "moe_debug_wait_flag")
 
 
+MOE_ALLOC_ANY, MOE_ALLOC_DEVICE, MOE_ALLOC_PINNED = 0, 1, 2
+
+
+def moe_debug_fail_allocs(kind: int, skip: int, n: int):
+    """Test hook: of the library's own allocations of `kind` (MOE_ALLOC_DEVICE,
+    MOE_ALLOC_PINNED or MOE_ALLOC_ANY), let `skip` succeed and fail the next `n`
+    as an exhausted device or host would; n = 0 disarms it."""
+    _check(lib().moe_debug_fail_allocs(int(kind), int(skip), int(n)), "moe_debug_fail_allocs")
+
+
 def moe_launch_count(ctx) -> int:
     return int(lib().moe_launch_count(ctx))
 
@@ -320,7 +332,12 @@ class MoeLayer:
         self.device = d
         with torch.cuda.device(self.device):
             self.ctx = moe_ctx_create(hidden, n_experts, top_k, intermediate, wdtype, flags)
-            self.slots = moe_slots_create(self.ctx, n_spare_slots)
+            try:
+                self.slots = moe_slots_create(self.ctx, n_spare_slots)
+            except MoeError:
+                moe_ctx_destroy(self.ctx)  # nothing of a half-built layer stays allocated
+                self.ctx = None
+                raise
         self._keep = {}
         self._ws = None
 

@@ -586,11 +586,53 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
 
 }  // namespace
 
+// ---------------------------------------------------- allocation hook --
+// Every allocation the library makes goes through lib_malloc / lib_host_alloc,
+// so that moe_debug_fail_allocs can make chosen ones fail as an exhausted
+// device or host would.
+namespace {
+std::mutex g_fail_mu;
+int g_fail_kind = MOE_ALLOC_ANY, g_fail_skip = 0, g_fail_n = 0;
+
+bool injected_alloc_failure(int kind) {
+  std::lock_guard<std::mutex> lock(g_fail_mu);
+  if (g_fail_n <= 0 || (g_fail_kind != MOE_ALLOC_ANY && g_fail_kind != kind)) return false;
+  if (g_fail_skip > 0) {
+    --g_fail_skip;
+    return false;
+  }
+  --g_fail_n;
+  return true;
+}
+
+template <typename P>
+cudaError_t lib_malloc(P** p, size_t bytes) {
+  if (injected_alloc_failure(MOE_ALLOC_DEVICE)) return cudaErrorMemoryAllocation;
+  return cudaMalloc(reinterpret_cast<void**>(p), bytes);
+}
+
+template <typename P>
+cudaError_t lib_host_alloc(P** p, size_t bytes) {
+  if (injected_alloc_failure(MOE_ALLOC_PINNED)) return cudaErrorMemoryAllocation;
+  return cudaHostAlloc(reinterpret_cast<void**>(p), bytes, cudaHostAllocDefault);
+}
+}  // namespace
+
 // =================================================================== ABI ==
 
 extern "C" {
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+moe_status_t moe_debug_fail_allocs(int kind, int skip, int n) {
+  if (kind < MOE_ALLOC_ANY || kind > MOE_ALLOC_PINNED || skip < 0 || n < 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_debug_fail_allocs: unknown kind or negative count");
+  std::lock_guard<std::mutex> lock(g_fail_mu);
+  g_fail_kind = kind;
+  g_fail_skip = skip;
+  g_fail_n = n;
+  return MOE_OK;
+}
 
 moe_status_t moe_ctx_create(moe_ctx_t** out, const moe_config_t* cfg) {
   if (!out || !cfg) return fail(MOE_ERR_INVALID_ARG, "NULL argument");
@@ -612,8 +654,8 @@ moe_status_t moe_ctx_create(moe_ctx_t** out, const moe_config_t* cfg) {
   ctx->num_sms = prop.multiProcessorCount;
   ctx->chain = !(cfg->flags & MOE_FLAG_NO_PDL);
   ctx->encode = reinterpret_cast<EncodeTiledFn>(fn);
-  if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess ||
-      cudaMalloc(&ctx->d_counters, sizeof(unsigned int) * kRouteSmallMaxT) != cudaSuccess) {
+  if (lib_malloc(&ctx->d_status, sizeof(int)) != cudaSuccess ||
+      lib_malloc(&ctx->d_counters, sizeof(unsigned int) * kRouteSmallMaxT) != cudaSuccess) {
     cudaFree(ctx->d_status);
     delete ctx;
     return fail(MOE_ERR_OOM, "cudaMalloc of the context's device words failed");
@@ -1330,14 +1372,14 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
     moe_slots_destroy(sl);
     return fail(st, msg);
   };
-  if (cudaMalloc(&sl->d_maps, sizeof(MapEntry) * (sl->E + n_spare)) != cudaSuccess)
+  if (lib_malloc(&sl->d_maps, sizeof(MapEntry) * (sl->E + n_spare)) != cudaSuccess)
     return cleanup(MOE_ERR_OOM, "cudaMalloc of the map table failed");
-  if (cudaMalloc(&sl->d_map_of, sizeof(int32_t) * sl->E) != cudaSuccess)
+  if (lib_malloc(&sl->d_map_of, sizeof(int32_t) * sl->E) != cudaSuccess)
     return cleanup(MOE_ERR_OOM, "cudaMalloc of the slot index failed");
-  if (n_spare > 0 && cudaMalloc(&sl->spare, sl->slot_bytes * n_spare) != cudaSuccess)
+  if (n_spare > 0 && lib_malloc(&sl->spare, sl->slot_bytes * n_spare) != cudaSuccess)
     return cleanup(MOE_ERR_OOM, "cudaMalloc of the spare slots failed");
   sl->h_pinned_ints = (size_t)(sl->E + 1) + 4 * (size_t)sl->E + 256;
-  if (cudaHostAlloc(&sl->h_pinned, sizeof(int32_t) * sl->h_pinned_ints, cudaHostAllocDefault) != cudaSuccess)
+  if (lib_host_alloc(&sl->h_pinned, sizeof(int32_t) * sl->h_pinned_ints) != cudaSuccess)
     return cleanup(MOE_ERR_OOM, "cudaHostAlloc failed");
   if (cudaStreamCreateWithFlags(&sl->copy_stream, cudaStreamNonBlocking) != cudaSuccess)
     return cleanup(MOE_ERR_CUDA, "cudaStreamCreate failed");
@@ -1366,7 +1408,7 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
                  o_st = take(n_spare * 8), o_es = take(E_ * 4), o_tick = take(8), o_cn = take(4),
                  o_ce = take(n_spare * 4), o_cs = take(n_spare * 4), o_stats = take(8 * 8);
     uint8_t* d = nullptr;
-    if (cudaMalloc(&d, o) != cudaSuccess) return cleanup(MOE_ERR_OOM, "cudaMalloc of the residency state failed");
+    if (lib_malloc(&d, o) != cudaSuccess) return cleanup(MOE_ERR_OOM, "cudaMalloc of the residency state failed");
     sl->d_res = d;
     ResidencyDev& r = sl->rdev;
     r.loc = reinterpret_cast<const int32_t*>(d + o_loc);
@@ -1396,7 +1438,7 @@ moe_status_t moe_slots_create(moe_slots_t** out, moe_ctx_t* ctx, int n_spare) {
         cudaMemset(d + o_stats, 0, 64) != cudaSuccess)  // ... except the records, tick, copy count, stats
       return cleanup(MOE_ERR_CUDA, "cudaMemset of the residency state failed");
     sl->h_lru_words = 9 + (size_t)n_spare + (2 * (size_t)n_spare + 2 * E_ + 1) / 2 + 1;
-    if (cudaHostAlloc(&sl->h_lru, 2 * sl->h_lru_words * sizeof(int64_t), cudaHostAllocDefault) != cudaSuccess)
+    if (lib_host_alloc(&sl->h_lru, 2 * sl->h_lru_words * sizeof(int64_t)) != cudaSuccess)
       return cleanup(MOE_ERR_OOM, "cudaHostAlloc of the residency staging failed");
   }
   for (int i = 0; i < n_spare; ++i) {
@@ -1470,7 +1512,7 @@ moe_status_t moe_slots_register(moe_slots_t* sl, int expert, const void* w_gu, c
       const int H = c.hidden, I = c.intermediate;
       const size_t gu_blk = (size_t)(2 * I / 128) * (H / 128) * 512, dn_blk = (size_t)(H / 128) * (I / 128) * 512;
       uint8_t* blk = nullptr;
-      if (cudaMalloc(&blk, gu_blk + dn_blk) != cudaSuccess) return fail(MOE_ERR_OOM, "cudaMalloc of MXFP4 scales failed");
+      if (lib_malloc(&blk, gu_blk + dn_blk) != cudaSuccess) return fail(MOE_ERR_OOM, "cudaMalloc of MXFP4 scales failed");
       cudaError_t err = launch_mx_block_scales(static_cast<const uint8_t*>(s_gu_), 2 * I, H, I, blk, nullptr);
       if (err == cudaSuccess)
         err = launch_mx_block_scales(static_cast<const uint8_t*>(s_dn_), H, I, 0, blk + gu_blk, nullptr);

@@ -203,3 +203,15 @@ def test_layer_methods_accept_valid_calls_and_reject_bad_ones(monkeypatch):
         F.register(0, qg, qd, sg.double(), sd)
     with pytest.raises(TypeError):
         F.register(0, qg, qd, None, sd)
+
+
+def test_allocation_failure_hook_argument_checks(lib):
+    """The host-side allocation hook (moe_debug_fail_allocs) refuses unknown
+    kinds and negative counts, and arming or disarming it needs no device."""
+    import mixture_experts_layer_24_b200 as M
+    for args in ((-1, 0, 1), (3, 0, 1), (0, -1, 1), (0, 0, -1)):
+        with pytest.raises(M.MoeError) as ei:
+            M.moe_debug_fail_allocs(*args)
+        assert ei.value.status == 1  # MOE_ERR_INVALID_ARG
+    M.moe_debug_fail_allocs(M.MOE_ALLOC_PINNED, 2, 1)
+    M.moe_debug_fail_allocs(M.MOE_ALLOC_ANY, 0, 0)  # disarmed

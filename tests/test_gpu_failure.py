@@ -135,3 +135,97 @@ def test_unregistered_expert_rows_are_zero_in_expert_ffn():
     ref = oracle.ffn_bf16(oracle.as_u16(case.x), ps_n[rows], pe, w_n[ps_n[rows], pk_n[rows]], gu, dn, E)
     assert np.max(np.abs(yn[rows] - ref)) <= 2e-2 * np.max(np.abs(ref))
     case.close()
+
+
+# ------------------------------------------------- failed allocations --
+
+MOE_ERR_OOM = 6
+
+
+def test_failed_allocations_return_oom_and_the_next_call_works():
+    """Host-side fault injection (no GPU fault): each of the library's own
+    allocations is made to fail in turn -- the context's device words, the slot
+    table's device arrays, its spare slots and device LRU state, and its two
+    pinned staging buffers. Each failing call returns MOE_ERR_OOM with what it
+    had allocated released (a half-built MoeLayer releases its context too);
+    with the hook disarmed the same calls succeed, and a layer with host-resident
+    experts behind those spare slots then matches the oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import mixture_experts_layer_24_b200 as M
+    H, E, K, I = 256, 8, 2, 512
+    try:
+        for skip in (0, 1):  # d_status, then d_counters
+            M.moe_debug_fail_allocs(M.MOE_ALLOC_DEVICE, skip, 1)
+            with pytest.raises(M.MoeError) as ei:
+                M.moe_ctx_create(H, E, K, I)
+            assert ei.value.status == MOE_ERR_OOM
+        M.moe_debug_fail_allocs(M.MOE_ALLOC_ANY, 0, 0)
+        ctx = M.moe_ctx_create(H, E, K, I)
+        # slot table with 4 spare slots: device maps, slot index, spare slots, LRU state; pinned staging words
+        # and LRU staging
+        for kind, skip in ((M.MOE_ALLOC_DEVICE, 0), (M.MOE_ALLOC_DEVICE, 1), (M.MOE_ALLOC_DEVICE, 2),
+                           (M.MOE_ALLOC_DEVICE, 3), (M.MOE_ALLOC_PINNED, 0), (M.MOE_ALLOC_PINNED, 1)):
+            M.moe_debug_fail_allocs(kind, skip, 1)
+            with pytest.raises(M.MoeError) as ei:
+                M.moe_slots_create(ctx, 4)
+            assert ei.value.status == MOE_ERR_OOM, (kind, skip)
+            M.moe_debug_fail_allocs(M.MOE_ALLOC_ANY, 0, 0)
+        slots = M.moe_slots_create(ctx, 4)
+        M.moe_slots_destroy(slots)
+        M.moe_ctx_destroy(ctx)
+        # a layer whose slot table cannot get its pinned words: the constructor raises and keeps nothing
+        M.moe_debug_fail_allocs(M.MOE_ALLOC_PINNED, 0, 1)
+        with pytest.raises(M.MoeError) as ei:
+            M.MoeLayer(H, E, K, I, n_spare_slots=4)
+        assert ei.value.status == MOE_ERR_OOM
+    finally:
+        M.moe_debug_fail_allocs(M.MOE_ALLOC_ANY, 0, 0)
+    case = LayerCase(16, H, E, K, I, seed=37, n_spare=4, hot={0, 1, 2, 3})
+    out = case.forward()
+    torch.cuda.synchronize()
+    assert case.layer.status() == 0
+    assert_close_out(oracle.as_u16(out), case.oracle_forward()["out"], 2e-2)
+    case.close()
+
+
+def test_failed_mxfp4_scale_allocation_then_registration_works():
+    """MXFP4 registration allocates the experts' blocked scales; when that
+    allocation fails the call returns MOE_ERR_OOM, and registering again
+    succeeds with results identical to a layer that never saw the failure."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import mixture_experts_layer_24_b200 as M
+    import synth
+    H, E, K, I, T = 256, 4, 2, 256, 8
+    dev = torch.device("cuda")
+    ws = []
+    for e in range(E):
+        g, d = synth.expert_weights(e, H, I, seed=41, device=dev)
+        qg = torch.empty((2 * I, H // 2), dtype=torch.uint8, device=dev)
+        sg = torch.empty((2 * I, H // 32), dtype=torch.uint8, device=dev)
+        qd = torch.empty((H, I // 2), dtype=torch.uint8, device=dev)
+        sd = torch.empty((H, I // 32), dtype=torch.uint8, device=dev)
+        M.moe_quantize_mx(g, 2 * I, H, 0, qg, sg)
+        M.moe_quantize_mx(d, H, I, 0, qd, sd)
+        ws.append((qg, qd, sg, sd))
+    x = synth.tokens(T, H, seed=41, device=dev)
+    wr = synth.router_weight(E, H, seed=41, device=dev)
+    outs = []
+    for inject in (False, True):
+        layer = M.MoeLayer(H, E, K, I, wdtype=M.MOE_MXFP4, device=dev)
+        for e in range(E):
+            if inject and e == 1:
+                M.moe_debug_fail_allocs(M.MOE_ALLOC_DEVICE, 0, 1)
+                try:
+                    with pytest.raises(M.MoeError) as ei:
+                        layer.register(e, *ws[e])
+                    assert ei.value.status == MOE_ERR_OOM
+                finally:
+                    M.moe_debug_fail_allocs(M.MOE_ALLOC_ANY, 0, 0)
+            layer.register(e, *ws[e])
+        outs.append(oracle.as_u16(layer.forward(x, wr)))
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        layer.close()
+    assert np.array_equal(outs[0], outs[1])
