@@ -50,8 +50,11 @@ def _run_ranks(world, make_steps, xs, wr, bias):
     return outs, status
 
 
-@pytest.mark.parametrize("world,wdtype", [(2, 0), (4, 0), (3, 0), (4, 1)])
+@pytest.mark.parametrize("world,wdtype", [(2, 0), (4, 0), (3, 0), (4, 1), (2, 2)])
 def test_ep_ranks_match_single_gpu_small(world, wdtype):
+    """bf16 (0), FP8 (1) and MXFP4 (2) experts split over `world` ranks. MXFP4
+    is checked bit for bit against the single-GPU MXFP4 forward, which
+    tests/test_gpu_mxfp4.py checks against the oracle."""
     _need_cuda()
     import mixture_experts_layer_24_b200 as M
     from mixture_experts_layer_24_b200 import ep
@@ -62,7 +65,15 @@ def test_ep_ranks_match_single_gpu_small(world, wdtype):
     ws = []
     for e in range(E):
         g, d = synth.expert_weights(e, H, I, seed=61, device=dev)
-        if wdtype == 1:
+        if wdtype == 2:
+            qg = torch.empty((2 * I, H // 2), dtype=torch.uint8, device=dev)
+            sg = torch.empty((2 * I, H // 32), dtype=torch.uint8, device=dev)
+            qd = torch.empty((H, I // 2), dtype=torch.uint8, device=dev)
+            sd = torch.empty((H, I // 32), dtype=torch.uint8, device=dev)
+            M.moe_quantize_mx(g, 2 * I, H, 0, qg, sg)
+            M.moe_quantize_mx(d, H, I, 0, qd, sd)
+            ws.append((qg, qd, sg, sd))
+        elif wdtype == 1:
             qg = torch.empty((2 * I, H), dtype=torch.uint8, device=dev)
             sg = torch.empty((2 * I // 128, H // 128), dtype=torch.float32, device=dev)
             qd = torch.empty((H, I), dtype=torch.uint8, device=dev)
@@ -92,6 +103,8 @@ def test_ep_ranks_match_single_gpu_small(world, wdtype):
         torch.cuda.synchronize()
         got = oracle.as_u16(outs[r])
         assert np.array_equal(got, oracle.as_u16(ref)), f"rank {r} of {world}"
+        if wdtype == 2:
+            continue
         tok = np.unique([0, T_of[r] // 2, T_of[r] - 1])
         ref_o = oracle_layer_out(oracle.as_u16(xs[r])[tok], wr.cpu().numpy(), bias.cpu().numpy(), K, E, H, I,
                                  seed=61, fp8=wdtype == 1)
