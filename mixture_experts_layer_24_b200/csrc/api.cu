@@ -858,11 +858,17 @@ moe_status_t ffn_decode_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, con
 
 // Decode batches with host-resident experts whose pairs cannot route to more host experts than there are
 // spare slots: the cache bookkeeping and the copies run on the device (residency.cu), no host round trip.
+// Decode batches with host-resident experts whose pairs fit the spare slots: the LRU plan and the copies run on
+// the device. bf16 then takes the one-launch decode FFN; FP8 the one-launch permutation and plan, the quantiser and
+// its GEMMs, which read the cached experts through the same slot table.
 bool residency_device_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, int T) {
   const moe_config_t& c = ctx->cfg;
-  return c.wdtype == MOE_BF16 && sl->n_host > 0 && sl->d_res && sl->policy == MOE_SLOTS_LRU &&
-         sl->n_unmapped == 0 && (long long)T * c.top_k <= sl->n_spare && T >= 1 && T <= kDecodeMaxT &&
-         (long long)T * c.top_k <= kDecodeMaxPairs && ((uintptr_t)x % 16) == 0 &&
+  const long long P = (long long)T * c.top_k;
+  if (sl->n_host <= 0 || !sl->d_res || sl->policy != MOE_SLOTS_LRU || sl->n_unmapped != 0 || T < 1 ||
+      P > sl->n_spare)
+    return false;
+  if (c.wdtype == MOE_FP8_E4M3_B128) return P <= kPermuteSmallMaxPairs;
+  return c.wdtype == MOE_BF16 && T <= kDecodeMaxT && P <= kDecodeMaxPairs && ((uintptr_t)x % 16) == 0 &&
          ffn_decode_smem_bytes(T, c.n_experts) <= 232448;
 }
 
@@ -877,7 +883,8 @@ bool decode_path_ok(const moe_ctx_t* ctx, const moe_slots_t* sl, const void* x, 
 // (bf16) the sorted rows; `pdl`: the previous launch is this forward's own.
 moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int32_t* perm_src,
                       const int32_t* perm_k, const int32_t* offsets, const float* topk_w, int T, float* y_pair,
-                      void* ws, cudaStream_t s, bool pdl, bool planned, const int32_t* inv = nullptr) {
+                      void* ws, cudaStream_t s, bool pdl, bool planned, const int32_t* inv = nullptr,
+                      bool cached_on_device = false) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const WsLayout W = ws_layout(c, T);
@@ -919,9 +926,13 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
                      s, ctx->chain, planned ? pdl : true);
   }
-  if (sl->n_host == 0) {
-    sl->stats.last_cold = 0;
-    sl->stats.last_touched = -1;
+  if (sl->n_host == 0 || cached_on_device) {
+    // every routed expert is in HBM: resident, or (cached_on_device) put in a spare slot by the device-side plan
+    // earlier in this forward, which also wrote the counts the stats report
+    if (!cached_on_device) {
+      sl->stats.last_cold = 0;
+      sl->stats.last_touched = -1;
+    }
     bool plan_ready_gu = false;
     if (!planned) {
       {
@@ -1237,7 +1248,17 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
       Prof p(ctx, MOE_PROF_GATHER, s);
       MOE_CUDA(launch_residency_copy(sl->rdev, sl->spare, ctx->num_sms, s, chain));
     }
-    if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched)) != MOE_OK) return st;
+    if (c.wdtype == MOE_BF16) {
+      if ((st = ffn_decode_impl(ctx, sl, x, idx, w, T, y, ws, s, sched)) != MOE_OK) return st;
+    } else {
+      // FP8: the permutation and tile plan read the expert -> map table the cache plan just updated
+      bool planned = false;
+      if ((st = permute_impl(ctx, idx, T, counts, offsets, ps, pk, inv, ws, s, chain, sl->d_map_of,
+                             ffn_block_n(T, c.wdtype), x, nullptr, &planned)) != MOE_OK)
+        return st;
+      if ((st = ffn_impl(ctx, sl, x, ps, pk, offsets, w, T, y, ws, s, chain, planned, inv, true)) != MOE_OK)
+        return st;
+    }
     sl->last_dev = true;
     Prof p(ctx, MOE_PROF_COMBINE, s);
     MOE_CUDA(launch_combine(y, inv, T, c.top_k, c.hidden, out, s, chain));

@@ -140,15 +140,17 @@ def test_reregistering_an_expert_drops_its_cached_copy():
     cache.close()
 
 
-def test_device_side_cache_in_a_cuda_graph():
+@pytest.mark.parametrize("wdtype", [0, 1])
+def test_device_side_cache_in_a_cuda_graph(wdtype):
     """Decode batches whose pairs fit in the spare slots keep the whole cache
     bookkeeping on the device (plan, copies of the missed experts, FFN), so the
     forward can be captured once and replayed: over replays with new tokens the
     cache fills, hits and evicts inside the graph, and every output equals the
-    all-resident layer's bits and the oracle within 2e-2."""
+    all-resident layer's bits and the oracle within 2e-2 (bf16) or 4e-2 (FP8:
+    the cached records include the weight block scales)."""
     _need_cuda()
     import mixture_experts_layer_24_b200 as M
-    ref, cache, wr, bias, keep = _layers(0, M.MOE_SLOTS_LRU)
+    ref, cache, wr, bias, keep = _layers(wdtype, M.MOE_SLOTS_LRU)
     dev = torch.device("cuda")
     T = 2  # 8 pairs <= 12 slots: the device-side path
     x = synth.tokens(T, H, seed=5, device=dev, first_token=9000)
@@ -162,7 +164,8 @@ def test_device_side_cache_in_a_cuda_graph():
         assert cache.status() == 0 and ref.status() == 0
         got = oracle.as_u16(out)
         assert np.array_equal(got, oracle.as_u16(a)), f"replay {i} differs"
-        assert_close_out(got, oracle_layer_out(oracle.as_u16(x), wr.cpu().numpy(), None, K, E, H, I, seed=5), TOL[0])
+        assert_close_out(got, oracle_layer_out(oracle.as_u16(x), wr.cpu().numpy(), None, K, E, H, I, seed=5,
+                                               fp8=wdtype == 1), TOL[wdtype])
         st = cache.stats()
         assert st["last_hits"] + st["last_cold"] == st["last_routed_cold"]
         seen_hits += st["last_hits"]
