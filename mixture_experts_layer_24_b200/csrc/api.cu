@@ -176,7 +176,12 @@ struct WsLayout {
   size_t logits, rank, chunk_counts, topk_idx, topk_w, counts, offsets, perm_src, perm_k, inv;
   size_t list_expert, list_map, nt_prefix, sched, x_perm, x_scale, h, hq, h_scale, y_pair, total;
   size_t x_sfb, h_sfb;  // MXFP4: activation scales in the tensor cores' block layout, per N tile
+  size_t nt_prefix2;    // MXFP4: N tiles of the (wider) down GEMM per listed expert
 };
+
+// MXFP4 down GEMM tile width for a gate/up width bn: 128 once gate/up is at its 64 (a 128-wide down tile keeps two
+// accumulators and ran 28% faster at 4096 tokens; a 128-wide gate/up tile has one and ran 42% slower).
+inline int mx_down_bn(int bn) { return bn >= 64 ? 128 : bn; }
 
 WsLayout ws_layout(const moe_config_t& c, int T) {
   WsLayout L{};
@@ -204,6 +209,7 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
   L.list_expert = take((2 * E + 64) * 4);
   L.list_map = take((2 * E + 64) * 4);
   L.nt_prefix = take((2 * E + 64) * 4);
+  L.nt_prefix2 = take(mx ? (E + 1) * 4 : 0);
   L.sched = take((size_t)fused_sched_entries((int)E) * 4);
   L.x_perm = take(P * H * ((fp8 || mx) ? 1 : 2));
   L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
@@ -416,13 +422,20 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   const int P = T * c.top_k;
   if (c.wdtype == MOE_MXFP4) {
     // both GEMMs on the block-scaled tensor cores; gate/up writes h as MX e4m3 codes and blocked scales
+    // the down GEMM runs on wider N tiles (bn_dn; its prefix from the plan), and gate/up writes h's scale blocks
+    // in that tiling
+    const int bn_dn = mx_down_bn(bn);
+    const int32_t* np_dn = at<int32_t>(ws, W.nt_prefix2);
+    const int max_ntiles_dn = (P + bn_dn - 1) / bn_dn + std::min(c.n_experts, P);
     ActMaps xm, hm;
     std::memset(&xm, 0, sizeof(xm));
     std::memset(&hm, 0, sizeof(hm));
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
       moe_status_t st = encode_3d_u8(ctx, &xm.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows);
       if (st != MOE_OK) return st;
-      st = encode_3d_u8(ctx, &hm.m[i], at<void>(ws, W.hq), c.intermediate, P, rows);
+    }
+    for (int i = 0, rows = 16; rows <= bn_dn; ++i, rows <<= 1) {
+      moe_status_t st = encode_3d_u8(ctx, &hm.m[i], at<void>(ws, W.hq), c.intermediate, P, rows);
       if (st != MOE_OK) return st;
     }
     GemmArgs a{};
@@ -437,6 +450,8 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     a.K = c.top_k;
     a.h_out = at<void>(ws, W.hq);
     a.h_sfb = at<uint8_t>(ws, W.h_sfb);
+    a.h_nt_prefix = np_dn;
+    a.h_bn = bn_dn;
     a.act_sfb = at<uint8_t>(ws, W.x_sfb);
     a.y_out = y_pair;
     a.topk_w = topk_w;
@@ -450,10 +465,11 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
       MOE_CUDA(launch_ffn_mxfp4(kGateUp, bn, xm, a, (c.intermediate / 128) * max_ntiles, s, pdl));
     }
     a.act_sfb = at<uint8_t>(ws, W.h_sfb);
+    a.nt_prefix = np_dn;
     a.plan_ready = pdl ? 1 : 0;  // the plan is at least two launches back from the down GEMM
     {
       Prof p(ctx, MOE_PROF_DOWN, s);
-      MOE_CUDA(launch_ffn_mxfp4(kDown, bn, hm, a, (c.hidden / 128) * max_ntiles, s, pdl));
+      MOE_CUDA(launch_ffn_mxfp4(kDown, bn_dn, hm, a, (c.hidden / 128) * max_ntiles_dn, s, pdl));
     }
     return MOE_OK;
   }
@@ -780,10 +796,12 @@ moe_status_t permute_impl(moe_ctx_t* ctx, const int32_t* topk_idx, int T, int32_
   if (planned) *planned = false;
   if ((long long)T * c.top_k <= kPermuteSmallMaxPairs) {
     Prof p(ctx, MOE_PROF_PERMUTE, s);
+    const bool mx2 = map_of && c.wdtype == MOE_MXFP4;  // also the down GEMM's wider N tiles
     MOE_CUDA(launch_permute_small(topk_idx, T, c.top_k, c.n_experts, counts, offsets, perm_src, perm_k, inv, map_of,
                                   bn, at<int32_t>(ws, W.list_expert), at<int32_t>(ws, W.list_map),
                                   at<int32_t>(ws, W.nt_prefix), x, c.hidden, x_perm, ctx->d_status, s, pdl,
-                                  map_of ? at<int>(ws, W.sched) : nullptr, fused_sched_entries(c.n_experts)));
+                                  map_of ? at<int>(ws, W.sched) : nullptr, fused_sched_entries(c.n_experts),
+                                  mx2 ? mx_down_bn(bn) : 0, mx2 ? at<int32_t>(ws, W.nt_prefix2) : nullptr));
     if (planned) *planned = map_of != nullptr;
     return MOE_OK;
   }
@@ -915,7 +933,8 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
     if (!planned) {
       Prof p(ctx, MOE_PROF_PERMUTE, s);
       MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl,
-                               at<int>(ws, W.sched), fused_sched_entries(E), drop));
+                               at<int>(ws, W.sched), fused_sched_entries(E), drop, mx_down_bn(bn),
+                               at<int32_t>(ws, W.nt_prefix2)));
     }
     {
       // MX e4m3 activation rows in sorted-pair order, scales in the block layout of their N tile

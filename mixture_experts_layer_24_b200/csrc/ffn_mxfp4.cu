@@ -108,13 +108,15 @@ struct MxCfg {
   static constexpr uint32_t kStageBytes = (kStageRaw + 1023u) & ~1023u;  // next stage's A stays 1024-aligned
   static constexpr int kStagesFit = (220 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
-  static constexpr int NBUF = 2;
+  // two accumulator buffers (the epilogue of one tile overlaps the next tile's MMAs) while they and the scale
+  // columns fit TMEM's 512 columns: every width but gate/up at 128, which is why gate/up stays at 64 or less
+  static constexpr int NBUF = 2 * NA * BN + 8 * NA <= 512 ? 2 : 1;
   static constexpr uint32_t kAcc = NA * BN;                 // TMEM columns of one accumulator buffer
   static constexpr uint32_t kSfCol = NBUF * kAcc;           // scale columns after the accumulators:
   static constexpr uint32_t kTmemCols = tmem_cols_for(kSfCol + 8 * NA);  // per issuer 4 weight + 4 activation
   static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 256 + 4 * BN;
   static_assert(kStages >= 2, "a pipeline needs two stages");
-  static_assert(BN <= 64, "two accumulators plus scale columns in 512 TMEM columns");
+  static_assert(NBUF * NA * BN + 8 * NA <= 512, "accumulators plus scale columns in 512 TMEM columns");
 };
 
 template <int MODE, int BN>
@@ -340,7 +342,11 @@ __global__ void __launch_bounds__(224, 1) ffn_mxfp4_kernel(const __grid_constant
           const int jj = ti.mt * 128 + r;
           uint8_t* hq = static_cast<uint8_t*>(a.h_out);
           const int KBd = a.I / 128;
-          uint8_t* hs = a.h_sfb + ((size_t)ti.ng * KBd + ti.mt) * 512 + warp;  // down stage mt, scale byte = warp
+          // h's scale blocks are laid out in the down GEMM's N tiles (width a.h_bn, a multiple of BN): pair
+          // `local` of the expert is row local % h_bn of block (N tile, K block mt); scale byte = warp
+          const int local0 = ti.row0 - a.offsets[ti.e];
+          const int ngd = a.h_nt_prefix[ti.li] + local0 / a.h_bn, n0d = local0 % a.h_bn;
+          uint8_t* hs = a.h_sfb + ((size_t)ngd * KBd + ti.mt) * 512 + warp;
 #pragma unroll 1
           for (int c = 0; c < BN; c += 16) {
             if (c >= ti.nvalid) break;
@@ -362,7 +368,7 @@ __global__ void __launch_bounds__(224, 1) ffn_mxfp4_kernel(const __grid_constant
                 const float inv = __int_as_float((127 - sexp) << 23);
                 hq[(size_t)(ti.row0 + n) * a.I + jj] =
                     static_cast<uint8_t>(__nv_cvt_float_to_fp8(hv * inv, __NV_SATFINITE, __NV_E4M3));
-                if (lane == 0) hs[16 * (n % 32) + 4 * (n / 32)] = static_cast<uint8_t>(sexp + 127);
+                if (lane == 0) hs[16 * ((n0d + n) % 32) + 4 * ((n0d + n) / 32)] = static_cast<uint8_t>(sexp + 127);
               }
             }
           }
@@ -418,6 +424,7 @@ cudaError_t launch_ffn_mxfp4(int mode, int bn, const ActMaps& act_maps, const Ge
       case 16: return launch_mx<kDown, 16>(act_maps, a, max_tiles, s, pdl);
       case 32: return launch_mx<kDown, 32>(act_maps, a, max_tiles, s, pdl);
       case 64: return launch_mx<kDown, 64>(act_maps, a, max_tiles, s, pdl);
+      case 128: return launch_mx<kDown, 128>(act_maps, a, max_tiles, s, pdl);
     }
   }
   return cudaErrorInvalidValue;

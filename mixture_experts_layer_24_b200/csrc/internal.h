@@ -87,6 +87,8 @@ struct GemmArgs {
                               // tiles of global N tile n (zeroed by the plan kernel)
   const uint8_t* act_sfb;     // MXFP4: the activation operand's E8M0 scales, blocked per N tile
   uint8_t* h_sfb;             // MXFP4 gate/up: h's scales, written blocked per N tile for the down GEMM
+  const int32_t* h_nt_prefix; // MXFP4 gate/up: [L+1] N tiles of the down GEMM per listed expert ...
+  int h_bn;                   // ... of this width (the blocks h_sfb is written in)
   int stages;                 // pipeline depth (set by the launcher)
   int est_tiles;              // host-side bound on the tiles of this launch
   int num_sms;
@@ -167,7 +169,7 @@ cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_
                                  int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
                                  int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
                                  void* x_perm, int* status, cudaStream_t s, bool pdl, int* sched = nullptr,
-                                 int sched_n = 0);
+                                 int sched_n = 0, int bn2 = 0, int32_t* nt_prefix2 = nullptr);
 
 // Permutation: rank -> scan -> scatter. chunk = tokens per warp-chunk.
 int permute_chunk_tokens(int T, int K);
@@ -192,9 +194,11 @@ struct DropArgs {
 };
 
 // FFN tile plan for the all-resident case: every expert with pairs, in order.
+// With nt_prefix2, also the prefix of N tiles of width bn2 (a down GEMM tiled
+// wider than gate/up; MXFP4).
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
                             int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched,
-                            int sched_n, const DropArgs& drop);
+                            int sched_n, const DropArgs& drop, int bn2 = 0, int32_t* nt_prefix2 = nullptr);
 // Drops the sorted pairs [p0, p1) (one unregistered expert) as above.
 cudaError_t launch_drop_pairs(int p0, int p1, const DropArgs& drop, cudaStream_t s);
 

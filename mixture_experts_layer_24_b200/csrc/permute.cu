@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
                                                          int32_t* __restrict__ list_expert,
                                                          int32_t* __restrict__ list_map,
                                                          int32_t* __restrict__ nt_prefix, int* status,
-                                                         int* __restrict__ sched, int sched_n, DropArgs drop) {
+                                                         int* __restrict__ sched, int sched_n, DropArgs drop, int bn2,
+                                                         int32_t* __restrict__ nt_prefix2) {
   __shared__ int sh[33];
   __shared__ int s_missing;
   pdl_wait();
@@ -191,6 +192,13 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
   const int pre = block_exclusive_scan_1024(nt, sh, &total);  // its barriers also publish s_missing
   if (e < E) nt_prefix[e] = pre;
   if (e == 0) nt_prefix[E] = total;
+  if (nt_prefix2) {  // block-uniform
+    const int nt2 = (e < E && nt > 0) ? (offsets[e + 1] - offsets[e] + bn2 - 1) / bn2 : 0;
+    int total2;
+    const int pre2 = block_exclusive_scan_1024(nt2, sh, &total2);
+    if (e < E) nt_prefix2[e] = pre2;
+    if (e == 0) nt_prefix2[E] = total2;
+  }
   if (!s_missing || !drop.y_pair) return;  // block-uniform
   for (int x = 0; x < E; ++x) {
     const int p0 = offsets[x], p1 = offsets[x + 1];
@@ -202,9 +210,9 @@ __global__ void __launch_bounds__(1024) ffn_plan_kernel(const int32_t* __restric
 
 cudaError_t launch_ffn_plan(const int32_t* offsets, const int32_t* map_of, int E, int bn, int32_t* list_expert,
                             int32_t* list_map, int32_t* nt_prefix, int* status, cudaStream_t s, bool pdl, int* sched,
-                            int sched_n, const DropArgs& drop) {
+                            int sched_n, const DropArgs& drop, int bn2, int32_t* nt_prefix2) {
   return launch_ex(ffn_plan_kernel, dim3(1), dim3(1024), 0, s, pdl, offsets, map_of, E, bn, list_expert, list_map,
-                   nt_prefix, status, sched, sched ? sched_n : 0, drop);
+                   nt_prefix, status, sched, sched ? sched_n : 0, drop, bn2, nt_prefix2);
 }
 
 // Pairs [p0, p1) of one unregistered expert on the host-synchronised path:
@@ -269,7 +277,8 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm_src, int32_t* __restrict__ perm_k,
     int32_t* __restrict__ inv, const int32_t* __restrict__ map_of, int bn, int32_t* __restrict__ list_expert,
     int32_t* __restrict__ list_map, int32_t* __restrict__ nt_prefix, const uint4* __restrict__ x, int vec_per_row,
-    uint4* __restrict__ x_perm, int* status, int* __restrict__ sched, int sched_n) {
+    uint4* __restrict__ x_perm, int* status, int* __restrict__ sched, int sched_n, int bn2,
+    int32_t* __restrict__ nt_prefix2) {
   __shared__ __align__(16) int s_e[kPermuteSmallMaxPairs];
   __shared__ int s_cnt[1024];
   __shared__ int s_off[1024];
@@ -342,6 +351,13 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
       const int pre = block_exclusive_scan_1024(nt, sh, &nt_total);
       if (i < E) nt_prefix[i] = pre;
       if (i == 0) nt_prefix[E] = nt_total;
+      if (nt_prefix2) {  // N tiles of the wider down GEMM (block-uniform)
+        const int nt2 = nt > 0 ? (cnt + bn2 - 1) / bn2 : 0;
+        int nt2_total;
+        const int pre2 = block_exclusive_scan_1024(nt2, sh, &nt2_total);
+        if (i < E) nt_prefix2[i] = pre2;
+        if (i == 0) nt_prefix2[E] = nt2_total;
+      }
     }
   }
   if (x_perm) {
@@ -357,13 +373,13 @@ cudaError_t launch_permute_small(const int32_t* idx, int T, int K, int E, int32_
                                  int32_t* perm_src, int32_t* perm_k, int32_t* inv, const int32_t* map_of, int bn,
                                  int32_t* list_expert, int32_t* list_map, int32_t* nt_prefix, const void* x, int H,
                                  void* x_perm, int* status, cudaStream_t s, bool pdl, int* sched,
-                                 int sched_n) {
+                                 int sched_n, int bn2, int32_t* nt_prefix2) {
   const int P = T * K;
   int ctas = 1;
   if (x_perm) ctas = std::max(1, std::min(64, (P + 31) / 32));
   return launch_ex(permute_small_kernel, dim3(ctas), dim3(1024), 0, s, pdl, idx, T, K, E, counts, offsets, perm_src,
                    perm_k, inv, map_of, bn, list_expert, list_map, nt_prefix, static_cast<const uint4*>(x), H / 8,
-                   static_cast<uint4*>(x_perm), status, sched, sched ? sched_n : 0);
+                   static_cast<uint4*>(x_perm), status, sched, sched ? sched_n : 0, bn2, nt_prefix2);
 }
 
 }  // namespace moe

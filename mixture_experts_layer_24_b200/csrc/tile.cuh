@@ -17,6 +17,7 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int cols) {
 struct TileInfo {
   int e, mapi, mt, row0, nvalid, nti;  // nti: N tiles of this expert (readers of each weight tile)
   int ng;                              // global index of the tile's N tile (nt_prefix[expert slot] + nt)
+  int li;                              // the expert's index in the launch's list
 };
 
 // The (expert, 128-row tile, N tile) of tile index `tile` (no range or status checks).
@@ -37,6 +38,7 @@ __device__ __forceinline__ void decode_tile_at(const GemmArgs& a, int m_tiles, i
   ti.nvalid = min(bn, a.offsets[ti.e + 1] - ti.row0);
   ti.nti = nti;
   ti.ng = a.nt_prefix[lo] + nt;
+  ti.li = lo;
 }
 
 __device__ __forceinline__ void tensormap_acquire(const void* map) {
