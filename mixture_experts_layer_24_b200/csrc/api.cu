@@ -183,6 +183,12 @@ struct WsLayout {
 // accumulators and ran 28% faster at 4096 tokens; a 128-wide gate/up tile has one and ran 42% slower).
 inline int mx_down_bn(int bn) { return bn >= 64 ? 128 : bn; }
 
+// bf16 down GEMM tile width on the all-resident path: 256 for chunks of at least kBf16WideDownMinT tokens (down
+// measured 8% faster at 16384 tokens and unchanged at 4096; gate/up stays at 128: at 256 it keeps one accumulator
+// and ran 27% slower).
+constexpr int kBf16WideDownMinT = 8192;
+inline int bf16_down_bn(int bn, int T) { return (bn == 128 && T >= kBf16WideDownMinT) ? 256 : bn; }
+
 WsLayout ws_layout(const moe_config_t& c, int T) {
   WsLayout L{};
   const size_t P = (size_t)T * c.top_k, E = c.n_experts, H = c.hidden, I = c.intermediate;
@@ -209,7 +215,7 @@ WsLayout ws_layout(const moe_config_t& c, int T) {
   L.list_expert = take((2 * E + 64) * 4);
   L.list_map = take((2 * E + 64) * 4);
   L.nt_prefix = take((2 * E + 64) * 4);
-  L.nt_prefix2 = take(mx ? (E + 1) * 4 : 0);
+  L.nt_prefix2 = take((E + 1) * 4);
   L.sched = take((size_t)fused_sched_entries((int)E) * 4);
   L.x_perm = take(P * H * ((fp8 || mx) ? 1 : 2));
   L.x_scale = take(fp8 ? P * (H / 128) * 4 : 0);
@@ -412,11 +418,12 @@ moe_status_t lru_push_async(moe_slots_t* sl, cudaStream_t s) {
 
 // Runs the two GEMMs (and, for FP8, the quantiser of h between them) for one
 // expert list whose arrays live in the workspace at list offset `lo`.
+// nt_prefix_dn / bn_dn (bf16): the down GEMM's own, wider N tiling (from the plan kernel), or null for bn.
 moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void* ws, int T, int bn,
                        const int32_t* perm_src, const int32_t* perm_k, const int32_t* offsets, const float* topk_w,
                        float* y_pair, const int32_t* list_expert, const int32_t* list_map, const int32_t* nt_prefix,
                        int L, int max_ntiles, cudaStream_t s, bool pdl, bool plan_ready_gu,
-                       int* sched = nullptr) {
+                       int* sched = nullptr, const int32_t* nt_prefix_dn = nullptr, int bn_dn = 0) {
   const moe_config_t& c = ctx->cfg;
   const bool fp8 = c.wdtype == MOE_FP8_E4M3_B128;
   const int P = T * c.top_k;
@@ -491,6 +498,8 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
       st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, kBf16GateUpChunks);
       if (st != MOE_OK) return st;
+    }
+    for (int i = 0, rows = 16; rows <= std::max(bn, bn_dn); ++i, rows <<= 1) {
       st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, kBf16DownChunks);
       if (st != MOE_OK) return st;
     }
@@ -592,10 +601,16 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     a.act_scale = at<float>(ws, W.h_scale);
   }
   a.plan_ready = pdl ? 1 : 0;  // the plan is at least two launches back from the down GEMM
-  a.est_tiles = (c.hidden / 128) * std::min(max_ntiles, max_experts * ((P + bn - 1) / bn));
+  int bnd = bn, max_ntiles_d = max_ntiles;
+  if (nt_prefix_dn && bn_dn > bn) {
+    bnd = bn_dn;
+    a.nt_prefix = nt_prefix_dn;
+    max_ntiles_d = (P + bnd - 1) / bnd + std::min(L, P);
+  }
+  a.est_tiles = (c.hidden / 128) * std::min(max_ntiles_d, max_experts * ((P + bnd - 1) / bnd));
   {
     Prof p(ctx, MOE_PROF_DOWN, s);
-    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bn, hmap, &hmaps, a, (c.hidden / 128) * max_ntiles, s, pdl));
+    MOE_CUDA(launch_ffn_gemm(kDown, c.wdtype, bnd, hmap, &hmaps, a, (c.hidden / 128) * max_ntiles_d, s, pdl));
   }
   return MOE_OK;
 }
@@ -953,11 +968,13 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
       sl->stats.last_touched = -1;
     }
     bool plan_ready_gu = false;
+    const int bn_dn = c.wdtype == MOE_BF16 && !planned ? bf16_down_bn(bn, T) : bn;
     if (!planned) {
       {
         Prof p(ctx, MOE_PROF_PERMUTE, s);
         MOE_CUDA(launch_ffn_plan(offsets, sl->d_map_of, E, bn, le, lm, np, ctx->d_status, s, pdl,
-                                 at<int>(ws, W.sched), fused_sched_entries(E), drop));
+                                 at<int>(ws, W.sched), fused_sched_entries(E), drop, bn_dn,
+                                 bn_dn != bn ? at<int32_t>(ws, W.nt_prefix2) : nullptr));
       }
       Prof pg(ctx, MOE_PROF_GATHER, s);
       if (fp8) {
@@ -972,7 +989,8 @@ moe_status_t ffn_impl(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const int3
       plan_ready_gu = pdl;  // permutation+plan -> quantiser -> gate/up
     }
     return run_gemms(ctx, sl, W, ws, T, bn, perm_src, perm_k, offsets, topk_w, y_pair, le, lm, np, E, ntile_bound,
-                     s, ctx->chain, plan_ready_gu, at<int>(ws, W.sched));
+                     s, ctx->chain, plan_ready_gu, at<int>(ws, W.sched),
+                     bn_dn != bn ? at<int32_t>(ws, W.nt_prefix2) : nullptr, bn_dn);
   }
 
   // activation rows in sorted-pair order (quantised for FP8); no PDL on the host-synchronised path

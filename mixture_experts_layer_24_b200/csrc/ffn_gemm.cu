@@ -736,6 +736,9 @@ static cudaError_t launch_mode(int wdtype, int bn, const CUtensorMap& map, const
       case 32: return launch_bf16<MODE, 32>(*maps, a, grid, s, pdl);
       case 64: return launch_bf16<MODE, 64>(*maps, a, grid, s, pdl);
       case 128: return launch_bf16<MODE, 128>(*maps, a, grid, s, pdl);
+      case 256:
+        if constexpr (MODE == kDown) return launch_bf16<MODE, 256>(*maps, a, grid, s, pdl);  // wide down tiles
+        break;
     }
     return cudaErrorInvalidValue;
   }

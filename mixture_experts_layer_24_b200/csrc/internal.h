@@ -94,10 +94,10 @@ struct GemmArgs {
   int num_sms;
 };
 
-// Activation-operand TMA descriptors for box heights 16, 32, 64, 128 rows
-// (the GEMMs pick, per tile, the smallest that holds its pairs).
+// Activation-operand TMA descriptors for box heights 16 .. 256 rows (the GEMMs
+// pick, per tile, the smallest that holds its pairs).
 struct alignas(64) ActMaps {
-  CUtensorMap m[4];
+  CUtensorMap m[5];  // 16, 32, 64, 128, 256 (the bf16 down GEMM's widest tile)
 };
 
 // Launches one FFN GEMM (gate/up+SwiGLU or down*weight) over the tile list.
