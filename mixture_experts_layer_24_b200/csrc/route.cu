@@ -13,6 +13,7 @@
 // token alone, whatever the batch.
 #include "common.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -178,77 +179,7 @@ cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, 
 }
 
 // ------------------------------------------------- warp top-k (registers) --
-// The token's logits sit in registers, NJ = ceil(E/32) per lane (expert
-// lane + 32 j). Each of the K rounds takes the lane's best expert not yet
-// taken (a tree over its NJ slots), then a warp arg-max; all comparisons use
-// the same total order (logit desc, expert asc), so ties (+0 == -0 included)
-// go to the lower index. Weights as in topk_kernel. Logits are read through L2
-// (ld.global.cg): other CTAs wrote them.
-struct Cand {
-  float v;
-  int e;  // INT_MAX = none
-};
-
-__device__ __forceinline__ Cand better(Cand a, Cand b) {
-  if (b.e == 0x7fffffff) return a;
-  if (a.e == 0x7fffffff) return b;
-  return ranks_before(a.v, a.e, b.v, b.e) ? a : b;
-}
-
-template <int NJ>
-__device__ __forceinline__ void topk_warp(const float* l, int E, int K, int32_t* idx, float* w) {
-  const int lane = threadIdx.x & 31;
-  float v[NJ];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = e < E ? __ldcg(l + e) : 0.0f;
-    if (e >= E) taken |= 1u << j;
-  }
-  float my_v = 0.0f;
-  int my_e = 0;
-  for (int r = 0; r < K; ++r) {
-    Cand c[NJ];
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) c[j] = Cand{v[j], ((taken >> j) & 1u) ? 0x7fffffff : lane + 32 * j};
-#pragma unroll
-    for (int step = 1; step < NJ; step <<= 1) {
-#pragma unroll
-      for (int j = 0; j + step < NJ; j += 2 * step) c[j] = better(c[j], c[j + step]);
-    }
-    Cand b = c[0];
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      Cand other{__shfl_xor_sync(0xffffffffu, b.v, o), __shfl_xor_sync(0xffffffffu, b.e, o)};
-      b = better(b, other);
-    }
-    if (b.e != 0x7fffffff && (b.e & 31) == lane) taken |= 1u << (b.e >> 5);
-    if (lane == r) {
-      my_v = b.v;
-      my_e = b.e;
-    }
-  }
-  const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
-  const float ex = (lane < K) ? expf(my_v - l0) : 0.0f;
-  float sum = 0.0f;
-  for (int k = 0; k < K; ++k) sum = sum + __shfl_sync(0xffffffffu, ex, k);
-  if (lane < K) {
-    idx[lane] = my_e;
-    w[lane] = ex / sum;
-  }
-}
-
-__device__ __forceinline__ void topk_warp_any(const float* l, int E, int K, int32_t* idx, float* w) {
-  const int nj = (E + 31) >> 5;
-  if (nj <= 1) topk_warp<1>(l, E, K, idx, w);
-  else if (nj <= 4) topk_warp<4>(l, E, K, idx, w);
-  else if (nj <= 8) topk_warp<8>(l, E, K, idx, w);
-  else if (nj <= 12) topk_warp<12>(l, E, K, idx, w);
-  else if (nj <= 16) topk_warp<16>(l, E, K, idx, w);
-  else topk_warp<32>(l, E, K, idx, w);
-}
-
+// One warp per token (topk.cuh: redux arg-max over order-preserving keys).
 __global__ void __launch_bounds__(256) topk_warp_kernel(const float* __restrict__ logits, int T, int E, int K,
                                                          int32_t* __restrict__ idx, float* __restrict__ w) {
   pdl_wait();
@@ -265,64 +196,89 @@ cudaError_t launch_topk_warp(const float* logits, int T, int E, int K, int32_t* 
 }
 
 // --------------------------------------------- register-tiled router GEMM --
-// fp32 GEMM in the same order. A warp owns WT tokens x WE experts and its lane
-// j keeps the WT*WE lane-j partials; NWT x NWE warps make the CTA tile
-// (TT = WT*NWT tokens, TE = WE*NWE experts). Each stage holds 256 consecutive
-// h of the tile's tokens and experts in shared memory as stored (cp.async,
-// kRgStages buffers, kRgStages - 1 in flight); lane j reads h = h0 + j + 32q,
-// q = 0..7: consecutive lanes, consecutive elements.
+// fp32 GEMM in the same order. A warp owns WT tokens x WE experts; NWT x NWE
+// warps make the CTA tile (TT = WT*NWT tokens, TE = WE*NWE experts). Each
+// stage holds 256 consecutive h of the tile's tokens and experts in shared
+// memory as stored (cp.async, kRgStages buffers, kRgStages - 1 in flight).
+// Each thread copies the same 16-byte parts of the same rows in every stage,
+// so their offsets are computed once.
+//
+// Lane (half, i) = (lane / 16, lane % 16) runs the two order chains 2i and
+// 2i+1 of the tokens 2m + half (m = 0 .. WT/2-1) against all WE experts: one
+// 32-bit load brings x[h], x[h+1] (h = h0 + 32q + 2i) of a token, one 64-bit
+// load the matching pair of Wr[e], and one paired FMA advances both chains.
+// The chains keep the order above (chain c runs h = c, c+32, ... in
+// increasing h), and the xor butterfly's offsets 16 .. 2 become lane offsets
+// 8 .. 1 inside each half, its offset 1 the sum of a lane's two chains. Token
+// rows are staged 576 bytes apart, so the two halves' rows (even and odd
+// tokens) fall in different banks.
 //   prefill:          WT = 8, WE = 8, 4 x 2 warps (32 tokens x 16 experts; two
-//                     CTAs per SM, 114 registers: each hides the other's stage
-//                     barriers; measured 4-6% faster than one 12-warp CTA, while
-//                     token-pair staging, wider tiles and more warps were not)
+//                     CTAs per SM: each hides the other's stage barriers)
 //   16 < T <= 64:     WT = 4, WE = 8, 2 x 2 warps (8 x 16)
 //   8 < T <= 16:      WT = 4, WE = 4, 2 x 2 warps (8 x 8)
 constexpr int kRgStages = 3;
+constexpr int kRgXPitch = 256 * 2 + 64;  // bytes per staged token row
 
 template <int WT, int WE, int NWT, int NWE>
 struct RgCfg {
   static constexpr int TT = WT * NWT, TE = WE * NWE, kThreads = 32 * NWT * NWE;
-  static constexpr size_t kStageBytes = (size_t)TT * 256 * 2 + (size_t)TE * 256 * 4;
+  static constexpr size_t kXBytes = (size_t)TT * kRgXPitch;
+  static constexpr size_t kStageBytes = kXBytes + (size_t)TE * 256 * 4;
   static constexpr size_t kSmem = kRgStages * kStageBytes;
+  static constexpr int kXCopies = TT * 32 / kThreads, kWCopies = TE * 64 / kThreads;  // 16-byte parts per thread
+  static_assert(TT * 32 % kThreads == 0 && TE * 64 % kThreads == 0, "whole parts per thread");
+  static_assert(kXBytes % 16 == 0, "Wr tile stays 16-byte aligned");
 };
 
 template <int WT, int WE, int NWT, int NWE>
-__global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(32 * NWT * NWE, 2) route_gemm_kernel(const uint16_t* __restrict__ x,
                                                                         const float* __restrict__ wr,
                                                                         const float* __restrict__ bias, int T, int H,
                                                                         int E, float* __restrict__ logits,
                                                                         int* __restrict__ sched, int sched_n) {
   using C = RgCfg<WT, WE, NWT, NWE>;
   constexpr int TT = C::TT, TE = C::TE, NT = C::kThreads;
+  static_assert(WT % 2 == 0, "each half-warp takes half of a warp's tokens");
   extern __shared__ __align__(16) uint8_t sm[];
   pdl_wait();  // x may come from the previous kernel
   pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int half = lane >> 4, li = lane & 15;
   if (blockIdx.x == 0 && blockIdx.y == 0)  // counters of the decode FFN that follows (first kernel of the forward)
     for (int i = tid; i < sched_n; i += NT) sched[i] = 0;
   const int tt0 = (warp / NWE) * WT, ee0 = (warp % NWE) * WE;
   const int tb = blockIdx.y * TT, eb = blockIdx.x * TE;
   const int nsteps = H / 256;
-  auto xs = [&](int buf) { return reinterpret_cast<uint16_t*>(sm + buf * C::kStageBytes); };
-  auto ws = [&](int buf) { return reinterpret_cast<float*>(sm + buf * C::kStageBytes + (size_t)TT * 256 * 2); };
+  // this thread's parts: token row tid/32 + k*NT/32, part tid%32 (8 bf16);
+  // expert row tid/64 + k*NT/64, part tid%64 (4 fp32). Rows past T or E
+  // re-read the last row (results discarded). Offsets in elements (< 2^29).
+  uint32_t xoff[C::kXCopies], woff[C::kWCopies];
+#pragma unroll
+  for (int k = 0; k < C::kXCopies; ++k)
+    xoff[k] = (uint32_t)min(tb + (tid >> 5) + k * (NT / 32), T - 1) * (uint32_t)H + (uint32_t)(tid & 31) * 8u;
+#pragma unroll
+  for (int k = 0; k < C::kWCopies; ++k)
+    woff[k] = (uint32_t)min(eb + (tid >> 6) + k * (NT / 64), E - 1) * (uint32_t)H + (uint32_t)(tid & 63) * 4u;
+  const uint32_t xdst0 = (uint32_t)((tid >> 5) * kRgXPitch + (tid & 31) * 16);
+  const uint32_t wdst0 = (uint32_t)(C::kXBytes + (tid >> 6) * 1024 + (tid & 63) * 16);
+  const uint32_t sbase = smem_u32(sm);
   auto load_stage = [&](int st, int buf) {
-    const int h0 = st * 256;
-    uint16_t* xd = xs(buf);
-    float* wd = ws(buf);
-    for (int c = tid; c < TT * 32; c += NT) {  // token row: 32 x 16 B
-      const int t = c >> 5, part = c & 31;
-      const int row = min(tb + t, T - 1);  // rows past T re-read row T-1 (results discarded)
-      cp_async16(xd + (size_t)t * 256 + part * 8, x + (size_t)row * H + h0 + part * 8);
-    }
-    for (int c = tid; c < TE * 64; c += NT) {  // expert row: 64 x 16 B
-      const int e = c >> 6, part = c & 63;
-      const int row = min(eb + e, E - 1);
-      cp_async16(wd + (size_t)e * 256 + part * 4, wr + (size_t)row * H + h0 + part * 4);
-    }
+    const uint16_t* xs0 = x + (size_t)st * 256;
+    const float* ws0 = wr + (size_t)st * 256;
+    const uint32_t d = sbase + (uint32_t)(buf * C::kStageBytes);
+#pragma unroll
+    for (int k = 0; k < C::kXCopies; ++k)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + xdst0 + k * (NT / 32) * kRgXPitch),
+                   "l"(xs0 + xoff[k])
+                   : "memory");
+#pragma unroll
+    for (int k = 0; k < C::kWCopies; ++k)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + wdst0 + k * (NT / 64) * 1024),
+                   "l"(ws0 + woff[k])
+                   : "memory");
   };
 
-  static_assert(WT % 2 == 0, "tokens go in pairs");
-  uint64_t acc2[WT / 2][WE];  // (token 2m, token 2m+1) partials of expert j
+  uint64_t acc2[WT / 2][WE];  // (chain 2i, chain 2i+1) of token tt0 + 2m + half, expert ee0 + j
 #pragma unroll
   for (int m = 0; m < WT / 2; ++m)
 #pragma unroll
@@ -333,52 +289,52 @@ __global__ void __launch_bounds__(32 * NWT * NWE, 1) route_gemm_kernel(const uin
     if (st < nsteps) load_stage(st, st);
     asm volatile("cp.async.commit_group;" ::: "memory");  // empty groups keep the count uniform
   }
+  int buf = 0;
   for (int st = 0; st < nsteps; ++st) {
-    const int buf = st % kRgStages;
     {
       const int nx = st + kRgStages - 1;  // its buffer was last read in iteration st - 1
-      if (nx < nsteps) load_stage(nx, nx % kRgStages);
+      int nbuf = buf + kRgStages - 1;
+      if (nbuf >= kRgStages) nbuf -= kRgStages;
+      if (nx < nsteps) load_stage(nx, nbuf);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("cp.async.wait_group %0;" ::"n"(kRgStages - 1) : "memory");
     __syncthreads();
-    const uint16_t* xb = xs(buf) + (size_t)tt0 * 256 + lane;
-    const float* wb = ws(buf) + (size_t)ee0 * 256 + lane;
-#pragma unroll 2
+    const uint8_t* xb = sm + buf * C::kStageBytes + (size_t)(tt0 + half) * kRgXPitch + 4 * li;
+    const float* wb = reinterpret_cast<const float*>(sm + buf * C::kStageBytes + C::kXBytes) + (size_t)ee0 * 256 + 2 * li;
+#pragma unroll
     for (int q = 0; q < 8; ++q) {
       uint64_t xp[WT / 2];
 #pragma unroll
-      for (int m = 0; m < WT / 2; ++m)
-        xp[m] = pack2(bf16_lo(xb[(size_t)(2 * m) * 256 + 32 * q]), bf16_lo(xb[(size_t)(2 * m + 1) * 256 + 32 * q]));
+      for (int m = 0; m < WT / 2; ++m) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(xb + (size_t)(2 * m) * kRgXPitch + 64 * q);
+        xp[m] = ((uint64_t)(v & 0xffff0000u) << 32) | (uint64_t)(v << 16);  // fp32 of bf16 x[h] (low), x[h+1]
+      }
 #pragma unroll
       for (int j = 0; j < WE; ++j) {
-        const float wv = wb[(size_t)j * 256 + 32 * q];
-        const uint64_t wp = pack2(wv, wv);
+        const uint64_t wp = *reinterpret_cast<const uint64_t*>(wb + (size_t)j * 256 + 32 * q);
 #pragma unroll
         for (int m = 0; m < WT / 2; ++m) fma2(acc2[m][j], xp[m], wp);
       }
     }
     __syncthreads();
+    if (++buf == kRgStages) buf = 0;
   }
-  float acc[WT][WE];
 #pragma unroll
-  for (int m = 0; m < WT / 2; ++m)
+  for (int m = 0; m < WT / 2; ++m) {
+    const int t = tb + tt0 + 2 * m + half;
 #pragma unroll
-    for (int j = 0; j < WE; ++j) unpack2(acc2[m][j], acc[2 * m][j], acc[2 * m + 1][j]);
+    for (int j = 0; j < WE; ++j) {
+      float lo, hi;
+      unpack2(acc2[m][j], lo, hi);
 #pragma unroll
-  for (int i = 0; i < WT; ++i)
-#pragma unroll
-    for (int j = 0; j < WE; ++j) butterfly_sum(acc[i][j]);
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < WT; ++i) {
-      const int t = tb + tt0 + i;
-      if (t >= T) continue;
-#pragma unroll
-      for (int j = 0; j < WE; ++j) {
-        const int e = eb + ee0 + j;
-        if (e < E) logits[(size_t)t * E + e] = bias ? acc[i][j] + bias[e] : acc[i][j];
+      for (int o = 8; o >= 1; o >>= 1) {  // chain offsets 16, 8, 4, 2
+        lo = lo + __shfl_xor_sync(0xffffffffu, lo, o);
+        hi = hi + __shfl_xor_sync(0xffffffffu, hi, o);
       }
+      const float r = lo + hi;  // chain offset 1
+      const int e = eb + ee0 + j;
+      if (li == 0 && t < T && e < E) logits[(size_t)t * E + e] = bias ? r + bias[e] : r;
     }
   }
 }

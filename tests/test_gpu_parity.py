@@ -140,6 +140,32 @@ def test_route_ties_go_to_lower_index():
     layer.close()
 
 
+@pytest.mark.parametrize("T", [1, 3, 8, 16, 40])
+def test_ties_through_the_decode_forward(T):
+    """Tied logits through the decode forward (the router's fused last-CTA
+    top-k up to 4 tokens, the warp top-k kernel above): router rows repeat
+    with period 13, so experts e, e+13, e+26 (and 39) tie, and the top-8
+    boundary cuts through a tied group. The lower index wins and goes first,
+    as in the oracle; a wrong pick brings another expert's FFN into the
+    output, a wrong order changes the bits of the k-ordered sum."""
+    H, E, K, I = 256, 40, 8, 128
+    case = LayerCase(T, H, E, K, I, seed=7 + T)
+    case.wr = case.wr[torch.arange(E, device=case.dev) % 13].contiguous()
+    out = oracle.as_u16(case.forward())
+    torch.cuda.synchronize()
+    assert case.layer.status() == 0
+    ref = case.oracle_forward()
+    lo = np.sort(oracle.route(*case.oracle_inputs(), K)[0], axis=1)[:, ::-1]
+    assert np.all(lo[:, K - 1] == lo[:, K]), "the top-8 boundary cuts through a tied group"
+    idx, _ = case.layer.route(case.x, case.wr, case.bias)
+    assert np.array_equal(idx.cpu().numpy(), ref["idx"])
+    assert_close_out(out, ref["out"], TOL_BF16)
+    # the same tokens inside a 200-token batch (router GEMM + top-k kernel): the same bits
+    xb = torch.cat([case.x, synth.tokens(200 - T, H, seed=99, device=case.dev)]).contiguous()
+    assert np.array_equal(oracle.as_u16(case.layer.forward(xb, case.wr, case.bias))[:T], out)
+    case.close()
+
+
 # ---------------------------------------------------------------- permute --
 
 @pytest.mark.parametrize("T,E,K,mode", [(1, 384, 8, "rand"), (17, 8, 2, "rand"), (4096, 384, 8, "zipf"),
