@@ -499,8 +499,9 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
       st = encode_3d_bf16(ctx, &xmaps.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, kBf16GateUpChunks);
       if (st != MOE_OK) return st;
     }
-    for (int i = 0, rows = 16; rows <= std::max(bn, bn_dn); ++i, rows <<= 1) {
-      st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, kBf16DownChunks);
+    const int bn_down = (nt_prefix_dn && bn_dn > bn) ? bn_dn : bn;  // the down GEMM's N tile width
+    for (int i = 0, rows = 16; rows <= bn_down; ++i, rows <<= 1) {
+      st = encode_3d_bf16(ctx, &hmaps.m[i], at<void>(ws, W.h), c.intermediate, P, rows, bf16_down_gemm_chunks(bn_down));
       if (st != MOE_OK) return st;
     }
     xmap = xmaps.m[0];
@@ -539,10 +540,13 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
   }
   if (fused_ok && !fp8) {
     // decode: both GEMMs in one launch (x with one K chunk per box, h with two)
-    ActMaps x1;
+    ActMaps x1, h2;
     std::memset(&x1, 0, sizeof(x1));
+    std::memset(&h2, 0, sizeof(h2));
     for (int i = 0, rows = 16; rows <= bn; ++i, rows <<= 1) {
       st = encode_3d_bf16(ctx, &x1.m[i], at<void>(ws, W.x_perm), c.hidden, P, rows, 1);
+      if (st != MOE_OK) return st;
+      st = encode_3d_bf16(ctx, &h2.m[i], at<void>(ws, W.h), c.intermediate, P, rows, 2);
       if (st != MOE_OK) return st;
     }
     GemmArgs a{};
@@ -564,7 +568,7 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     a.sched = sched;
     a.num_sms = ctx->num_sms;
     Prof p(ctx, MOE_PROF_FFN_FUSED, s);
-    MOE_CUDA(launch_ffn_fused(bn, x1, hmaps, a, (c.intermediate / 128 + c.hidden / 128) * max_ntiles, s, pdl));
+    MOE_CUDA(launch_ffn_fused(bn, x1, h2, a, (c.intermediate / 128 + c.hidden / 128) * max_ntiles, s, pdl));
     return MOE_OK;
   }
   GemmArgs a{};
@@ -601,7 +605,7 @@ moe_status_t run_gemms(moe_ctx_t* ctx, moe_slots_t* sl, const WsLayout& W, void*
     a.act_scale = at<float>(ws, W.h_scale);
   }
   a.plan_ready = pdl ? 1 : 0;  // the plan is at least two launches back from the down GEMM
-  int bnd = bn, max_ntiles_d = max_ntiles;
+  int bnd = bn, max_ntiles_d = max_ntiles;  // bnd: as the h maps above were encoded
   if (nt_prefix_dn && bn_dn > bn) {
     bnd = bn_dn;
     a.nt_prefix = nt_prefix_dn;

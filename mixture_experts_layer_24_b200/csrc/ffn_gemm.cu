@@ -32,12 +32,17 @@
 namespace moe {
 
 // bf16: one pipeline stage holds kKC consecutive 64-wide K chunks, fetched by
-// one 3-D TMA copy per operand (one chunk for gate/up, two for down: the
-// depths measured fastest).
+// one 3-D TMA copy per operand. NA weight operands share each staged
+// activation tile, each with its own accumulator: gate/up stages the gate and
+// up rows of the same 128 rows; down, up to BN = 128, stages two consecutive
+// 128-row blocks of the output, so each h tile comes from L2 once per 256
+// output rows (at BN = 256 one operand: two accumulators of 256 columns would
+// not fit twice in TMEM). Two-operand stages hold one chunk, one-operand
+// stages two (the depths measured fastest).
 template <int MODE, int BN>
 struct Bf16Cfg {
-  static constexpr int NA = MODE == kGateUp ? 2 : 1;
-  static constexpr int KC = MODE == kGateUp ? kBf16GateUpChunks : kBf16DownChunks;
+  static constexpr int KC = MODE == kGateUp ? kBf16GateUpChunks : bf16_down_gemm_chunks(BN);
+  static constexpr int NA = (MODE == kGateUp || KC == 1) ? 2 : 1;
   static constexpr uint32_t kChunkA = kABytes;     // 128 rows x 128 B
   static constexpr uint32_t kChunkB = BN * 128;    // BN rows x 128 B
   static constexpr uint32_t kStageBytes = KC * (NA * kChunkA + kChunkB);
@@ -67,7 +72,9 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
   constexpr uint32_t B_OFF = NA * A_OP;        // stage: [A gate][A up][B], kKC chunks each
   constexpr uint32_t ACC = NA * BN;            // TMEM columns of one accumulator buffer
   constexpr int S = C::kStagesMax;  // compile-time depth: no division by a launch value in the K loops
-  const int m_tiles = (MODE == kGateUp ? a.I : a.H) / 128;
+  // weight tiles of NA operands; with an odd number of 128-row blocks in H the last down tile's second block lies
+  // past the weight rows: its TMA box reads the zero fill and its results are not stored
+  const int m_tiles = MODE == kGateUp ? a.I / 128 : (a.H + 128 * NA - 1) / (128 * NA);
   const int KB = (MODE == kGateUp ? a.H : a.I) / (64 * kKC);  // K steps per tile
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -139,6 +146,9 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
         const void* wmap = MODE == kGateUp ? static_cast<const void*>(kKC == 1 ? &me->gu : &me->gu2)
                                            : static_cast<const void*>(kKC == 1 ? &me->dn : &me->dn2);
         tensormap_acquire(wmap);
+        // weight rows of the two operands: gate and up rows of the same 128 rows, or (down) two consecutive blocks
+        const int ra0 = MODE == kGateUp ? ti.mt * 128 : ti.mt * 128 * NA;
+        const int ra1 = MODE == kGateUp ? a.I + ti.mt * 128 : ra0 + 128;
         int kb = 0;
         if (first) {
           first = false;
@@ -148,8 +158,8 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
           for (int j = 0; j < npre; ++j) {
             const uint32_t st = base + j * STAGE;
             mbar_arrive_expect_tx(full(j), stage_tx);
-            tma_load_3d_hint(st, wmap, full(j), 0, ti.mt * 128, j * kKC, pol_w);
-            if (MODE == kGateUp) tma_load_3d_hint(st + A_OP, wmap, full(j), 0, a.I + ti.mt * 128, j * kKC, pol_w);
+            tma_load_3d_hint(st, wmap, full(j), 0, ra0, j * kKC, pol_w);
+            if (NA == 2) tma_load_3d_hint(st + A_OP, wmap, full(j), 0, ra1, j * kKC, pol_w);
           }
           if (a.plan_ready) {
             pdl_wait();
@@ -168,8 +178,8 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
           }
           const uint32_t st = base + s * STAGE;
           mbar_arrive_expect_tx(full(s), stage_tx);
-          tma_load_3d_hint(st, wmap, full(s), 0, ti.mt * 128, kb * kKC, pol_w);
-          if (MODE == kGateUp) tma_load_3d_hint(st + A_OP, wmap, full(s), 0, a.I + ti.mt * 128, kb * kKC, pol_w);
+          tma_load_3d_hint(st, wmap, full(s), 0, ra0, kb * kKC, pol_w);
+          if (NA == 2) tma_load_3d_hint(st + A_OP, wmap, full(s), 0, ra1, kb * kKC, pol_w);
           tma_load_3d(st + B_OFF, amap, full(s), 0, ti.row0, kb * kKC);
         }
       }
@@ -180,7 +190,8 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
       pdl_trigger();
     }
   } else if (warp == 5 || warp == 6) {
-    // ------------------------------------------------------------ MMA issuers: warp 5 gate (or down), warp 6 up
+    // ------------------------------------------------------------ MMA issuers: warp 5 gate (or the first down
+    // block), warp 6 up (or the second)
     // (each tcgen05 instruction holds its issuing thread for tens of cycles, about as long as a 128 x 128 x 16
     // MMA computes, so two threads issue the two accumulators' MMAs)
     if (a.plan_ready) {
@@ -292,16 +303,21 @@ __global__ void __launch_bounds__(224, 1) ffn_bf16_kernel(const __grid_constant_
             }
           }
         } else {
-          const int o = ti.mt * 128 + r;
+          const int o = ti.mt * 128 * NA + r;  // output column of accumulator 0; accumulator 1 is 128 further
 #pragma unroll 1
           for (int c = 0; c < BN; c += 16) {
             if (c >= ti.nvalid) break;
-            uint32_t v[16];
+            uint32_t v[16], v1[16];
             tmem_ld16(tl + c, v);
+            if (NA == 2) tmem_ld16(tl + BN + c, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
-              if (c + q < ti.nvalid) a.y_out[(size_t)(ti.row0 + c + q) * a.H + o] = wcol[c + q] * __uint_as_float(v[q]);
+              if (c + q < ti.nvalid) {
+                float* yrow = a.y_out + (size_t)(ti.row0 + c + q) * a.H;
+                yrow[o] = wcol[c + q] * __uint_as_float(v[q]);
+                if (NA == 2 && o + 128 < a.H) yrow[o + 128] = wcol[c + q] * __uint_as_float(v1[q]);
+              }
             }
           }
         }

@@ -36,10 +36,17 @@ enum FfnMode { kGateUp = 0, kDown = 1 };
 // 64-wide K chunks per pipeline stage (one 3-D TMA copy per operand) of the
 // bf16 GEMMs, measured at BN = 128 (4096 and 16384 tokens): gate/up streams
 // two weight operands per chunk, and one-chunk stages (4 of 48 KB in flight
-// instead of 2 of 96 KB) ran 4-10% faster; down stages are half that size,
-// and two-chunk stages (3 of 64 KB) ran 7-24% faster than one-chunk ones.
+// instead of 2 of 96 KB) ran 4-10% faster. A down GEMM with one weight
+// operand has stages half that size, where two-chunk stages (3 of 64 KB) ran
+// 7-24% faster than one-chunk ones; with two weight operands (two output
+// blocks per h tile) it takes the gate/up depth.
 constexpr int kBf16GateUpChunks = 1;
 constexpr int kBf16DownChunks = 2;
+// Chunks per stage of the separate bf16 down GEMM at N tile width bn: up to
+// 128 it stages two weight operands (two 128-row output blocks) against each
+// h tile, one chunk per stage like gate/up; at 256, one operand and two
+// chunks. Its h tensor maps carry the same count per box.
+constexpr int bf16_down_gemm_chunks(int bn) { return bn <= 128 ? kBf16GateUpChunks : kBf16DownChunks; }
 
 // Launches `kern` on `s`, with programmatic stream serialisation when pdl is
 // true (the kernel must then follow the pdl_wait / pdl_trigger rule).
