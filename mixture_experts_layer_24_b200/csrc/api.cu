@@ -781,16 +781,21 @@ namespace {
 // stream serialisation (only when the preceding launch is this library's own
 // kernel of the same forward).
 
+// rd / map_of / planned: the device-side residency plan, which the decode router's last CTA runs after the top-k
+// when it can (*planned = true); otherwise the caller launches it.
 moe_status_t route_impl(moe_ctx_t* ctx, const void* x, const float* w_router, const float* logit_bias, int T,
                         int32_t* topk_idx, float* topk_w, void* ws, cudaStream_t s, int* sched = nullptr,
-                        int sched_n = 0) {
+                        int sched_n = 0, const ResidencyDev* rd = nullptr, int32_t* map_of = nullptr,
+                        bool* planned = nullptr) {
+  if (planned) *planned = false;
   const moe_config_t& c = ctx->cfg;
   const WsLayout W = ws_layout(c, T);
   float* logits = at<float>(ws, W.logits);
   if (T <= kRouteSmallMaxT) {
     Prof p(ctx, MOE_PROF_ROUTER, s);
     MOE_CUDA(launch_route_small(x, w_router, logit_bias, T, c.hidden, c.n_experts, c.top_k, logits, topk_idx,
-                                topk_w, ctx->d_counters, ctx->d_status, s, ctx->chain, sched, sched_n));
+                                topk_w, ctx->d_counters, ctx->d_status, s, ctx->chain, sched, sched_n, rd, map_of,
+                                planned));
     return MOE_OK;
   }
   {
@@ -1280,8 +1285,11 @@ moe_status_t moe_forward(moe_ctx_t* ctx, moe_slots_t* sl, const void* x, const f
     // every routed expert is resident or cached) -> FFN planned from the top-k -> combine
     int* sched = at<int>(ws, W.sched);
     const int sched_n = 1 + std::min(c.n_experts, T * c.top_k);
-    if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n)) != MOE_OK) return st;
-    {
+    bool planned = false;  // up to 4 tokens the router's last CTA runs the cache plan after the top-k
+    if ((st = route_impl(ctx, x, w_router, logit_bias, T, idx, w, ws, s, sched, sched_n, &sl->rdev, sl->d_map_of,
+                         &planned)) != MOE_OK)
+      return st;
+    if (!planned) {
       Prof p(ctx, MOE_PROF_PERMUTE, s);
       MOE_CUDA(launch_residency_plan(idx, T * c.top_k, c.n_experts, sl->rdev, sl->d_map_of, s, chain));
     }

@@ -158,9 +158,13 @@ cudaError_t launch_topk(const float* logits, int T, int E, int K, int32_t* idx, 
 // counters: >= kRouteSmallMaxT zero-initialised words owned by the caller's
 // context (each is returned to zero by the kernel that uses it).
 constexpr int kRouteSmallMaxT = 64;
+// rd / map_of: up to 4 tokens (one CTA then holds every token's top-k) the
+// fused last CTA also runs the residency plan; *planned says whether it did.
+struct ResidencyDev;
 cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                                float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0);
+                               cudaStream_t s, bool pdl, int* sched = nullptr, int sched_n = 0,
+                               const ResidencyDev* rd = nullptr, int32_t* map_of = nullptr, bool* planned = nullptr);
 // Prefill-regime router logits (register-tiled fp32 GEMM in the same order).
 cudaError_t launch_route_gemm(const void* x, const float* wr, const float* bias, int T, int H, int E,
                               float* logits, cudaStream_t s);

@@ -13,6 +13,7 @@
 // token alone, whatever the batch.
 #include "common.cuh"
 #include "internal.h"
+#include "residency.cuh"
 #include "topk.cuh"
 
 namespace moe {
@@ -384,9 +385,11 @@ __global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16
                                                                      int32_t* __restrict__ idx, float* __restrict__ w,
                                                                      unsigned int* __restrict__ counters,
                                                                      int fuse_topk, int* status,
-                                                                     int* __restrict__ sched, int sched_n) {
+                                                                     int* __restrict__ sched, int sched_n,
+                                                                     ResidencyDev rd, int32_t* map_of, int res_plan) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
+  __shared__ ResidencyPlanSmem s_plan;
   pdl_trigger();  // first kernel of a forward: the next one may launch (it waits for us)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && blockIdx.y == 0)  // counters of the decode FFN that follows
@@ -451,13 +454,20 @@ __global__ void __launch_bounds__(kRsWarps * 32) route_small_kernel(const uint16
     const int t = t0 + i;
     topk_warp_any(logits + (size_t)t * E, E, K, idx + (size_t)t * K, w + (size_t)t * K);
   }
+  if (res_plan) {
+    // one CTA holds every token (T <= TG): the LRU plan of the spare slots follows the top-k here instead of
+    // in a launch of its own
+    __syncthreads();
+    residency_plan_block(idx, T * K, E, rd, map_of, s_plan);
+  }
   if (threadIdx.x == 0) counters[blockIdx.y] = 0u;
 }
 
 template <int TG>
 static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                              float* logits, int32_t* idx, float* w, unsigned int* counters, int fuse, int* status,
-                             cudaStream_t s, int* sched, int sched_n) {
+                             cudaStream_t s, int* sched, int sched_n, const ResidencyDev* rd = nullptr,
+                             int32_t* map_of = nullptr) {
   const size_t smem = route_small_smem(TG, H);
   cudaError_t err = cudaFuncSetAttribute(route_small_kernel<TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -465,7 +475,7 @@ static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, 
   dim3 grid((E + kRsWarps - 1) / kRsWarps, (T + TG - 1) / TG);
   return launch_ex(route_small_kernel<TG>, grid, dim3(kRsWarps * 32), smem, s, false,
                    static_cast<const uint16_t*>(x), wr, bias, T, H, E, K, logits, idx, w, counters, fuse, status,
-                   sched, sched ? sched_n : 0);
+                   sched, sched ? sched_n : 0, rd ? *rd : ResidencyDev{}, map_of, rd ? 1 : 0);
 }
 
 // T <= 4: logits + fused top-k in one launch; up to 64 tokens: logits, then
@@ -477,7 +487,9 @@ static cudaError_t launch_rs(const void* x, const float* wr, const float* bias, 
 // large for shared memory) go through the direct kernel.
 cudaError_t launch_route_small(const void* x, const float* wr, const float* bias, int T, int H, int E, int K,
                                float* logits, int32_t* idx, float* w, unsigned int* counters, int* status,
-                               cudaStream_t s, bool pdl, int* sched, int sched_n) {
+                               cudaStream_t s, bool pdl, int* sched, int sched_n, const ResidencyDev* rd,
+                               int32_t* map_of, bool* planned) {
+  if (planned) *planned = false;
   if (T <= 0) return cudaSuccess;
   const bool bulk_ok = ((uintptr_t)x % 16 == 0) && ((uintptr_t)wr % 16 == 0) && (H % 8 == 0) &&
                        route_small_smem(8, H) <= 200 * 1024;
@@ -487,9 +499,15 @@ cudaError_t launch_route_small(const void* x, const float* wr, const float* bias
     if (err != cudaSuccess) return err;
     return launch_topk_warp(logits, T, E, K, idx, w, s, false);
   }
-  if (T <= 1) return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
-  if (T <= 2) return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
-  if (T <= 4) return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n);
+  // the fused last CTA runs the residency plan when the caller asks for it (and learns it through *planned)
+  const ResidencyDev* rdp = (T <= 4 && planned) ? rd : nullptr;
+  if (rdp) *planned = true;
+  if (T <= 1)
+    return launch_rs<1>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n, rdp, map_of);
+  if (T <= 2)
+    return launch_rs<2>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n, rdp, map_of);
+  if (T <= 4)
+    return launch_rs<4>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 1, status, s, sched, sched_n, rdp, map_of);
   if (T <= 8) {
     const cudaError_t err = launch_rs<8>(x, wr, bias, T, H, E, K, logits, idx, w, counters, 0, status, s, sched,
                                          sched_n);
