@@ -321,22 +321,43 @@ __global__ void __launch_bounds__(32 * NWT * NWE, 2) route_gemm_kernel(const uin
     __syncthreads();
     if (++buf == kRgStages) buf = 0;
   }
+  // The 32 chain partials of each of the warp's WT x WE outputs go through shared memory (the stage buffers are
+  // free: every copy has landed and the last barrier has passed): row (token i, expert j) holds chain c at
+  // 16-byte chunk (c / 4) ^ (row % 8), so a lane's 16-byte reads of its own row and the other lanes' rows fall
+  // in different banks. Lane l then sums rows l, l + 32, ... by the xor butterfly's tree in registers: offsets
+  // 16, 8, 4, 2, 1, each partial added to its partner, as the shuffles would.
+  static_assert((size_t)NWT * NWE * WT * WE * 32 * 4 <= C::kSmem, "the partials fit the stage buffers");
+  float* red = reinterpret_cast<float*>(sm) + (size_t)warp * WT * WE * 32;
 #pragma unroll
-  for (int m = 0; m < WT / 2; ++m) {
-    const int t = tb + tt0 + 2 * m + half;
+  for (int m = 0; m < WT / 2; ++m)
 #pragma unroll
     for (int j = 0; j < WE; ++j) {
+      const int row = (2 * m + half) * WE + j;
+      const int chunk = (li >> 1) ^ (row & 7);  // chains 2li, 2li+1 sit in chunk li / 2, at (2li) % 4
       float lo, hi;
       unpack2(acc2[m][j], lo, hi);
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) {  // chain offsets 16, 8, 4, 2
-        lo = lo + __shfl_xor_sync(0xffffffffu, lo, o);
-        hi = hi + __shfl_xor_sync(0xffffffffu, hi, o);
-      }
-      const float r = lo + hi;  // chain offset 1
-      const int e = eb + ee0 + j;
-      if (li == 0 && t < T && e < E) logits[(size_t)t * E + e] = bias ? r + bias[e] : r;
+      *reinterpret_cast<float2*>(red + row * 32 + chunk * 4 + ((2 * li) & 3)) = make_float2(lo, hi);
     }
+  __syncwarp();
+#pragma unroll
+  for (int rr = 0; rr < (WT * WE + 31) / 32; ++rr) {
+    const int row = lane + 32 * rr;
+    if (row >= WT * WE) break;
+    float c[32];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 v = *reinterpret_cast<const float4*>(red + row * 32 + (k ^ (row & 7)) * 4);
+      c[4 * k] = v.x;
+      c[4 * k + 1] = v.y;
+      c[4 * k + 2] = v.z;
+      c[4 * k + 3] = v.w;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < o; ++q) c[q] = c[q] + c[q + o];
+    const int t = tb + tt0 + row / WE, e = eb + ee0 + row % WE;
+    if (t < T && e < E) logits[(size_t)t * E + e] = bias ? c[0] + bias[e] : c[0];
   }
 }
 
