@@ -209,8 +209,8 @@ cudaError_t launch_topk_warp(const float* logits, int T, int E, int K, int32_t* 
 // 32-bit load brings x[h], x[h+1] (h = h0 + 32q + 2i) of a token, one 64-bit
 // load the matching pair of Wr[e], and one paired FMA advances both chains.
 // The chains keep the order above (chain c runs h = c, c+32, ... in
-// increasing h), and the xor butterfly's offsets 16 .. 2 become lane offsets
-// 8 .. 1 inside each half, its offset 1 the sum of a lane's two chains. Token
+// increasing h); at the end the 32 chains of each output meet in shared
+// memory and one lane sums them by the xor butterfly's pairwise tree. Token
 // rows are staged 576 bytes apart, so the two halves' rows (even and odd
 // tokens) fall in different banks.
 //   prefill:          WT = 8, WE = 8, 4 x 2 warps (32 tokens x 16 experts; two
