@@ -22,11 +22,6 @@ __device__ __forceinline__ float bf16_lo(uint32_t bits16) { return __uint_as_flo
 
 // Two fp32 values in one 64-bit register, and the paired fused multiply-add
 // (two independent IEEE fmaf with round-to-nearest, one instruction).
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
 __device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
